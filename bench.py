@@ -1,0 +1,405 @@
+"""Decode-step benchmark of libspectra on B200.
+
+One step = one decode step through a stack of attention layers shaped like the
+named model: per layer, spectra_encode_append of the new token (projection +
+quantise + pack + append) followed by spectra_decode_attend over the whole
+latent cache.  Caches and codec factors of all layers (> L2) are resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama|qwen|stress]
+                    [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Metric: cache tokens/s/head = sum over layers of
+batch * context * n_kv_heads per second of step time.  ``roofline`` reports the
+decode-attention launch sequence against the measured HBM copy bandwidth over
+the packed bytes it must read.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+MODEL_LAYERS = {"llama": 32, "qwen": 28, "stress": 32}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "src": "measured"}
+    return dict(FALLBACK_PEAKS, src="fallback")
+
+
+def _workload_name(cfg, layers):
+    return (f"{cfg.name}: {layers} layers x (d_model {cfg.d_model}, {cfg.n_q_heads}q/{cfg.n_kv_heads}kv heads, "
+            f"d_head {cfg.d_head}, groups of {cfg.group}, {cfg.budget_bits} bits/side), "
+            f"batch {cfg.batch} decode at {cfg.cache_len} context")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+def cpu_oracle_sample(cfg, target_s=12.0):
+    import numpy as np
+
+    import oracle
+    from workloads import get_config
+
+    rng = np.random.default_rng(cfg.seed)
+    s2 = np.arange(1, cfg.rank + 1) ** -cfg.spectrum_exp
+    widths = oracle.allocate_widths(s2, cfg.group, cfg.budget_bits, cfg.count_overhead)
+    w1 = [[widths, widths]]
+    P = cfg.page_tokens
+    n_tok = 8192
+    lay = oracle.page_layout(w1, cfg.group, P)
+    pool = np.zeros(lay["page_bytes"] * (n_tok // P), np.uint8)
+    table = np.arange(n_tok // P)[None, :]
+    nk = int(sum(cfg.group for b in widths if b > 0))
+    lat = (rng.standard_normal((n_tok, 2 * nk)) * 0.3).astype(np.float32)
+    oracle.append_tokens(pool, lay["page_bytes"], lay, w1, cfg.group, P, table, np.zeros(1),
+                         np.zeros(n_tok, np.int64), lat, 1)
+    q, _ = np.linalg.qr(rng.standard_normal((cfg.d_head, cfg.d_head)))
+    W_up = [[q[:nk].astype(np.float32), q[:nk].astype(np.float32)]]
+    qs = rng.standard_normal((1, cfg.gq, cfg.d_head)).astype(np.float32)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decode_reference(pool, lay["page_bytes"], lay, cfg.group, P, table, np.array([n_tok]), qs,
+                                W_up, cfg.gq, 1)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= target_s:
+            break
+    value = reps * n_tok / el  # tokens/s/head (one KV head per pass)
+    cores = os.cpu_count() or 1
+    sample = (f"oracle decode of 1 KV head ({cfg.gq} q heads) over {n_tok} of {cfg.cache_len} context tokens "
+              f"of one {cfg.name} layer, {reps} passes in {el:.1f} s")
+    return value, cores, sample
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) < 9:
+                        continue
+                    try:
+                        sm.append(float(p[1]))
+                        mx = float(p[2])
+                    except ValueError:
+                        continue
+                    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+                    for nm, v in zip(names, p[5:9]):
+                        if v.lower().startswith("active"):
+                            reasons.add(nm)
+        except OSError:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.remove(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_gpu(args, rank, world):
+    import numpy as np
+    import torch
+
+    import spectral_transform_coding_b200 as st
+    from spectral_transform_coding_b200.codec import make_config
+    from workloads import get_config
+    from workloads.synthetic import _basis
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = get_config(args.workload)
+    L = args.layers or MODEL_LAYERS[args.workload]
+    B = cfg.batch
+    ctx = cfg.cache_len
+    steps, warm = args.steps, args.warmup
+    P = cfg.page_tokens
+    cap_tokens = ctx + steps + warm + 2
+    max_pages = (cap_tokens + P - 1) // P
+    c = make_config(cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head, cfg.rank, cfg.group,
+                    cfg.budget_bits, cfg.count_overhead, P)
+    gen = torch.Generator(device=dev)
+
+    # activations h = z sqrt(lambda) Q^T with the workload's basis, generated on the GPU
+    basis = _basis(cfg.d_model, cfg.seed)
+    lam = torch.arange(1, cfg.d_model + 1, device=dev, dtype=torch.float32) ** (-cfg.spectrum_exp)
+    q1 = torch.from_numpy(basis[1]).to(dev, torch.float32)
+    q2 = torch.from_numpy(basis[2]).to(dev, torch.float32) if basis[0] == "kron" else None
+
+    def acts(n, seed):
+        gen.manual_seed(seed)
+        y = torch.randn((n, cfg.d_model), generator=gen, device=dev) * lam.sqrt()
+        if q2 is None:
+            h = y @ q1.T
+        else:
+            a, b = q1.shape[0], q2.shape[0]
+            h = torch.einsum("ia,nab,jb->nij", q1, y.view(n, a, b), q2).reshape(n, a * b)
+        if cfg.dist == "student_t":
+            w = torch.distributions.Chi2(torch.tensor(cfg.nu, device=dev)).sample((n,))
+            h = h * torch.sqrt(cfg.nu / w)[:, None]
+        return h.to(torch.bfloat16)
+
+    codecs, caches = [], []
+    kvw = cfg.n_kv_heads * cfg.d_head
+    for l in range(L):
+        gen.manual_seed(1000 * cfg.seed + l)
+        W_K = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+        W_V = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+        codec = st.Codec.calibrate(c, acts(cfg.calib_tokens, 7000 + l), W_K, W_V)
+        del W_K, W_V
+        cache = st.LatentCache(codec, batch=B, max_pages_per_seq=max_pages, device=dev, zero=False)
+        chunk = 8192
+        for b in range(B):
+            for t0 in range(0, ctx, chunk):
+                n = min(chunk, ctx - t0)
+                codec.encode_append(cache, acts(n, 10_000_000 + l * 1000 + b * 97 + t0 // chunk),
+                                    torch.full((n,), b, dtype=torch.int32, device=dev))
+        codec.device_status()
+        codecs.append(codec)
+        caches.append(cache)
+    torch.cuda.synchronize()
+
+    # per-step inputs and workspaces (device-resident)
+    H_new = acts(L * B, 99).view(L, B, cfg.d_model).contiguous()
+    gen.manual_seed(123)
+    Q = (torch.randn((L, B, cfg.n_q_heads, cfg.d_head), generator=gen, device=dev) * 0.5).contiguous()
+    OUT = torch.empty_like(Q)
+    seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
+    ews = [torch.empty(codecs[l].encode_workspace_bytes(B), dtype=torch.uint8, device=dev) for l in range(L)]
+    dws = [torch.empty(codecs[l].decode_workspace_bytes(B, cap_tokens), dtype=torch.uint8, device=dev)
+           for l in range(L)]
+    stream = torch.cuda.Stream(device=dev)
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+
+    def step(record=False):
+        for l in range(L):
+            codecs[l].encode_append(caches[l], H_new[l], seq_ids, workspace=ews[l], stream=stream)
+            if record:
+                ev_dec[l][0].record(stream)
+            codecs[l].decode_attend(caches[l], Q[l], OUT[l], workspace=dws[l], stream=stream)
+            if record:
+                ev_dec[l][1].record(stream)
+
+    # host (pinned) buffers for the end-to-end arm
+    H_host = H_new.cpu().pin_memory()
+    Q_host = Q.cpu().pin_memory()
+    OUT_host = torch.empty(OUT.shape, dtype=OUT.dtype).pin_memory()
+
+    def step_e2e():
+        H_new.copy_(H_host, non_blocking=True)
+        Q.copy_(Q_host, non_blocking=True)
+        step()
+        OUT_host.copy_(OUT, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            step()
+    torch.cuda.synchronize()
+    len0 = int(caches[0].lengths.float().mean().item())
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    # ---- device-resident timed region (K steps) ----
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dec_ms = []
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for k in range(steps):
+                step(record=True)
+                if k == steps - 1:
+                    pass
+            t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    # decode-attention launch durations (events recorded on the launching stream)
+    with torch.cuda.stream(stream):
+        pass
+    for l in range(L):
+        dec_ms.append(ev_dec[l][0].elapsed_time(ev_dec[l][1]))
+    total_ms = t_start.elapsed_time(t_end)
+    clk = clocks.summary()
+
+    # ---- end-to-end arm (host buffers, copies inside the timed region) ----
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ksteps_e2e = max(3, steps // 4)
+    with torch.cuda.stream(stream):
+        step_e2e()
+    torch.cuda.synchronize()
+    barrier()
+    with torch.cuda.stream(stream):
+        e_start.record(stream)
+        for _ in range(ksteps_e2e):
+            step_e2e()
+        e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / ksteps_e2e
+
+    codecs[0].device_status(stream)
+    ms_per_step = total_ms / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_per_step, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step, e2e_ms = float(t[0]), float(t[1])
+    mean_ctx = len0 + (steps + 1) / 2.0
+    tok_per_step = L * B * mean_ctx * cfg.n_kv_heads
+    value = tok_per_step / (ms_per_step / 1e3) * world
+    e2e_value = tok_per_step / (e2e_ms / 1e3) * world
+
+    # roofline: packed bytes the decode reads per layer
+    bytes_per_tok_all_heads = codecs[0].page_bytes / P
+    dec_bytes = B * mean_ctx * bytes_per_tok_all_heads
+    dec_avg_ms = statistics.mean(dec_ms)
+    peaks = _peaks()
+    achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
+    launches_per_layer = 3 + 3  # encode: projection, append plan, quantise/pack; decode: fold, split, combine
+    h2d = H_new.numel() * 2 + Q.numel() * 4
+    d2h = OUT.numel() * 4
+
+    result = {
+        "metric": "latent-KV decode attention: cache tokens/s/head",
+        "value": value,
+        "unit": "tokens/s/head",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warm,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u8 codes, fp16 scale/zero, fp32 accumulate",
+        "data": "synthetic (seeded power-law activations, random bf16 weights; calibrated per layer)",
+        "config": {
+            "workload": _workload_name(cfg, L),
+            "layers": L, "batch": B, "context_start": len0, "n_kv_heads": cfg.n_kv_heads,
+            "bytes_per_token_per_layer": bytes_per_tok_all_heads,
+            "l2": "inputs larger than L2 (caches + factors of all layers)",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "kernel": "decode attention launch sequence (fold, split-K latent flash-decode, combine)",
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "peak_src": peaks["src"], "avg_launch_us": dec_avg_ms * 1e3,
+            "algorithmic_bytes_per_launch": dec_bytes,
+        },
+        "e2e": {"value": e2e_value, "unit": "tokens/s/head", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_layer * L * steps,
+        "clocks": clk,
+    }
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama", choices=sorted(MODEL_LAYERS))
+    ap.add_argument("--layers", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    from workloads import get_config
+    cfg = get_config(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        value, cores, sample = cpu_oracle_sample(cfg, target_s=max(3.0, min(30.0, 2.0 * args.steps)))
+        L = args.layers or MODEL_LAYERS[args.workload]
+        out = {
+            "impl": "reference", "metric": "latent-KV decode attention: cache tokens/s/head", "value": value,
+            "unit": "tokens/s/head", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": _workload_name(cfg, L)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s/head", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s/head", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(out), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(cfg)
+    res = run_gpu(args, rank, world)
+    if rank == 0:
+        if cpu is not None:
+            res["cpu_baseline"] = {"value": cpu[0], "unit": "tokens/s/head", "cores": cpu[1], "kind": "oracle",
+                                   "sample": cpu[2]}
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

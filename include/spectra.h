@@ -1,0 +1,296 @@
+/*
+ * libspectra -- C ABI of a SPECTRA-style spectral latent KV-cache codec for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes follows "SPECTRA: Pushing the KV Cache Beyond the 2-Bit Cliff
+ * via Spectral Transform Coding" (technical summary):
+ *   - "SPECTRA pipeline", stage 1 (G-weighted transform): the activation Gram
+ *     G = E[h^T h] (observation 3) whitens W_K / W_V; the SVD of G^{1/2} W gives
+ *     an energy-ordered, second-moment-orthogonal latent basis; W_down = W V_r
+ *     projects a token down, W_up = V_r^T rebuilds it;
+ *   - stage 2 (rate-distortion quantisation): reverse water-filling on the
+ *     latent second moments decides bits; adjacent coordinates share one width
+ *     ("grouping"); zero bits drop a group (observation 2);
+ *   - stage 3 (system integration): every new token is projected down,
+ *     quantised per token and appended to an append-only latent cache;
+ *   - "Significance and claims": attention computed directly in the latent
+ *     space (the query is folded with W_up, W_up^V is applied once per head).
+ *
+ * Conventions
+ *   - Every entry point returns a spectra_status and never throws.  On failure,
+ *     spectra_last_error() returns a thread-local message.
+ *   - "device" pointers are CUDA global-memory addresses on the current device;
+ *     "host" pointers are ordinary CPU memory.  `stream` is a cudaStream_t passed
+ *     as void* (NULL = legacy default stream).  Device-side work is enqueued on
+ *     `stream` and the call returns without synchronising, except where stated.
+ *   - The caller owns every large device buffer (activations, queries,
+ *     outputs, the cache pool, page table, lengths, workspaces); sizes come
+ *     from the *_bytes helpers.  A codec owns only its small device tables and
+ *     factors and is released by spectra_codec_destroy.
+ *   - Conditions found on the device (capacity overflow, unsorted seq_ids, a
+ *     bounded wait that gave up) set the codec's device error word; read and
+ *     clear it with spectra_device_status.
+ *   - No function here calls into a CPU fallback: without a usable CUDA device
+ *     the device entry points fail with SPECTRA_ERR_CUDA.
+ *
+ * Canonical page layout (this library's definition; the pages only fix that
+ * codes are appended per token with one width per group):
+ *   A page holds P = page_tokens tokens of one sequence for every KV head.
+ *   page = head sections a = 0..n_kv_heads-1; head section = K side then V side;
+ *   side section = for each group j with b_j > 0, ascending:
+ *       b_j bit-planes (plane p = bit p of every code, p = 0 first), each
+ *       P*g/8 bytes, then P/2 records of 8 bytes:
+ *       fp16 {s[2u], s[2u+1], z[2u], z[2u+1]} (little-endian).
+ *   A bit-plane is a run of 256-bit blocks (8 little-endian uint32 words), one
+ *   per 256/g consecutive tokens.  Entry (token tau of the block, coordinate k
+ *   of the group) sits at word `word`, bit `4*slot + t4`, where
+ *     g = 16: K side row = tau/2 (tau even) or 8 + tau/2 (tau odd), col = k;
+ *             V side row = k, col = tau;
+ *             word = row % 8, t4 = (col % 8)/2,
+ *             slot = row/8 + 2*(col/8) + 4*(col % 2);
+ *     g = 8 (32-token blocks; mi = tau/16, tl = tau%16):
+ *             K side row from tl as above, word = row % 8, t4 = k/2,
+ *                    slot = row/8 + 2*mi + 4*(k % 2);
+ *             V side word = k, t4 = (tl % 8)/2,
+ *                    slot = mi + 2*(tl/8) + 4*(tl % 2).
+ *   (This places, after one rotate per plane, each lane's codes of an
+ *   mma.sync A fragment into 4-bit fields.)  A page therefore takes exactly
+ *   P * sum over kept groups of (g*b_j + 32)/8 bytes; all offsets are multiples
+ *   of 16 bytes.
+ *
+ * Quantiser (per token, per kept group of g fp32 latents, every step one IEEE
+ * fp32 operation): s = fp16_rn(sat((max - min) / (2^b - 1))), z = fp16_rn(sat(min)),
+ * code = clamp(rint_half_even((x - z) / s), 0, 2^b - 1); s == 0 gives codes 0;
+ * sat clamps to +-65504.  Dequantised value: code*s + z.
+ */
+#ifndef SPECTRA_H
+#define SPECTRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPECTRA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SPECTRA_API __attribute__((visibility("default")))
+#else
+#define SPECTRA_API
+#endif
+
+typedef enum spectra_status {
+  SPECTRA_OK = 0,
+  SPECTRA_ERR_INVALID = 1,     /* bad argument: null pointer, size, alignment or shape */
+  SPECTRA_ERR_CUDA = 2,        /* a CUDA runtime or driver call failed */
+  SPECTRA_ERR_CAPACITY = 3,    /* page table / pool too small; nothing was written */
+  SPECTRA_ERR_NUMERIC = 4,     /* non-finite data, Gram not positive definite, eigen failure */
+  SPECTRA_ERR_UNSUPPORTED = 5, /* a shape outside what the kernels implement */
+  SPECTRA_ERR_TIMEOUT = 6,     /* a bounded device wait gave up; the kernel returned early */
+  SPECTRA_ERR_ORDER = 7        /* seq_ids of an append were not non-decreasing; nothing written */
+} spectra_status;
+
+typedef enum spectra_dtype { SPECTRA_F32 = 0, SPECTRA_BF16 = 1 } spectra_dtype;
+
+/* Shapes and budget of one attention layer's codec. */
+typedef struct spectra_config {
+  int32_t d_model;        /* width of the layer input h */
+  int32_t n_q_heads;      /* query heads */
+  int32_t n_kv_heads;     /* KV heads; n_q_heads % n_kv_heads == 0, ratio (GQA) <= 8 */
+  int32_t d_head;         /* head dimension (<= 256) */
+  int32_t rank;           /* latent coordinates kept before allocation, <= d_head, multiple of group */
+  int32_t group;          /* coordinates per group: 8 or 16 */
+  int32_t budget_bits;    /* bits per token, per KV head, per side (K or V) */
+  int32_t count_overhead; /* nonzero: a kept group costs group*b + 32 bits (fp16 s and z) */
+  int32_t page_tokens;    /* P, tokens per cache page: multiple of 32, 32..1024 */
+} spectra_config;
+
+typedef struct spectra_codec spectra_codec; /* opaque, library-owned */
+
+/* A paged, append-only latent cache.  All pointers are device memory owned by
+ * the caller.  Page i occupies pool[i*page_bytes, (i+1)*page_bytes); the pool
+ * must be 16-byte aligned.  page_table[b*max_pages_per_seq + k] is the page that
+ * holds tokens [k*P, (k+1)*P) of sequence b.  lengths[b] is the number of
+ * tokens of sequence b in the cache; encode advances it. */
+typedef struct spectra_cache {
+  void* pool;
+  int64_t n_pages;
+  const int32_t* page_table;
+  int32_t* lengths;
+  int32_t batch;
+  int32_t max_pages_per_seq;
+} spectra_cache;
+
+/* Summary of a codec. */
+typedef struct spectra_codec_info {
+  spectra_config config;
+  int32_t n_groups;          /* rank / group */
+  int32_t n_eff;             /* latent columns of W_down: kept coordinates over all heads and sides */
+  int64_t page_bytes;        /* bytes per cache page */
+  int64_t bits_per_token;    /* sum over heads and sides of the spent bits (incl. overhead) */
+  int32_t max_kept;          /* largest kept-coordinate count of one (head, side) */
+} spectra_codec_info;
+
+/* ------------------------------------------------------------------------- */
+/* Calibration (once per layer, off the hot path)                             */
+/* ------------------------------------------------------------------------- */
+
+/* spectra_calibrate -- SPECTRA pipeline stages 1-2.
+ *   H        device [n_tokens][d_model], dtype `dtype`: calibration activations.
+ *   W_K, W_V device [d_model][n_kv_heads*d_head], dtype `dtype`: head a uses
+ *            columns [a*d_head, (a+1)*d_head).
+ * Accumulates G = sum_t h_t^T h_t on the GPU (tcgen05 tensor cores for bf16),
+ * forms M = W^T G W per head and side on the GPU, and on the host (fp64)
+ * eigen-decomposes M (Jacobi), sorts by decreasing eigenvalue, fixes signs
+ * (largest-magnitude entry of each vector positive), allocates group widths
+ * (spectra_allocate_widths) and folds W_down = W V_r (bf16) and W_up = V_r^T
+ * (fp32).  Synchronises `stream`.  Allocates and frees its own temporary device
+ * memory (O(d_model^2) bytes).  On success *out receives a new codec. */
+SPECTRA_API spectra_status spectra_calibrate(const spectra_config* cfg, int32_t dtype, const void* H,
+                                 int64_t n_tokens, const void* W_K, const void* W_V,
+                                 spectra_codec** out, void* stream);
+
+/* spectra_codec_create -- build a codec from given factors (no calibration).
+ *   widths   host [n_kv_heads][2][rank/group], each in {0,1,2,3,4,8}.
+ *   W_down   host fp32 [d_model][n_eff]; columns head-major, K then V, kept
+ *            coordinates ascending (n_eff = number of kept coordinates over all
+ *            heads and sides); rounded to bf16 (nearest, ties to even).
+ *   W_up     host fp32 [n_kv_heads][2][rank][d_head] (rows of V_r^T; rows of
+ *            dropped groups are ignored).
+ *   sigma2   host [n_kv_heads][2][rank] or NULL (stored for info/serialisation). */
+SPECTRA_API spectra_status spectra_codec_create(const spectra_config* cfg, const int32_t* widths,
+                                    const float* W_down, const float* W_up,
+                                    const double* sigma2, spectra_codec** out);
+
+SPECTRA_API void spectra_codec_destroy(spectra_codec* codec);
+
+SPECTRA_API spectra_status spectra_codec_get_info(const spectra_codec* codec, spectra_codec_info* out);
+
+/* Host copies of the codec state.  Any output pointer may be NULL.
+ *   widths [n_kv_heads][2][n_groups]; sigma2 [n_kv_heads][2][rank];
+ *   theta [n_kv_heads][2] (continuous water level for the spent payload bits);
+ *   W_down [d_model][n_eff] (the bf16 values as fp32); W_up [n_kv_heads][2][rank][d_head]. */
+SPECTRA_API spectra_status spectra_codec_get_state(const spectra_codec* codec, int32_t* widths,
+                                       double* sigma2, double* theta, float* W_down,
+                                       float* W_up);
+
+/* Versioned binary blob of the codec (config, widths, sigma2, theta, W_down
+ * bf16, W_up fp32).  Call with buf == NULL to get the size in *bytes. */
+SPECTRA_API spectra_status spectra_codec_serialize(const spectra_codec* codec, void* buf, size_t* bytes);
+SPECTRA_API spectra_status spectra_codec_deserialize(const void* buf, size_t bytes, spectra_codec** out);
+
+/* spectra_wo_correction -- SPECTRA pipeline stage 1, "Refinement": a closed-form,
+ * training-free correction of W_O for the rank truncation.  Reading used here
+ * (the pages give no formula): treat the calibration tokens as one causal
+ * sequence; for each q head h (KV head a = h / (n_q/n_kv)) let O_h be the
+ * attention output with exact K, V and Oh_h the one with the rank-truncated,
+ * unquantised K, V (kept coordinates only); M_h = (Oh^T Oh + eps I)^-1 Oh^T O with
+ * eps = 1e-8 tr(Oh^T Oh)/d_head, and W_O' = blockdiag(M_h) W_O.
+ *   H device [n_tokens][d_model]; W_Q device [d_model][n_q_heads*d_head];
+ *   W_K, W_V as for calibrate; W_O device [n_q_heads*d_head][d_model];
+ *   W_O_out device fp32 [n_q_heads*d_head][d_model].  All inputs in `dtype`.
+ * Synchronises `stream`; n_tokens <= 4096. */
+SPECTRA_API spectra_status spectra_wo_correction(const spectra_codec* codec, int32_t dtype, const void* H,
+                                     int64_t n_tokens, const void* W_Q, const void* W_K,
+                                     const void* W_V, const void* W_O, float* W_O_out,
+                                     void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Hot path                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* Workspace bytes for spectra_encode_append with up to max_tokens tokens. */
+SPECTRA_API spectra_status spectra_encode_workspace_bytes(const spectra_codec* codec, int64_t max_tokens,
+                                              size_t* bytes);
+/* Workspace bytes for spectra_decode_attend with `batch` sequences of up to
+ * max_len tokens. */
+SPECTRA_API spectra_status spectra_decode_workspace_bytes(const spectra_codec* codec, int32_t batch,
+                                              int64_t max_len, size_t* bytes);
+
+/* spectra_project -- stage 3 "projected down": latents = H W_down.
+ *   H device bf16 [T][d_model]; latents device fp32 [T][n_eff].
+ * bf16 x bf16 products accumulated in fp32: tcgen05 tensor cores for T >= 64,
+ * a bandwidth-bound CUDA-core kernel for smaller T. */
+SPECTRA_API spectra_status spectra_project(const spectra_codec* codec, const void* H, int64_t T,
+                               float* latents, void* stream);
+
+/* spectra_quantize_append -- stage 3 "quantised per token, appended": quantise
+ * fp32 latents (layout of spectra_project's output) and write them into the
+ * cache at lengths[seq]; then advance lengths.
+ *   latents device fp32 [T][n_eff]; seq_ids device int32 [T], non-decreasing,
+ *   each in [0, batch).  Token i goes to position lengths[seq_ids[i]] + (i minus
+ *   the first index of its sequence in this call).  If any token would not fit
+ *   (position >= max_pages_per_seq*P, or a needed page id outside [0, n_pages))
+ *   or seq_ids are not sorted, nothing is written and the device error word is
+ *   set (SPECTRA_ERR_CAPACITY / SPECTRA_ERR_ORDER).  workspace: device,
+ *   >= spectra_encode_workspace_bytes(T), 256-byte aligned (per-token positions). */
+SPECTRA_API spectra_status spectra_quantize_append(const spectra_codec* codec, const spectra_cache* cache,
+                                       const float* latents, const int32_t* seq_ids, int64_t T,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* spectra_encode_append -- spectra_project followed by spectra_quantize_append.
+ *   H device bf16 [T][d_model]; seq_ids as above; latents_out device fp32
+ *   [T][n_eff] or NULL (when given, the latents are kept there);
+ *   workspace device, >= spectra_encode_workspace_bytes(T), 256-byte aligned. */
+SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, const spectra_cache* cache,
+                                     const void* H, const int32_t* seq_ids, int64_t T,
+                                     float* latents_out, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* spectra_decode_attend -- one decode step of attention for every sequence of
+ * the cache, in the latent space: q_lat = q W_up^K^T, scores against the
+ * dequantised latent keys of all lengths[b] tokens, exact (online) softmax,
+ * sum_t p_t c_V,t, then W_up^V once per head.  Split-K over the context; no
+ * masking beyond lengths[b].
+ *   q   device fp32 [batch][n_q_heads][d_head]
+ *   out device fp32 [batch][n_q_heads][d_head] (attention output before W_O)
+ *   workspace device, >= spectra_decode_workspace_bytes, 256-byte aligned. */
+SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, const spectra_cache* cache,
+                                     const float* q, float* out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the codec's device error word.
+ * Returns the recorded device-side status (SPECTRA_OK if none). */
+SPECTRA_API spectra_status spectra_device_status(const spectra_codec* codec, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Host-only helpers (no GPU needed)                                          */
+/* ------------------------------------------------------------------------- */
+
+/* Grouped widths for one (head, side): b_j in {0,1,2,3,4,8} minimising
+ * sum_j S_j 4^-b_j (S_j = sum of sigma2 over group j, summed in ascending order;
+ * b = 0 leaves S_j) subject to sum_j cost(b_j) <= budget_bits, cost(b) =
+ * group*b (+32 with count_overhead) for b > 0.  Exact backward dynamic programme
+ * over groups; ties go to the smaller width.  This is the discrete, grouped form
+ * of reverse water-filling (stage 2).  widths_out [rank/group]; distortion_out
+ * may be NULL. */
+SPECTRA_API spectra_status spectra_allocate_widths(const double* sigma2, int32_t rank, int32_t group,
+                                       int32_t budget_bits, int32_t count_overhead,
+                                       int32_t* widths_out, double* distortion_out);
+
+/* Continuous reverse water-filling: theta with sum_i max(0, 1/2 log2(sigma2_i/theta))
+ * = rate_bits; rates_out [n] (may be NULL). */
+SPECTRA_API spectra_status spectra_water_fill(const double* sigma2, int32_t n, double rate_bits,
+                                  double* theta_out, double* rates_out);
+
+/* Symmetric eigen-decomposition (cyclic Jacobi, fp64) of the row-major n x n
+ * matrix M (n <= 512): eigenvalues decreasing, eigenvectors as columns of the
+ * row-major n x n `vecs`, each with its largest-magnitude entry positive. */
+SPECTRA_API spectra_status spectra_sym_eigen(const double* M, int32_t n, double* vals, double* vecs);
+
+/* Page size and group placement for given widths ([n_kv_heads][2][rank/group]).
+ * offsets (may be NULL) receives, per (head, side, group), the byte offset of
+ * the group's first bit-plane in the page (-1 for dropped groups), followed by
+ * the same count of record offsets. */
+SPECTRA_API spectra_status spectra_page_layout(const spectra_config* cfg, const int32_t* widths,
+                                   int64_t* page_bytes, int64_t* offsets);
+
+SPECTRA_API const char* spectra_last_error(void);
+SPECTRA_API int32_t spectra_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPECTRA_H */

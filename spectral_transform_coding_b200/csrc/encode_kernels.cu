@@ -1,0 +1,316 @@
+// Encode side of libspectra: "tokens are projected down, quantised per token and
+// appended to the latent cache" (SPECTRA technical summary, "SPECTRA pipeline",
+// stage 3), with groups of adjacent latent coordinates sharing one width (stage 2,
+// "grouping").
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace spectra {
+
+// ---------------------------------------------------------------------------
+// latents[t][n] = sum_k H[t][k] * W_down[k][n]   for small T (decode steps).
+// W_down is stored transposed (wt[n][k], bf16); each warp owns 4 columns and
+// streams their rows once with 16-byte loads; H rows (small) come from L2.
+// bf16 x bf16 products are exact in fp32; accumulation is fp32.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kGemvCols = 4;   // columns per warp
+constexpr int kGemvRows = 8;   // H rows per pass
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float f[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+}  // namespace
+
+__global__ void __launch_bounds__(256) project_gemv_kernel(const uint16_t* __restrict__ wt,
+                                                           const uint16_t* __restrict__ H, int T,
+                                                           int d_model, int n_eff,
+                                                           float* __restrict__ C, int64_t ldc) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = warp * kGemvCols;
+  if (n0 >= n_eff) return;
+  for (int t0 = 0; t0 < T; t0 += kGemvRows) {
+    float acc[kGemvCols][kGemvRows];
+#pragma unroll
+    for (int c = 0; c < kGemvCols; ++c)
+#pragma unroll
+      for (int r = 0; r < kGemvRows; ++r) acc[c][r] = 0.f;
+    for (int k = lane * 8; k < d_model; k += 256) {
+      float w[kGemvCols][8];
+#pragma unroll
+      for (int c = 0; c < kGemvCols; ++c) {
+        const int n = min(n0 + c, n_eff - 1);
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(wt + (size_t)n * d_model + k));
+        bf16x8_to_f32(v, w[c]);
+      }
+#pragma unroll
+      for (int r = 0; r < kGemvRows; ++r) {
+        if (t0 + r < T) {
+          float h[8];
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(H + (size_t)(t0 + r) * d_model + k));
+          bf16x8_to_f32(v, h);
+#pragma unroll
+          for (int c = 0; c < kGemvCols; ++c)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[c][r] = fmaf(w[c][e], h[e], acc[c][r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < kGemvCols; ++c)
+#pragma unroll
+      for (int r = 0; r < kGemvRows; ++r) {
+        float v = acc[c][r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && n0 + c < n_eff && t0 + r < T) C[(size_t)(t0 + r) * ldc + n0 + c] = v;
+      }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Append planner (one block): checks seq_ids are non-decreasing and in range,
+// gives every token its cache position lengths[s] + (i - first index of s),
+// checks capacity and page ids, and only if everything fits writes the positions,
+// advances lengths and raises ok_flag.  Otherwise nothing is written and the
+// codec's error word records SPECTRA_ERR_ORDER or SPECTRA_ERR_CAPACITY.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) append_plan_kernel(
+    const int32_t* __restrict__ seq_ids, int T, int batch, int32_t* __restrict__ lengths,
+    const int32_t* __restrict__ page_table, int max_pages, int64_t n_pool_pages, int P,
+    int32_t* __restrict__ pos_out, int32_t* __restrict__ ok_flag, int32_t* __restrict__ err) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+    const int s = seq_ids[i];
+    if (s < 0 || s >= batch || (i > 0 && seq_ids[i - 1] > s)) atomicMax(&bad, (int)SPECTRA_ERR_ORDER);
+  }
+  __syncthreads();
+  if (bad == 0) {
+    for (int i = threadIdx.x; i < T; i += blockDim.x) {
+      const int s = seq_ids[i];
+      int lo = 0, hi = i;  // first index with seq_ids[idx] == s (array is sorted)
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (seq_ids[mid] < s) lo = mid + 1;
+        else hi = mid;
+      }
+      const int64_t pos = (int64_t)lengths[s] + (i - lo);
+      if (pos < 0 || pos >= (int64_t)max_pages * P) {
+        atomicMax(&bad, (int)SPECTRA_ERR_CAPACITY);
+      } else {
+        const int pid = page_table[(size_t)s * max_pages + pos / P];
+        if (pid < 0 || pid >= n_pool_pages) atomicMax(&bad, (int)SPECTRA_ERR_CAPACITY);
+      }
+      pos_out[i] = (int32_t)pos;
+    }
+  }
+  __syncthreads();
+  if (bad == 0) {
+    for (int i = threadIdx.x; i < T; i += blockDim.x)
+      if (i == T - 1 || seq_ids[i + 1] != seq_ids[i]) lengths[seq_ids[i]] = pos_out[i] + 1;
+  }
+  if (threadIdx.x == 0) {
+    *ok_flag = bad ? 0 : 1;
+    if (bad) device_error(err, bad);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Quantise + pack + append.  Block (4 warps) = one chunk of 256/G input tokens
+// for one (head, side); warps take the kept groups in turn.  For G = 16 a warp
+// quantises two groups at once (lanes 0-15 and 16-31, one token per lane); for
+// G = 8 one group with one token per lane.
+//
+// Per token and group (every step one IEEE fp32 operation, no contraction):
+//   s = fp16(sat((max - min) / (2^b - 1))), z = fp16(sat(min)),
+//   code = clamp(rint((x - z) / s), 0, 2^b - 1), s == 0 -> 0.
+// Bits go to the page's bit-planes at the canonical (word, bit) addresses; the
+// token's bits are cleared then set with atomics, so tokens of one 256-bit block
+// written by different blocks of this grid (or by different calls) never race.
+// ---------------------------------------------------------------------------
+namespace {
+
+__device__ __forceinline__ float sat16(float x) { return fminf(fmaxf(x, -65504.f), 65504.f); }
+
+template <int G>
+__device__ __forceinline__ void k_side_addr(int tb, int k, int* word, int* bit) {
+  if (G == 16) {
+    const int row = (tb & 1) ? 8 + (tb >> 1) : (tb >> 1);
+    const int slot = (row >> 3) + 2 * (k >> 3) + 4 * (k & 1);
+    *word = row & 7;
+    *bit = 4 * slot + ((k & 7) >> 1);
+  } else {
+    const int mi = tb >> 4, tl = tb & 15;
+    const int row = (tl & 1) ? 8 + (tl >> 1) : (tl >> 1);
+    const int slot = (row >> 3) + 2 * mi + 4 * (k & 1);
+    *word = row & 7;
+    *bit = 4 * slot + (k >> 1);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void v_side_addr(int tb, int k, int* word, int* bit) {
+  if (G == 16) {
+    const int slot = (k >> 3) + 2 * (tb >> 3) + 4 * (tb & 1);
+    *word = k & 7;
+    *bit = 4 * slot + ((tb & 7) >> 1);
+  } else {
+    const int mi = tb >> 4, tl = tb & 15;
+    const int slot = mi + 2 * (tl >> 3) + 4 * (tl & 1);
+    *word = k;
+    *bit = 4 * slot + ((tl & 7) >> 1);
+  }
+}
+
+}  // namespace
+
+template <int G>
+__global__ void __launch_bounds__(128) quantize_append_kernel(
+    const CodecDev* __restrict__ cd, const float* __restrict__ C, int64_t ldc,
+    const int32_t* __restrict__ seq_ids, const int32_t* __restrict__ pos,
+    const int32_t* __restrict__ ok_flag, int T, uint8_t* __restrict__ pool,
+    const int32_t* __restrict__ page_table, int max_pages) {
+  constexpr int TB = 256 / G;               // tokens per 256-bit block
+  constexpr int LANES_PER_TOKENSET = TB;    // 16 or 32
+  constexpr int GROUPS_PER_WARP = 32 / LANES_PER_TOKENSET;
+  if (*ok_flag == 0) return;
+  const int a = blockIdx.y >> 1, side = blockIdx.y & 1;
+  const SideDev& sd = cd->head[a].side[side];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * TB + (lane % TB);
+  if (i >= T) return;
+  const int P = cd->P;
+  const int p_tok = pos[i];
+  const int seq = seq_ids[i];
+  const int pid = page_table[(size_t)seq * max_pages + p_tok / P];
+  uint8_t* page = pool + (size_t)pid * (size_t)cd->page_bytes;
+  const int tau = p_tok % P;
+  const int blk = tau / TB, tb = tau % TB;
+  const float* crow = C + (size_t)i * ldc + sd.c_col0;
+  const int plane_stride = P * G / 8;
+  const int n_groups = sd.n_groups;
+  for (int j = warp * GROUPS_PER_WARP + lane / LANES_PER_TOKENSET; j < n_groups;
+       j += 4 * GROUPS_PER_WARP) {
+    const GroupDev gd = sd.grp[j];
+    const int b = gd.b;
+    float x[G];
+#pragma unroll
+    for (int q = 0; q < G / 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4*>(crow + gd.col + 4 * q);
+      x[4 * q] = v.x;
+      x[4 * q + 1] = v.y;
+      x[4 * q + 2] = v.z;
+      x[4 * q + 3] = v.w;
+    }
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int k = 1; k < G; ++k) {
+      mn = fminf(mn, x[k]);
+      mx = fmaxf(mx, x[k]);
+    }
+    const float levels = (float)((1 << b) - 1);
+    const __half s_h = __float2half_rn(sat16(__fdiv_rn(__fsub_rn(mx, mn), levels)));
+    const __half z_h = __float2half_rn(sat16(mn));
+    const float sf = __half2float(s_h), zf = __half2float(z_h);
+    uint32_t code[G];
+#pragma unroll
+    for (int k = 0; k < G; ++k) {
+      float c = 0.f;
+      if (sf > 0.f) {
+        const float t = __fdiv_rn(__fsub_rn(x[k], zf), sf);
+        c = fminf(fmaxf(rintf(t), 0.f), levels);
+      }
+      code[k] = (uint32_t)c;
+    }
+    uint32_t* plane0 = reinterpret_cast<uint32_t*>(page + gd.plane_off + blk * 32);
+    if (side == 0) {
+      int word = 0, bit;
+      uint32_t mask = 0;
+#pragma unroll
+      for (int k = 0; k < G; ++k) {
+        k_side_addr<G>(tb, k, &word, &bit);
+        mask |= 1u << bit;
+      }
+      for (int p = 0; p < b; ++p) {
+        uint32_t val = 0;
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+          k_side_addr<G>(tb, k, &word, &bit);
+          val |= ((code[k] >> p) & 1u) << bit;
+        }
+        uint32_t* w = plane0 + p * (plane_stride / 4) + word;
+        atomicAnd(w, ~mask);
+        atomicOr(w, val);
+      }
+    } else {
+      for (int p = 0; p < b; ++p) {
+        uint32_t m8[8], v8[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) m8[w] = v8[w] = 0;
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+          int word, bit;
+          v_side_addr<G>(tb, k, &word, &bit);
+          m8[word] |= 1u << bit;
+          v8[word] |= ((code[k] >> p) & 1u) << bit;
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          uint32_t* wp = plane0 + p * (plane_stride / 4) + w;
+          atomicAnd(wp, ~m8[w]);
+          atomicOr(wp, v8[w]);
+        }
+      }
+    }
+    __half* rec = reinterpret_cast<__half*>(page + gd.sz_off + 8 * (tau >> 1));
+    rec[tau & 1] = s_h;
+    rec[2 + (tau & 1)] = z_h;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_project_gemv(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
+                                float* C, int64_t ldc, cudaStream_t st) {
+  const int warps = (h.n_eff + kGemvCols - 1) / kGemvCols;
+  const int blocks = (warps * 32 + 255) / 256;
+  project_gemv_kernel<<<blocks, 256, 0, st>>>(wt, H, T, h.d_model, h.n_eff, C, ldc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_plan(const int32_t* seq_ids, int T, const spectra_cache& cache, int P,
+                               int32_t* pos, int32_t* ok_flag, int32_t* err, cudaStream_t st) {
+  append_plan_kernel<<<1, 1024, 0, st>>>(seq_ids, T, cache.batch, cache.lengths, cache.page_table,
+                                         cache.max_pages_per_seq, cache.n_pages, P, pos, ok_flag, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const float* C, int64_t ldc,
+                                   const int32_t* seq_ids, const int32_t* pos, const int32_t* ok_flag,
+                                   int T, const spectra_cache& cache, cudaStream_t st) {
+  const int tb = 256 / h.group;
+  dim3 grid((T + tb - 1) / tb, h.n_kv * 2);
+  if (h.group == 16)
+    quantize_append_kernel<16><<<grid, 128, 0, st>>>(d, C, ldc, seq_ids, pos, ok_flag, T,
+                                                     (uint8_t*)cache.pool, cache.page_table,
+                                                     cache.max_pages_per_seq);
+  else
+    quantize_append_kernel<8><<<grid, 128, 0, st>>>(d, C, ldc, seq_ids, pos, ok_flag, T,
+                                                    (uint8_t*)cache.pool, cache.page_table,
+                                                    cache.max_pages_per_seq);
+  return cudaGetLastError();
+}
+
+}  // namespace spectra

@@ -1,0 +1,55 @@
+// Kernel launchers of libspectra (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "spectra_internal.h"
+
+namespace spectra {
+
+// encode_kernels.cu
+cudaError_t launch_project_gemv(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
+                                float* C, int64_t ldc, cudaStream_t st);
+cudaError_t launch_append_plan(const int32_t* seq_ids, int T, const spectra_cache& cache, int P,
+                               int32_t* pos, int32_t* ok_flag, int32_t* err, cudaStream_t st);
+cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const float* C, int64_t ldc,
+                                   const int32_t* seq_ids, const int32_t* pos, const int32_t* ok_flag,
+                                   int T, const spectra_cache& cache, cudaStream_t st);
+
+// decode_kernels.cu
+struct DecodePlan {
+  int n_split;       // context splits per (sequence, KV head)
+  int stages;        // bulk-copy stages per warp
+  int stage_bytes;   // bytes per stage (largest head section, rounded to 16)
+  int smem_bytes;    // dynamic shared memory per CTA
+  size_t qlat_off, qsum_off, part_off, ws_bytes;  // workspace carve-up
+  int part_stride;   // floats per partial record
+};
+DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq);
+cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,
+                          const float* q, float* out, void* ws, const DecodePlan& plan,
+                          cudaStream_t st);
+
+// gemm_sm100.cu (tcgen05)
+cudaError_t launch_project_tcgen05(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
+                                   float* C, int64_t ldc, cudaStream_t st);
+cudaError_t launch_gram_tcgen05(const uint16_t* H, int64_t n_tokens, int d_model, float* G,
+                                cudaStream_t st);
+
+// calib_kernels.cu
+cudaError_t launch_gram_f32(const float* H, int64_t n_tokens, int d_model, float* G, cudaStream_t st);
+// C[M][N] = sum_k A[k][m] * B[k][n] (A^T B), A and B row-major with leading dims lda, ldb;
+// `a_bf16`/`b_bf16` select bf16 inputs (else fp32).  fp32 accumulate.
+cudaError_t launch_gemm_tn_f32(const void* A, bool a_bf16, int64_t lda, const void* B, bool b_bf16,
+                               int64_t ldb, float* C, int64_t ldc, int M, int N, int K,
+                               cudaStream_t st);
+// C[M][N] = A[M][K] B[K][N], row-major, fp32 (A, B may be bf16).
+cudaError_t launch_gemm_nn_f32(const void* A, bool a_bf16, int64_t lda, const void* B, bool b_bf16,
+                               int64_t ldb, float* C, int64_t ldc, int M, int N, int K,
+                               cudaStream_t st);
+cudaError_t launch_causal_attention(const float* Q, const float* K, const float* V, float* O,
+                                    int n, int d, int64_t ldq, int64_t ldk, int64_t ldo,
+                                    cudaStream_t st);
+cudaError_t launch_check_finite(const void* X, bool bf16, int64_t n, int32_t* flag, cudaStream_t st);
+
+}  // namespace spectra

@@ -1,0 +1,265 @@
+"""GPU parity of the CUDA path against the CPU oracle, through the C ABI.
+
+Bars: packed codes bit-exact when both sides quantise the same fp32 latents;
+projected latents within 1e-3 relative (per token and head-side, L2); attention
+within 2e-3 (max over (sequence, q head) of ||diff||_inf / ||ref||_inf) against
+the oracle evaluated on the same packed cache."""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_helpers import (attention_rel_err, codec_from, dev, kept_wup, make_cfg, oracle_pool_after,
+                         oracle_widths, random_factors, synthetic_latents, torch_mod)
+from workloads import bf16_round, get_config, make_activations, make_layer, make_queries
+
+pytestmark = pytest.mark.gpu
+
+# (name, d_model, n_q, n_kv, d_h, rank, group, widths per (head, side) or None, P)
+SHAPES = {
+    "toy": (256, 4, 1, 64, 32, 8, [[4, 2, 1, 1], [4, 2, 1, 1]], 64),
+    "llama4x": (512, 8, 2, 128, 128, 16, [[4, 2, 2, 2, 2, 2, 1, 1], [4, 3, 2, 2, 2, 1, 1, 1]], 64),
+    "qwen8x": (512, 7, 1, 128, 128, 16, [[4, 2, 1, 1, 0, 0, 0, 0], [4, 3, 3, 0, 0, 0, 0, 0]], 64),
+    "stress12x": (512, 8, 2, 128, 128, 16, [[4, 2, 0, 0, 0, 0, 0, 0], [4, 2, 0, 0, 0, 0, 0, 0]], 64),
+    "allwidths": (256, 4, 1, 128, 128, 16, [[8, 4, 3, 2, 1, 8, 1, 0], [1, 2, 3, 4, 8, 0, 3, 1]], 32),
+    "zeroside": (256, 8, 1, 64, 64, 16, [[2, 1, 0, 0], [0, 0, 0, 0]], 64),
+    "g8wide": (256, 16, 2, 64, 64, 8, [[8, 4, 3, 2, 1, 1, 0, 0], [3, 3, 2, 2, 1, 1, 1, 1]], 96),
+}
+
+
+def _setup(name, seed=0):
+    d_model, n_q, n_kv, d_h, rank, group, w, P = SHAPES[name]
+    widths = np.array([w] * n_kv, np.int32).reshape(n_kv, 2, rank // group)
+    if n_kv > 1:  # give heads different widths
+        widths[1:] = np.roll(widths[1:], 1, axis=2)
+    widths, W_down, W_up = random_factors(d_model, n_kv, d_h, rank, group, widths, seed=seed)
+    cfg = make_cfg(d_model, n_q, n_kv, d_h, rank, group, 512, True, P)
+    codec = codec_from(cfg, widths, W_down, W_up)
+    return dict(cfg=cfg, codec=codec, widths=widths, W_down=W_down, W_up=W_up, group=group, P=P,
+                n_q=n_q, n_kv=n_kv, d_h=d_h, d_model=d_model)
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_quantize_append_bit_exact(name):
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup(name)
+    codec, P = s["codec"], s["P"]
+    cache = st.LatentCache(codec, batch=2, max_pages_per_seq=6, device=dev())
+    # sequence 0 gets 150 tokens, sequence 1 gets 37, then a second call appends
+    # 21 + 5 more at unaligned positions
+    seqs1 = np.array([0] * 150 + [1] * 37, np.int32)
+    seqs2 = np.array([0] * 21 + [1] * 5, np.int32)
+    lat1 = synthetic_latents(len(seqs1), codec.n_eff, seed=1)
+    lat2 = synthetic_latents(len(seqs2), codec.n_eff, seed=2, scale=30.0)
+    table = cache.page_table.cpu().numpy()
+    ref = None
+    lengths = np.zeros(2, np.int64)
+    for seqs, lat in ((seqs1, lat1), (seqs2, lat2)):
+        codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+        codec.device_status()
+        ref, lengths, _ = oracle_pool_after({"group": s["group"]}, s["widths"], cache.pool.numel(),
+                                            codec.page_bytes, table, lengths, seqs, lat, P, base_pool=ref)
+        got = cache.pool.cpu().numpy()
+        bad = np.nonzero(got != ref)[0]
+        assert bad.size == 0, f"{bad.size} bytes differ, first at {bad[:8]}"
+        np.testing.assert_array_equal(cache.lengths.cpu().numpy(), lengths)
+
+
+def test_single_token_decode_steps_bit_exact():
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup("llama4x")
+    codec, P = s["codec"], s["P"]
+    B = 3
+    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=2, device=dev())
+    table = cache.page_table.cpu().numpy()
+    ref = np.zeros(cache.pool.numel(), np.uint8)
+    lengths = np.zeros(B, np.int64)
+    seqs = np.arange(B, dtype=np.int32)
+    for step in range(70):
+        lat = synthetic_latents(B, codec.n_eff, seed=100 + step)
+        codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+        ref, lengths, _ = oracle_pool_after({"group": 16}, s["widths"], ref.size, codec.page_bytes, table,
+                                            lengths, seqs, lat, P, base_pool=ref)
+    codec.device_status()
+    assert np.array_equal(cache.pool.cpu().numpy(), ref)
+    assert list(cache.lengths.cpu().numpy()) == [70] * B
+
+
+@pytest.mark.parametrize("T", [1, 3, 16, 37])
+def test_project_small_T(T):
+    torch = torch_mod()
+    s = _setup("llama4x")
+    rng = np.random.default_rng(T)
+    H = bf16_round(rng.standard_normal((T, s["d_model"])).astype(np.float32))
+    lat = s["codec"].project(torch.from_numpy(H).to(dev()).to(torch.bfloat16)).cpu().numpy()
+    ref = H.astype(np.float64) @ s["W_down"].astype(np.float64)
+    _check_latents(lat, ref, s)
+
+
+def _check_latents(lat, ref, s):
+    c0 = 0
+    for a in range(s["n_kv"]):
+        for side in range(2):
+            nk = int(sum(s["group"] for b in s["widths"][a, side] if b > 0))
+            if nk == 0:
+                continue
+            d = lat[:, c0:c0 + nk] - ref[:, c0:c0 + nk]
+            rel = np.linalg.norm(d, axis=1) / np.maximum(np.linalg.norm(ref[:, c0:c0 + nk], axis=1), 1e-30)
+            assert rel.max() <= 1e-3, rel.max()
+            c0 += nk
+
+
+def _decode_case(name, lengths, seed=0, peaked=False, P_pages=None):
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup(name, seed=seed)
+    codec, P = s["codec"], s["P"]
+    B = len(lengths)
+    maxp = P_pages or max(1, (max(lengths) + P - 1) // P)
+    # shuffled physical pages to exercise the page table
+    rng = np.random.default_rng(seed + 7)
+    perm = rng.permutation(B * maxp).astype(np.int32).reshape(B, maxp)
+    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=maxp, device=dev(),
+                           page_table=torch.from_numpy(perm))
+    seqs = np.concatenate([np.full(L, b, np.int32) for b, L in enumerate(lengths)])
+    if seqs.size:
+        lat = synthetic_latents(seqs.size, codec.n_eff, seed=seed + 11, decay=0.5, scale=2.0)
+        codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+    q = rng.standard_normal((B, s["n_q"], s["d_h"])).astype(np.float32) * 0.6
+    if peaked:
+        q *= 6.0
+    out = codec.decode_attend(cache, torch.from_numpy(q).to(dev()))
+    codec.device_status()
+    lay = oracle.page_layout(oracle_widths(s["widths"]), s["group"], P)
+    ref = oracle.decode_reference(cache.pool.cpu().numpy(), codec.page_bytes, lay, s["group"], P, perm,
+                                  np.array(lengths), q, kept_wup(s["W_up"], s["widths"], s["group"]),
+                                  s["n_q"], s["n_kv"])
+    got = out.cpu().numpy()
+    for b, L in enumerate(lengths):
+        if L == 0:
+            assert np.all(got[b] == 0)
+    live = [b for b, L in enumerate(lengths) if L > 0]
+    return attention_rel_err(got[live], ref[live])
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_decode_parity(name):
+    err = _decode_case(name, [333, 64, 1, 129])
+    assert err <= 2e-3, err
+
+
+@pytest.mark.parametrize("lengths", [[1], [31], [32], [33], [63], [64], [65], [1000], [0, 17], [4096]])
+def test_decode_edge_lengths(lengths):
+    err = _decode_case("llama4x", lengths, seed=3)
+    assert err <= 2e-3, err
+
+
+@pytest.mark.parametrize("name", ["toy", "qwen8x", "llama4x"])
+def test_decode_peaked_queries(name):
+    err = _decode_case(name, [700, 2000], seed=5, peaked=True)
+    assert err <= 2e-3, err
+
+
+def test_decode_many_sequences_stress_shape():
+    err = _decode_case("stress12x", [257] * 16, seed=9)
+    assert err <= 2e-3, err
+
+
+def test_toy_end_to_end_calibrate_encode_decode():
+    """fp32 calibration on the toy layer, bf16 encode, decode; codes bit-exact vs
+    the oracle's quantisation of the GPU latents; calibration close to the oracle's."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    cfgw = get_config("toy")
+    layer = make_layer(cfgw)
+    cfg = make_cfg(cfgw.d_model, cfgw.n_q_heads, cfgw.n_kv_heads, cfgw.d_head, cfgw.rank, cfgw.group,
+                   cfgw.budget_bits, cfgw.count_overhead, cfgw.page_tokens)
+    codec = st.Codec.calibrate(cfg, torch.from_numpy(layer["H_calib"]).to(dev()),
+                               torch.from_numpy(layer["W_K"]).to(dev()), torch.from_numpy(layer["W_V"]).to(dev()))
+    state = codec.state()
+    ref = oracle.calibrate(cfgw, layer["H_calib"], layer["W_K"], layer["W_V"])
+    for sidx, side in enumerate("KV"):
+        hs = ref["heads"][0][side]
+        np.testing.assert_allclose(state["sigma2"][0, sidx], hs["sigma2"], rtol=1e-4, atol=1e-7)
+        np.testing.assert_array_equal(state["widths"][0, sidx], hs["widths"])
+        V_gpu = state["W_up"][0, sidx].T.astype(np.float64)
+        # leading directions agree (sign fixed)
+        assert np.abs(V_gpu[:, :8] - hs["V"][:, :8]).max() < 1e-3
+    # encode + decode through the C ABI
+    n = cfgw.cache_len
+    h = bf16_round(make_activations(cfgw, n, stream=3))
+    cache = st.LatentCache(codec, batch=1, max_pages_per_seq=n // cfgw.page_tokens, device=dev())
+    lat = torch.empty((n, codec.n_eff), dtype=torch.float32, device=dev())
+    codec.encode_append(cache, torch.from_numpy(h).to(dev()).to(torch.bfloat16),
+                        torch.zeros(n, dtype=torch.int32, device=dev()), latents_out=lat)
+    codec.device_status()
+    lat_np = lat.cpu().numpy()
+    s = dict(n_kv=1, group=cfgw.group, widths=state["widths"])
+    _check_latents(lat_np, h.astype(np.float64) @ state["W_down"].astype(np.float64), s)
+    table = cache.page_table.cpu().numpy()
+    pool_ref, _, lay = oracle_pool_after({"group": cfgw.group}, state["widths"], cache.pool.numel(),
+                                         codec.page_bytes, table, np.zeros(1), np.zeros(n, np.int64), lat_np,
+                                         cfgw.page_tokens)
+    assert np.array_equal(cache.pool.cpu().numpy(), pool_ref)
+    q = make_queries(cfgw, 1)
+    out = codec.decode_attend(cache, torch.from_numpy(q).to(dev())).cpu().numpy()
+    ref_o = oracle.decode_reference(pool_ref, codec.page_bytes, lay, cfgw.group, cfgw.page_tokens, table,
+                                    np.array([n]), q, kept_wup(state["W_up"], state["widths"], cfgw.group),
+                                    cfgw.n_q_heads, 1)
+    assert attention_rel_err(out, ref_o) <= 2e-3
+
+
+def test_calibrate_bf16_llama_shaped_head():
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    cfgw = get_config("llama", n_q_heads=8, n_kv_heads=2, calib_tokens=2048)
+    layer = make_layer(cfgw)
+    W_K = layer["W_K"][:, :2 * 128]
+    W_V = layer["W_V"][:, :2 * 128]
+    cfg = make_cfg(cfgw.d_model, 8, 2, 128, 128, 16, cfgw.budget_bits, True, 64)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev()).to(torch.bfloat16)
+    codec = st.Codec.calibrate(cfg, t(layer["H_calib"]), t(W_K), t(W_V))
+    state = codec.state()
+    G = oracle.gram(layer["H_calib"])
+    for a in range(2):
+        for sidx, W in enumerate((W_K, W_V)):
+            b = oracle.latent_basis(G, W[:, a * 128:(a + 1) * 128].astype(np.float64), 128)
+            np.testing.assert_allclose(state["sigma2"][a, sidx], b["sigma2"], rtol=2e-3,
+                                       atol=1e-6 * b["sigma2"][0])
+            w_or = oracle.allocate_widths(b["sigma2"], 16, cfgw.budget_bits, True)
+            np.testing.assert_array_equal(state["widths"][a, sidx], w_or)
+
+
+def test_serialize_round_trip():
+    import spectral_transform_coding_b200 as st
+    s = _setup("llama4x")
+    blob = s["codec"].serialize()
+    c2 = st.Codec.deserialize(blob)
+    a, b = s["codec"].state(), c2.state()
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k])
+    assert c2.serialize() == blob
+    with pytest.raises(st.SpectraError):
+        st.Codec.deserialize(blob[:-3])
+
+
+def test_wo_correction_matches_oracle():
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    cfgw = get_config("toy", d_model=64, n_q_heads=2, n_kv_heads=1, d_head=16, rank=16, group=8,
+                      budget_bits=16, calib_tokens=96)
+    layer = make_layer(cfgw)
+    cfg = make_cfg(64, 2, 1, 16, 16, 8, 16, False, 64)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev())
+    codec = st.Codec.calibrate(cfg, t(layer["H_calib"]), t(layer["W_K"]), t(layer["W_V"]))
+    W_Op = codec.wo_correction(t(layer["H_calib"]), t(layer["W_Q"]), t(layer["W_K"]), t(layer["W_V"]),
+                               t(layer["W_O"])).cpu().numpy()
+    ref_codec = oracle.calibrate(cfgw, layer["H_calib"], layer["W_K"], layer["W_V"])
+    state = codec.state()
+    for sidx, side in enumerate("KV"):
+        np.testing.assert_array_equal(state["widths"][0, sidx], ref_codec["heads"][0][side]["widths"])
+    ref = oracle.wo_correction(layer["H_calib"], layer["W_Q"], layer["W_K"], layer["W_V"], layer["W_O"],
+                               ref_codec, 2, 1, 16)
+    err = np.abs(W_Op - ref["W_O"]).max() / np.abs(ref["W_O"]).max()
+    assert err < 2e-2, err
