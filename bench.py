@@ -165,7 +165,7 @@ def run_gpu(args, rank, world):
     ctx = cfg.cache_len
     steps, warm = args.steps, args.warmup
     P = cfg.page_tokens
-    cap_tokens = ctx + steps + warm + 2
+    cap_tokens = ctx + warm + steps + max(3, steps // 4) + 8
     max_pages = (cap_tokens + P - 1) // P
     c = make_config(cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head, cfg.rank, cfg.group,
                     cfg.budget_bits, cfg.count_overhead, P)
@@ -220,16 +220,17 @@ def run_gpu(args, rank, world):
     dws = [torch.empty(codecs[l].decode_workspace_bytes(B, cap_tokens), dtype=torch.uint8, device=dev)
            for l in range(L)]
     stream = torch.cuda.Stream(device=dev)
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
 
-    def step(record=False):
+    def encode_layer(l):
+        codecs[l].encode_append(caches[l], H_new[l], seq_ids, workspace=ews[l], stream=stream)
+
+    def decode_layer(l):
+        codecs[l].decode_attend(caches[l], Q[l], OUT[l], workspace=dws[l], stream=stream)
+
+    def step():
         for l in range(L):
-            codecs[l].encode_append(caches[l], H_new[l], seq_ids, workspace=ews[l], stream=stream)
-            if record:
-                ev_dec[l][0].record(stream)
-            codecs[l].decode_attend(caches[l], Q[l], OUT[l], workspace=dws[l], stream=stream)
-            if record:
-                ev_dec[l][1].record(stream)
+            encode_layer(l)
+            decode_layer(l)
 
     # host (pinned) buffers for the end-to-end arm
     H_host = H_new.cpu().pin_memory()
@@ -248,65 +249,65 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
     len0 = int(caches[0].lengths.float().mean().item())
 
+    # CUDA graphs: one decode step of all layers; decode attention of all layers;
+    # the step with its host<->device copies
+    g_step, g_dec, g_e2e = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        step()
+    with torch.cuda.graph(g_dec, stream=stream):
+        for l in range(L):
+            decode_layer(l)
+    with torch.cuda.graph(g_e2e, stream=stream):
+        step_e2e()
+    torch.cuda.synchronize()
+    for codec in codecs:
+        codec.device_status()
+
     def barrier():
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
 
-    # ---- device-resident timed region (K steps) ----
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dec_ms = []
-    with ClockSampler(local) as clocks:
+    def timed(graph, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            t_start.record(stream)
-            for k in range(steps):
-                step(record=True)
-                if k == steps - 1:
-                    pass
-            t_end.record(stream)
+            a.record(stream)
+            for _ in range(n):
+                graph.replay()
+            b.record(stream)
         torch.cuda.synchronize()
         barrier()
-    # decode-attention launch durations (events recorded on the launching stream)
-    with torch.cuda.stream(stream):
-        pass
-    for l in range(L):
-        dec_ms.append(ev_dec[l][0].elapsed_time(ev_dec[l][1]))
-    total_ms = t_start.elapsed_time(t_end)
+        return a.elapsed_time(b)
+
+    # ---- device-resident timed region: K decode steps ----
+    with ClockSampler(local) as clocks:
+        total_ms = timed(g_step, steps)
     clk = clocks.summary()
-
-    # ---- end-to-end arm (host buffers, copies inside the timed region) ----
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    len_after = int(caches[0].lengths.float().mean().item())
+    # ---- decode-attention launches alone (same kernels, same resident caches) ----
+    dec_ms = timed(g_dec, steps) / (steps * L)
+    # ---- end-to-end: host buffers, copies inside the timed region ----
     ksteps_e2e = max(3, steps // 4)
-    with torch.cuda.stream(stream):
-        step_e2e()
-    torch.cuda.synchronize()
-    barrier()
-    with torch.cuda.stream(stream):
-        e_start.record(stream)
-        for _ in range(ksteps_e2e):
-            step_e2e()
-        e_end.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / ksteps_e2e
-
-    codecs[0].device_status(stream)
+    e2e_ms = timed(g_e2e, ksteps_e2e) / ksteps_e2e
+    for codec in codecs:
+        codec.device_status(stream)
     ms_per_step = total_ms / steps
     if world > 1:
         import torch.distributed as dist
-        t = torch.tensor([ms_per_step, e2e_ms], device=dev)
+        t = torch.tensor([ms_per_step, e2e_ms, dec_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step, e2e_ms = float(t[0]), float(t[1])
-    mean_ctx = len0 + (steps + 1) / 2.0
+        ms_per_step, e2e_ms, dec_ms = float(t[0]), float(t[1]), float(t[2])
+    mean_ctx = (len0 + len_after) / 2.0
     tok_per_step = L * B * mean_ctx * cfg.n_kv_heads
     value = tok_per_step / (ms_per_step / 1e3) * world
     e2e_value = tok_per_step / (e2e_ms / 1e3) * world
 
     # roofline: packed bytes the decode reads per layer
     bytes_per_tok_all_heads = codecs[0].page_bytes / P
-    dec_bytes = B * mean_ctx * bytes_per_tok_all_heads
-    dec_avg_ms = statistics.mean(dec_ms)
+    dec_bytes = B * len_after * bytes_per_tok_all_heads
+    dec_avg_ms = dec_ms
     peaks = _peaks()
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     launches_per_layer = 3 + 3  # encode: projection, append plan, quantise/pack; decode: fold, split, combine

@@ -185,9 +185,11 @@ SPECTRA_API spectra_status spectra_codec_deserialize(const void* buf, size_t byt
  * training-free correction of W_O for the rank truncation.  Reading used here
  * (the pages give no formula): treat the calibration tokens as one causal
  * sequence; for each q head h (KV head a = h / (n_q/n_kv)) let O_h be the
- * attention output with exact K, V and Oh_h the one with the rank-truncated,
- * unquantised K, V (kept coordinates only); M_h = (Oh^T Oh + eps I)^-1 Oh^T O with
- * eps = 1e-8 tr(Oh^T Oh)/d_head, and W_O' = blockdiag(M_h) W_O.
+ * attention output with exact K, V and L_h the latent output of attention with
+ * the rank-truncated, unquantised K and the values projected on the kept value
+ * directions U_a (kept coordinates only).  M'_h = (L_h^T L_h + eps I)^-1 L_h^T O_h
+ * with eps = 1e-8 tr(L_h^T L_h)/n_kept, M_h = U_a M'_h, W_O' = blockdiag(M_h) W_O
+ * (the minimum-norm least-squares map from the truncated output to the exact one).
  *   H device [n_tokens][d_model]; W_Q device [d_model][n_q_heads*d_head];
  *   W_K, W_V as for calibrate; W_O device [n_q_heads*d_head][d_model];
  *   W_O_out device fp32 [n_q_heads*d_head][d_model].  All inputs in `dtype`.

@@ -582,13 +582,16 @@ def wo_correction(H: np.ndarray, W_Q: np.ndarray, W_K: np.ndarray, W_V: np.ndarr
                   eps_rel: float = 1e-8) -> dict:
     """Closed-form, training-free W_O correction (parity unpinned beyond special cases).
 
-    Reading: for each q head h (KV head a = h // Gq) on the calibration tokens as
-    one causal sequence, O_h uses exact K, V and O^_h the rank-truncated,
-    unquantised ones (kept coordinates only: k~ = k V_r P V_r^T).  The least
-    squares map M_h = (O^^T O^ + eps I)^-1 O^^T O with eps = eps_rel tr(O^^T O^)/d_h
-    is folded into W_O: W_O' = blockdiag(M_h) W_O.  Pinned only by: M_h = I when
-    nothing is truncated (eps -> 0), and the corrected residual never exceeds
-    the uncorrected one.
+    Reading: for each q head h (KV head a = h // Gq), on the calibration tokens as
+    one causal sequence, O_h is the attention output with exact K, V and O^_h the
+    one with the rank-truncated, unquantised K, V (kept coordinates only:
+    k~ = k V_r P V_r^T).  O^_h lies in the span of the kept value directions U_a,
+    so write O^_h = L_h U_a^T (L_h = latent output).  The least-squares map from
+    L_h to O_h, M'_h = (L_h^T L_h + eps I)^-1 L_h^T O_h with eps = eps_rel
+    tr(L_h^T L_h)/n_kept, gives M_h = U_a M'_h and W_O' = blockdiag(M_h) W_O.
+    As eps -> 0 this is the minimum-norm solution of min ||O^_h M - O_h||.  Pinned
+    only by: M_h = I when nothing is truncated (eps -> 0), and the corrected
+    residual never exceeds the uncorrected one.
     """
     H64 = np.asarray(H, dtype=np.float64)
     gq = n_q // n_kv
@@ -601,16 +604,18 @@ def wo_correction(H: np.ndarray, W_Q: np.ndarray, W_K: np.ndarray, W_V: np.ndarr
         q = H64 @ np.asarray(W_Q, dtype=np.float64)[:, h * d_h:(h + 1) * d_h]
         k = H64 @ np.asarray(W_K, dtype=np.float64)[:, sl]
         v = H64 @ np.asarray(W_V, dtype=np.float64)[:, sl]
-        tr = []
-        for side, x in (("K", k), ("V", v)):
-            hs = codec["heads"][a][side]
-            Vr = hs["V"][:, hs["keep"]]
-            tr.append(x @ Vr @ Vr.T)
+        hk, hv = codec["heads"][a]["K"], codec["heads"][a]["V"]
+        Vk = hk["V"][:, hk["keep"]]
+        U = hv["V"][:, hv["keep"]]
         O = causal_attention(q, k, v)
-        Oh = causal_attention(q, tr[0], tr[1])
-        A = Oh.T @ Oh
-        eps = eps_rel * np.trace(A) / d_h
-        M = np.linalg.solve(A + eps * np.eye(d_h), Oh.T @ O)
+        lat = causal_attention(q, k @ Vk @ Vk.T, v @ U)  # latent value output L_h
+        if U.shape[1] == 0:
+            M = np.zeros((d_h, d_h))
+        else:
+            A = lat.T @ lat
+            eps = eps_rel * np.trace(A) / U.shape[1]
+            Mp = np.linalg.solve(A + eps * np.eye(U.shape[1]), lat.T @ O)
+            M = U @ Mp
         Ms.append(M)
         W_Op[h * d_h:(h + 1) * d_h, :] = M @ W_O[h * d_h:(h + 1) * d_h, :]
     return dict(M=Ms, W_O=W_Op)

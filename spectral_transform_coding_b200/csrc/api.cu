@@ -164,14 +164,15 @@ spectra_status check_cache(const spectra_codec* c, const spectra_cache* cache) {
 }
 
 spectra_status do_project(const spectra_codec* c, const void* H, int64_t T, float* C, cudaStream_t st) {
+  // T >= 64 rows: tcgen05 tensor-core GEMM; fewer rows: the projection is a
+  // weight-streaming GEMV bounded by HBM, done on CUDA cores.
   if (T >= 64) {
-    cudaError_t e = launch_project_tcgen05(c->h, c->h.wt_down, static_cast<const uint16_t*>(H), (int)T,
-                                           C, c->h.n_eff, st);
-    if (e == cudaSuccess) return SPECTRA_OK;
-    if (e != cudaErrorNotSupported) return fail(SPECTRA_ERR_CUDA, std::string("projection: ") + cudaGetErrorString(e));
+    CUDA_TRY(launch_project_tcgen05(c->h, c->h.wt_down, static_cast<const uint16_t*>(H), (int)T, C,
+                                    c->h.n_eff, st));
+  } else {
+    CUDA_TRY(launch_project_gemv(c->h, c->h.wt_down, static_cast<const uint16_t*>(H), (int)T, C,
+                                 c->h.n_eff, st));
   }
-  CUDA_TRY(launch_project_gemv(c->h, c->h.wt_down, static_cast<const uint16_t*>(H), (int)T, C,
-                               c->h.n_eff, st));
   return SPECTRA_OK;
 }
 
@@ -354,11 +355,7 @@ spectra_status spectra_calibrate(const spectra_config* cfg, int32_t dtype, const
   CUDA_TRY(launch_check_finite(W_V, bf, (int64_t)dm * kvw, flag, st));
   // G = sum_t h_t^T h_t
   if (bf) {
-    cudaError_t e = launch_gram_tcgen05(static_cast<const uint16_t*>(H), n_tokens, dm, G, st);
-    if (e == cudaErrorNotSupported) {
-      e = launch_gemm_tn_f32(H, true, dm, H, true, dm, G, dm, dm, dm, (int)n_tokens, st);
-    }
-    CUDA_TRY(e);
+    CUDA_TRY(launch_gram_tcgen05(static_cast<const uint16_t*>(H), n_tokens, dm, G, st));
   } else {
     CUDA_TRY(launch_gram_f32(static_cast<const float*>(H), n_tokens, dm, G, st));
   }
@@ -456,71 +453,91 @@ spectra_status spectra_wo_correction(const spectra_codec* c, int32_t dtype, cons
   const int dm = cfg.d_model, dh = cfg.d_head, nkv = cfg.n_kv_heads, nq = cfg.n_q_heads;
   const int gq = nq / nkv, n = (int)n_tokens, ng = c->n_groups;
   const size_t esz = bf ? 2 : 4;
+  // kept directions per (head, side): columns of V_r for groups with b > 0
+  auto kept_basis = [&](int a, int s, std::vector<float>& U) {
+    const size_t hs = (size_t)a * 2 + s;
+    std::vector<int> rows;
+    for (int j = 0; j < ng; ++j)
+      if (c->widths[hs * ng + j] != 0)
+        for (int k = 0; k < cfg.group; ++k) rows.push_back(j * cfg.group + k);
+    U.assign((size_t)dh * rows.size(), 0.f);  // [dh][kept]
+    for (size_t r = 0; r < rows.size(); ++r)
+      for (int d = 0; d < dh; ++d) U[(size_t)d * rows.size() + r] = c->wup[(hs * cfg.rank + rows[r]) * dh + d];
+    return (int)rows.size();
+  };
   DevBuf buf;
-  const size_t szQ = (size_t)n * nq * dh * 4, szKV = (size_t)n * nkv * dh * 4;
-  const size_t szO = (size_t)n * dh * 4, szP = (size_t)dh * dh * 4;
-  CUDA_TRY(cudaMalloc(&buf.p, szQ + 4 * szKV + 2 * szO + 3 * szP + 1024));
+  const size_t szQ = (size_t)n * nq * dh, szKV = (size_t)n * nkv * dh;
+  const size_t total = (szQ + 4 * szKV + 2 * (size_t)n * dh + 3 * (size_t)dh * dh) * 4 + 4096;
+  CUDA_TRY(cudaMalloc(&buf.p, total));
   float* Q = static_cast<float*>(buf.p);
-  float* K = Q + (size_t)n * nq * dh;
-  float* V = K + (size_t)n * nkv * dh;
-  float* Kt = V + (size_t)n * nkv * dh;
-  float* Vt = Kt + (size_t)n * nkv * dh;
-  float* O = Vt + (size_t)n * nkv * dh;
-  float* Oh = O + (size_t)n * dh;
-  float* Pm = Oh + (size_t)n * dh;
+  float* K = Q + szQ;
+  float* V = K + szKV;
+  float* Kt = V + szKV;    // truncated keys, [n][nkv*dh]
+  float* Vl = Kt + szKV;   // latent values per head, [n][nkv*dh] (first kept columns used)
+  float* O = Vl + szKV;    // [n][dh]
+  float* Ol = O + (size_t)n * dh;
+  float* Pm = Ol + (size_t)n * dh;
   float* AB = Pm + (size_t)dh * dh;
   CUDA_TRY(launch_gemm_nn_f32(H, bf, dm, W_Q, bf, nq * dh, Q, nq * dh, n, nq * dh, dm, st));
   CUDA_TRY(launch_gemm_nn_f32(H, bf, dm, W_K, bf, nkv * dh, K, nkv * dh, n, nkv * dh, dm, st));
   CUDA_TRY(launch_gemm_nn_f32(H, bf, dm, W_V, bf, nkv * dh, V, nkv * dh, n, nkv * dh, dm, st));
-  // rank-truncated keys / values: x V_r,kept V_r,kept^T
-  std::vector<float> P((size_t)dh * dh);
-  for (int a = 0; a < nkv; ++a)
-    for (int s = 0; s < 2; ++s) {
-      const size_t hs = (size_t)a * 2 + s;
-      std::vector<double> Pd((size_t)dh * dh, 0.0);
-      for (int j = 0; j < ng; ++j) {
-        if (c->widths[hs * ng + j] == 0) continue;
-        for (int k = 0; k < cfg.group; ++k) {
-          const float* v = c->wup.data() + (hs * cfg.rank + j * cfg.group + k) * dh;
-          for (int x = 0; x < dh; ++x)
-            for (int y = 0; y < dh; ++y) Pd[(size_t)x * dh + y] += (double)v[x] * v[y];
-        }
+  std::vector<int> keptV(nkv);
+  std::vector<std::vector<float>> UV(nkv);
+  for (int a = 0; a < nkv; ++a) {
+    std::vector<float> Uk;
+    const int kk = kept_basis(a, 0, Uk);
+    std::vector<float> P((size_t)dh * dh, 0.f);  // U_k U_k^T
+    for (int x = 0; x < dh; ++x)
+      for (int y = 0; y < dh; ++y) {
+        double acc = 0.0;
+        for (int r = 0; r < kk; ++r) acc += (double)Uk[(size_t)x * kk + r] * Uk[(size_t)y * kk + r];
+        P[(size_t)x * dh + y] = (float)acc;
       }
-      for (size_t i = 0; i < P.size(); ++i) P[i] = (float)Pd[i];
-      CUDA_TRY(cudaMemcpyAsync(Pm, P.data(), P.size() * 4, cudaMemcpyHostToDevice, st));
-      const float* X = (s == 0 ? K : V) + (size_t)a * dh;
-      float* Y = (s == 0 ? Kt : Vt) + (size_t)a * dh;
-      CUDA_TRY(launch_gemm_nn_f32(X, false, nkv * dh, Pm, false, dh, Y, nkv * dh, n, dh, dh, st));
-      CUDA_TRY(cudaStreamSynchronize(st));  // P is reused for the next head
+    CUDA_TRY(cudaMemcpyAsync(Pm, P.data(), P.size() * 4, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(launch_gemm_nn_f32(K + (size_t)a * dh, false, nkv * dh, Pm, false, dh, Kt + (size_t)a * dh, nkv * dh,
+                                n, dh, dh, st));
+    keptV[a] = kept_basis(a, 1, UV[a]);
+    if (keptV[a] > 0) {
+      CUDA_TRY(cudaMemcpyAsync(Pm + (size_t)dh * dh, UV[a].data(), UV[a].size() * 4, cudaMemcpyHostToDevice, st));
+      CUDA_TRY(launch_gemm_nn_f32(V + (size_t)a * dh, false, nkv * dh, Pm + (size_t)dh * dh, false, keptV[a],
+                                  Vl + (size_t)a * dh, nkv * dh, n, keptV[a], dh, st));
     }
-  std::vector<float> Ahost((size_t)dh * dh), Bhost((size_t)dh * dh), Ms((size_t)dh * dh);
+    CUDA_TRY(cudaStreamSynchronize(st));  // host buffers are reused for the next head
+  }
+  std::vector<float> Ah((size_t)dh * dh), Bh((size_t)dh * dh), Ms((size_t)dh * dh);
   for (int h = 0; h < nq; ++h) {
-    const int a = h / gq;
-    const float* Qh = Q + (size_t)h * dh;
-    CUDA_TRY(launch_causal_attention(Qh, K + (size_t)a * dh, V + (size_t)a * dh, O, n, dh, nq * dh,
-                                     nkv * dh, dh, st));
-    CUDA_TRY(launch_causal_attention(Qh, Kt + (size_t)a * dh, Vt + (size_t)a * dh, Oh, n, dh, nq * dh,
-                                     nkv * dh, dh, st));
-    CUDA_TRY(launch_gemm_tn_f32(Oh, false, dh, Oh, false, dh, AB, dh, dh, dh, n, st));
-    CUDA_TRY(launch_gemm_tn_f32(Oh, false, dh, O, false, dh, AB + (size_t)dh * dh, dh, dh, dh, n, st));
-    CUDA_TRY(cudaMemcpyAsync(Ahost.data(), AB, Ahost.size() * 4, cudaMemcpyDeviceToHost, st));
-    CUDA_TRY(cudaMemcpyAsync(Bhost.data(), AB + (size_t)dh * dh, Bhost.size() * 4, cudaMemcpyDeviceToHost, st));
-    CUDA_TRY(cudaStreamSynchronize(st));
-    std::vector<double> A2((size_t)dh * dh), B2((size_t)dh * dh);
-    double tr = 0.0;
-    for (int i = 0; i < dh; ++i) tr += Ahost[(size_t)i * dh + i];
-    const double eps = 1e-8 * tr / dh;
-    for (size_t i = 0; i < A2.size(); ++i) {
-      A2[i] = Ahost[i];
-      B2[i] = Bhost[i];
+    const int a = h / gq, kv = keptV[a];
+    std::fill(Ms.begin(), Ms.end(), 0.f);
+    if (kv > 0) {
+      const float* Qh = Q + (size_t)h * dh;
+      CUDA_TRY(launch_causal_attention(Qh, K + (size_t)a * dh, V + (size_t)a * dh, O, n, dh, dh, nq * dh,
+                                       nkv * dh, nkv * dh, dh, st));
+      CUDA_TRY(launch_causal_attention(Qh, Kt + (size_t)a * dh, Vl + (size_t)a * dh, Ol, n, dh, kv, nq * dh,
+                                       nkv * dh, nkv * dh, kv, st));
+      CUDA_TRY(launch_gemm_tn_f32(Ol, false, kv, Ol, false, kv, AB, kv, kv, kv, n, st));
+      CUDA_TRY(launch_gemm_tn_f32(Ol, false, kv, O, false, dh, AB + (size_t)dh * dh, dh, kv, dh, n, st));
+      CUDA_TRY(cudaMemcpyAsync(Ah.data(), AB, (size_t)kv * kv * 4, cudaMemcpyDeviceToHost, st));
+      CUDA_TRY(cudaMemcpyAsync(Bh.data(), AB + (size_t)dh * dh, (size_t)kv * dh * 4, cudaMemcpyDeviceToHost, st));
+      CUDA_TRY(cudaStreamSynchronize(st));
+      std::vector<double> A2((size_t)kv * kv), B2((size_t)kv * dh);
+      double tr = 0.0;
+      for (int i = 0; i < kv; ++i) tr += Ah[(size_t)i * kv + i];
+      const double eps = 1e-8 * tr / kv;
+      for (size_t i = 0; i < A2.size(); ++i) A2[i] = Ah[i];
+      for (size_t i = 0; i < B2.size(); ++i) B2[i] = Bh[i];
+      for (int i = 0; i < kv; ++i) A2[(size_t)i * kv + i] += eps;
+      if (!solve_dense(A2, B2, kv, dh)) return fail(SPECTRA_ERR_NUMERIC, "singular W_O correction system");
+      // M = U M'  (dh x dh)
+      for (int x = 0; x < dh; ++x)
+        for (int y = 0; y < dh; ++y) {
+          double acc = 0.0;
+          for (int r = 0; r < kv; ++r) acc += (double)UV[a][(size_t)x * kv + r] * B2[(size_t)r * dh + y];
+          Ms[(size_t)x * dh + y] = (float)acc;
+        }
     }
-    for (int i = 0; i < dh; ++i) A2[(size_t)i * dh + i] += eps;
-    if (!solve_dense(A2, B2, dh, dh)) return fail(SPECTRA_ERR_NUMERIC, "singular W_O correction system");
-    for (size_t i = 0; i < Ms.size(); ++i) Ms[i] = (float)B2[i];
     CUDA_TRY(cudaMemcpyAsync(Pm, Ms.data(), Ms.size() * 4, cudaMemcpyHostToDevice, st));
     const void* WOh = static_cast<const uint8_t*>(W_O) + (size_t)h * dh * dm * esz;
-    CUDA_TRY(launch_gemm_nn_f32(Pm, false, dh, WOh, bf, dm, W_O_out + (size_t)h * dh * dm, dm, dh, dm,
-                                dh, st));
+    CUDA_TRY(launch_gemm_nn_f32(Pm, false, dh, WOh, bf, dm, W_O_out + (size_t)h * dh * dm, dm, dh, dm, dh, st));
     CUDA_TRY(cudaStreamSynchronize(st));
   }
   return SPECTRA_OK;

@@ -85,25 +85,26 @@ cudaError_t gemm_dispatch(const void* A, bool a_bf16, int64_t lda, const void* B
   return cudaGetLastError();
 }
 
-// One block per query row: scores against keys 0..i, softmax, weighted values.
+// One block per query row: scores against keys 0..i (width dk), softmax,
+// weighted values (width dv).
 __global__ void __launch_bounds__(256) causal_attention_kernel(const float* __restrict__ Q,
                                                                const float* __restrict__ K,
                                                                const float* __restrict__ V,
-                                                               float* __restrict__ O, int n, int d,
-                                                               int64_t ldq, int64_t ldk,
-                                                               int64_t ldo) {
+                                                               float* __restrict__ O, int n, int dk,
+                                                               int dv, int64_t ldq, int64_t ldk,
+                                                               int64_t ldv, int64_t ldo) {
   extern __shared__ float sh[];
-  float* q = sh;          // [d]
-  float* s = sh + d;      // [n]
+  float* q = sh;          // [dk]
+  float* s = sh + dk;     // [n]
   __shared__ float red[32];
   const int i = blockIdx.x;
-  for (int e = threadIdx.x; e < d; e += blockDim.x) q[e] = Q[(int64_t)i * ldq + e];
+  for (int e = threadIdx.x; e < dk; e += blockDim.x) q[e] = Q[(int64_t)i * ldq + e];
   __syncthreads();
-  const float scale = rsqrtf((float)d);
+  const float scale = rsqrtf((float)dk);
   float mx = -CUDART_INF_F;
   for (int j = threadIdx.x; j <= i; j += blockDim.x) {
     float acc = 0.f;
-    for (int e = 0; e < d; ++e) acc = fmaf(q[e], K[(int64_t)j * ldk + e], acc);
+    for (int e = 0; e < dk; ++e) acc = fmaf(q[e], K[(int64_t)j * ldk + e], acc);
     s[j] = acc * scale;
     mx = fmaxf(mx, s[j]);
   }
@@ -133,9 +134,9 @@ __global__ void __launch_bounds__(256) causal_attention_kernel(const float* __re
   }
   __syncthreads();
   const float inv = 1.f / red[30];
-  for (int e = threadIdx.x; e < d; e += blockDim.x) {
+  for (int e = threadIdx.x; e < dv; e += blockDim.x) {
     float acc = 0.f;
-    for (int j = 0; j <= i; ++j) acc = fmaf(s[j], V[(int64_t)j * ldk + e], acc);
+    for (int j = 0; j <= i; ++j) acc = fmaf(s[j], V[(int64_t)j * ldv + e], acc);
     O[(int64_t)i * ldo + e] = acc * inv;
   }
 }
@@ -169,14 +170,15 @@ cudaError_t launch_gram_f32(const float* H, int64_t n_tokens, int d_model, float
 }
 
 cudaError_t launch_causal_attention(const float* Q, const float* K, const float* V, float* O, int n,
-                                    int d, int64_t ldq, int64_t ldk, int64_t ldo, cudaStream_t st) {
-  const int smem = (d + n) * 4;
+                                    int dk, int dv, int64_t ldq, int64_t ldk, int64_t ldv, int64_t ldo,
+                                    cudaStream_t st) {
+  const int smem = (dk + n) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(causal_attention_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  causal_attention_kernel<<<n, 256, smem, st>>>(Q, K, V, O, n, d, ldq, ldk, ldo);
+  causal_attention_kernel<<<n, 256, smem, st>>>(Q, K, V, O, n, dk, dv, ldq, ldk, ldv, ldo);
   return cudaGetLastError();
 }
 

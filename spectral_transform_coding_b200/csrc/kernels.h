@@ -48,8 +48,8 @@ cudaError_t launch_gemm_nn_f32(const void* A, bool a_bf16, int64_t lda, const vo
                                int64_t ldb, float* C, int64_t ldc, int M, int N, int K,
                                cudaStream_t st);
 cudaError_t launch_causal_attention(const float* Q, const float* K, const float* V, float* O,
-                                    int n, int d, int64_t ldq, int64_t ldk, int64_t ldo,
-                                    cudaStream_t st);
+                                    int n, int dk, int dv, int64_t ldq, int64_t ldk, int64_t ldv,
+                                    int64_t ldo, cudaStream_t st);
 cudaError_t launch_check_finite(const void* X, bool bf16, int64_t n, int32_t* flag, cudaStream_t st);
 
 }  // namespace spectra

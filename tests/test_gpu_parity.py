@@ -97,6 +97,19 @@ def test_project_small_T(T):
     _check_latents(lat, ref, s)
 
 
+@pytest.mark.parametrize("T,name", [(64, "llama4x"), (130, "llama4x"), (1000, "qwen8x"), (257, "toy"),
+                                    (300, "allwidths")])
+def test_project_tcgen05(T, name):
+    """T >= 64 runs on the tcgen05 tensor-core GEMM (ragged M and N tails)."""
+    torch = torch_mod()
+    s = _setup(name)
+    rng = np.random.default_rng(T)
+    H = bf16_round(rng.standard_normal((T, s["d_model"])).astype(np.float32))
+    lat = s["codec"].project(torch.from_numpy(H).to(dev()).to(torch.bfloat16)).cpu().numpy()
+    ref = H.astype(np.float64) @ s["W_down"].astype(np.float64)
+    _check_latents(lat, ref, s)
+
+
 def _check_latents(lat, ref, s):
     c0 = 0
     for a in range(s["n_kv"]):
