@@ -253,6 +253,25 @@ SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, con
                                      const float* q, float* out, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* spectra_decode_attend_noalloc -- the decode attention of spectra_decode_attend
+ * for callers that cannot allocate device memory while they decode (a runtime
+ * that plans all of its buffers ahead of time, a process whose device allocator
+ * belongs to another framework, code running where an allocation would stall
+ * or be refused).  No counterpart on the SPECTRA pages: an interface of this
+ * library only.  Arguments as for spectra_decode_attend minus the workspace.
+ * The scratch (folded queries, split-K partials) lives in one static 4 MiB
+ * device array per GPU, kept until the process exits.  The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress), so make
+ * the first call on each device before any stream capture.  Every call shares
+ * the array and leaves its contents behind; nothing in it needs to start at
+ * zero.  Calls whose kernels can overlap on the GPU (other streams, other
+ * codecs at the same time) race on the array: serialise them.  A batch/context
+ * whose scratch would exceed 4 MiB fails with SPECTRA_ERR_CAPACITY.  Calls no
+ * cudaMalloc, cudaFree or allocating library routine. */
+SPECTRA_API spectra_status spectra_decode_attend_noalloc(const spectra_codec* codec,
+                                                         const spectra_cache* cache, const float* q,
+                                                         float* out, void* stream);
+
 /* Synchronises `stream`, then reads and clears the codec's device error word.
  * Returns the recorded device-side status (SPECTRA_OK if none). */
 SPECTRA_API spectra_status spectra_device_status(const spectra_codec* codec, void* stream);

@@ -62,6 +62,7 @@ _SIGS = {
     "spectra_quantize_append": [_vp, _P(CacheDesc), _vp, _vp, _i64, _vp, _sz, _vp],
     "spectra_encode_append": [_vp, _P(CacheDesc), _vp, _vp, _i64, _vp, _vp, _sz, _vp],
     "spectra_decode_attend": [_vp, _P(CacheDesc), _vp, _vp, _vp, _sz, _vp],
+    "spectra_decode_attend_noalloc": [_vp, _P(CacheDesc), _vp, _vp, _vp],
     "spectra_device_status": [_vp, _vp],
     "spectra_allocate_widths": [_vp, _i32, _i32, _i32, _i32, _vp, _vp],
     "spectra_water_fill": [_vp, _i32, ctypes.c_double, _vp, _vp],

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <memory>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -630,3 +631,61 @@ spectra_status spectra_device_status(const spectra_codec* c, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without any allocation.
+//
+// Some callers cannot allocate device memory at all when they run decode: a
+// runtime that plans every buffer statically ahead of time, a host process
+// whose allocator is owned by another framework, or code that runs where a
+// cudaMalloc would stall or be refused.  They still own their inputs and
+// outputs, but have nowhere to put the decode's scratch (folded queries and
+// the split-K partial records).  This entry point keeps that scratch in one
+// file-scope device array of fixed size instead.  The array exists on every
+// GPU that loads the library until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB per device
+static __device__ __align__(256) uint8_t g_static_decode_scratch[kStaticScratchBytes];
+
+struct StaticScratch {
+  std::mutex mu;
+  void* ptr[64] = {};
+};
+StaticScratch g_static_scratch;
+
+}  // namespace
+
+extern "C" spectra_status spectra_decode_attend_noalloc(const spectra_codec* c, const spectra_cache* cache,
+                                                        const float* q, float* out, void* stream) {
+  if (!c || !q || !out) return fail(SPECTRA_ERR_INVALID, "null pointer");
+  if (!c->decode_ok) return fail(SPECTRA_ERR_UNSUPPORTED, c->decode_why);
+  if (!aligned(q, 16) || !aligned(out, 16)) return fail(SPECTRA_ERR_INVALID, "misaligned buffer");
+  spectra_status s = check_cache(c, cache);
+  if (s != SPECTRA_OK) return s;
+  s = check_device(c);
+  if (s != SPECTRA_OK) return s;
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(SPECTRA_ERR_UNSUPPORTED, "device ordinal above 63");
+  void* scratch = nullptr;
+  {
+    // First call on this device: look up the device address of the static array
+    // (the host-side symbol is not a device address).
+    std::lock_guard<std::mutex> lock(g_static_scratch.mu);
+    if (!g_static_scratch.ptr[dev]) {
+      void* p = nullptr;
+      CUDA_TRY(cudaGetSymbolAddress(&p, g_static_decode_scratch));
+      g_static_scratch.ptr[dev] = p;
+    }
+    scratch = g_static_scratch.ptr[dev];
+  }
+  const DecodePlan plan = make_decode_plan(c->h, cache->batch, cache->max_pages_per_seq);
+  if (plan.ws_bytes > kStaticScratchBytes)
+    return fail(SPECTRA_ERR_CAPACITY, "decode needs " + std::to_string(plan.ws_bytes) +
+                                          " bytes of scratch; the static area holds 4 MiB (use "
+                                          "spectra_decode_attend with a caller workspace)");
+  CUDA_TRY(launch_decode(c->h, c->d, *cache, q, out, scratch, plan, static_cast<cudaStream_t>(stream)));
+  return SPECTRA_OK;
+}
