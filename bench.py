@@ -217,7 +217,7 @@ def run_gpu(args, rank, world):
     OUT = torch.empty_like(Q)
     seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
     ews = [torch.empty(codecs[l].encode_workspace_bytes(B), dtype=torch.uint8, device=dev) for l in range(L)]
-    dws = [torch.empty(codecs[l].decode_workspace_bytes(B, cap_tokens), dtype=torch.uint8, device=dev)
+    dws = [torch.zeros(codecs[l].decode_workspace_bytes(B, cap_tokens), dtype=torch.uint8, device=dev)
            for l in range(L)]
     stream = torch.cuda.Stream(device=dev)
 
@@ -335,7 +335,8 @@ def run_gpu(args, rank, world):
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
-            "kernel": "decode attention launch sequence (fold, split-K latent flash-decode, combine)",
+            "kernel": "split_kernel (latent flash-decode over the packed pages), timed with its fold and combine "
+                      "launches chained by programmatic dependent launch",
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": None,
             "peak_src": peaks["src"], "avg_launch_us": dec_avg_ms * 1e3,

@@ -127,7 +127,7 @@ class Codec:
 
     def _workspace(self, nbytes, device):
         torch = _torch()
-        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
     # -- hot path ----------------------------------------------------------
     def project(self, H, out=None, stream=None):

@@ -129,13 +129,18 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
   for (int a = 0; a < cfg.n_kv_heads; ++a)
     for (int s = 0; s < 2; ++s) {
       const SideDev& sd = c->h.head[a].side[s];
+      // V side row-major [n_kept][d_h]; K side transposed [d_h][n_kept] (the query
+      // fold reads it column-wise)
       int row = 0;
       for (int j = 0; j < c->n_groups; ++j) {
         if (widths[((size_t)a * 2 + s) * c->n_groups + j] == 0) continue;
         for (int k = 0; k < cfg.group; ++k, ++row) {
           const int src = j * cfg.group + k;
           const float* from = W_up + (((size_t)a * 2 + s) * cfg.rank + src) * dh;
-          std::copy(from, from + dh, wu.begin() + sd.wup_off + (size_t)row * dh);
+          for (int d = 0; d < dh; ++d) {
+            const size_t at = s == 0 ? (size_t)d * sd.n_kept + row : (size_t)row * dh + d;
+            wu[sd.wup_off + at] = from[d];
+          }
         }
       }
     }

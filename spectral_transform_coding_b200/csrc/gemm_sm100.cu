@@ -246,11 +246,9 @@ cudaError_t gemm_tn(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t l
   if ((lda * 2) % 16 || (ldb * 2) % 16 || ((uintptr_t)A) % 16 || ((uintptr_t)B) % 16) return cudaErrorNotSupported;
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, M, K, lda, BM) || !make_map(&mb, B, N, K, ldb, BN)) return cudaErrorNotSupported;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemm_tcgen05_kernel), SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
   gemm_tcgen05_kernel<<<grid, 128, SMEM_BYTES, st>>>(ma, mb, C, ldc, M, N, K, err);

@@ -17,13 +17,16 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
                                    int T, const spectra_cache& cache, cudaStream_t st);
 
 // decode_kernels.cu
+// Raises `kern`'s dynamic shared-memory limit on the current device to at least
+// `bytes` (one record per kernel and device; the limit never shrinks).
+cudaError_t ensure_dynamic_smem(const void* kern, int bytes);
 struct DecodePlan {
-  int n_split;       // context splits per (sequence, KV head)
+  int n_split;       // context splits per (sequence, KV head), before clamping to the cache's pages
   int stages;        // bulk-copy stages per warp
   int stage_bytes;   // bytes per stage (largest head section, rounded to 16)
-  int smem_bytes;    // dynamic shared memory per CTA
-  size_t qlat_off, qsum_off, part_off, ws_bytes;  // workspace carve-up
-  int part_stride;   // floats per partial record
+  int smem_bytes;    // dynamic shared memory of the split kernel
+  size_t frag_off, part_off, ws_bytes;  // workspace carve-up: folded-query fragments, partial records
+  int part_stride;   // floats per partial record (multiple of 4)
 };
 DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq);
 cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,

@@ -27,7 +27,8 @@ struct SideDev {
   int32_t n_groups;  // kept groups
   int32_t n_kept;    // kept coordinates = group * n_groups
   int32_t c_col0;    // first column of this (head, side) in the latent matrix [T][n_eff]
-  int32_t wup_off;   // offset (floats) of W_up rows [n_kept][d_head] in the codec buffer
+  int32_t wup_off;   // offset (floats) of this side's W_up in the codec buffer:
+                     // V side rows [n_kept][d_head], K side transposed [d_head][n_kept]
   GroupDev grp[kMaxGroups];
 };
 

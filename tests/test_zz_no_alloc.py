@@ -73,7 +73,8 @@ def test_noalloc_rejects_scratch_beyond_its_limit():
 
     import spectral_transform_coding_b200 as st
 
-    shape = (256, 8, 1, 64, 32, 8, [[4, 2, 1, 1], [4, 2, 1, 1]], 64, [1] * 1000)
+    # 200 sequences x 64 q heads x (2 + 128) floats of split partials > 4 MiB
+    shape = (256, 64, 8, 128, 128, 16, [[4, 2, 2, 2, 2, 2, 1, 1], [4, 3, 2, 2, 2, 1, 1, 1]], 64, [1] * 200)
     codec, cache, q = _case(5, shape)
     out = torch.empty_like(q)
     d = cache.desc()
