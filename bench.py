@@ -51,18 +51,21 @@ def _workload_name(cfg, layers):
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same workload)
 # ---------------------------------------------------------------------------
-def cpu_oracle_sample(cfg, target_s=12.0):
+TRAFFIC_PER_ALGO_BYTE = {"llama": 33_888_768 / (32_772 * 1024)}
+
+
+def _oracle_decode_case(cfg, n_tok=8192):
+    """One KV head of the workload's layer for the CPU oracle: widths from the
+    workload's spectrum, a packed pool of ``n_tok`` seeded tokens, W_up, queries."""
     import numpy as np
 
     import oracle
-    from workloads import get_config
 
     rng = np.random.default_rng(cfg.seed)
     s2 = np.arange(1, cfg.rank + 1) ** -cfg.spectrum_exp
     widths = oracle.allocate_widths(s2, cfg.group, cfg.budget_bits, cfg.count_overhead)
     w1 = [[widths, widths]]
     P = cfg.page_tokens
-    n_tok = 8192
     lay = oracle.page_layout(w1, cfg.group, P)
     pool = np.zeros(lay["page_bytes"] * (n_tok // P), np.uint8)
     table = np.arange(n_tok // P)[None, :]
@@ -73,20 +76,64 @@ def cpu_oracle_sample(cfg, target_s=12.0):
     q, _ = np.linalg.qr(rng.standard_normal((cfg.d_head, cfg.d_head)))
     W_up = [[q[:nk].astype(np.float32), q[:nk].astype(np.float32)]]
     qs = rng.standard_normal((1, cfg.gq, cfg.d_head)).astype(np.float32)
+
+    def run(tokens):
+        oracle.decode_reference(pool, lay["page_bytes"], lay, cfg.group, P, table, np.array([tokens]), qs,
+                                W_up, cfg.gq, 1)
+    return run, n_tok
+
+
+def _blas_threads():
+    # numpy runs the unpacking and softmax on one thread; only the BLAS matmuls
+    # (rebuilding K and V from the latents) fan out, to the BLAS pool's threads
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
+    except Exception:
+        return 1
+
+
+def _sample_text(cfg, tokens, what):
+    return (f"oracle decode of 1 KV head ({cfg.gq} q heads) over {tokens} of {cfg.cache_len} context tokens "
+            f"of one {cfg.name} layer, {what}; numpy float64, unpacking on one thread, BLAS matmuls on "
+            f"{_blas_threads()} threads of {os.cpu_count()} host cores")
+
+
+def cpu_oracle_sample(cfg, target_s=12.0):
+    """The oracle's decode throughput over a bounded sample (about ``target_s`` s)."""
+    run, n_tok = _oracle_decode_case(cfg)
     t0 = time.perf_counter()
     reps = 0
     while True:
-        oracle.decode_reference(pool, lay["page_bytes"], lay, cfg.group, P, table, np.array([n_tok]), qs,
-                                W_up, cfg.gq, 1)
+        run(n_tok)
         reps += 1
         el = time.perf_counter() - t0
         if el >= target_s:
             break
     value = reps * n_tok / el  # tokens/s/head (one KV head per pass)
-    cores = os.cpu_count() or 1
-    sample = (f"oracle decode of 1 KV head ({cfg.gq} q heads) over {n_tok} of {cfg.cache_len} context tokens "
-              f"of one {cfg.name} layer, {reps} passes in {el:.1f} s")
-    return value, cores, sample
+    return value, _blas_threads(), _sample_text(cfg, n_tok, f"{reps} passes in {el:.1f} s")
+
+
+def cpu_oracle_steps(cfg, steps, warm, budget_s=120.0):
+    """The oracle as the reference arm: ``warm`` untimed and ``steps`` timed steps,
+    each the decode of one KV head over a context sample sized so that the whole
+    run takes about ``budget_s`` seconds."""
+    run, n_max = _oracle_decode_case(cfg)
+    P = cfg.page_tokens
+    t0 = time.perf_counter()
+    run(n_max)
+    t_full = time.perf_counter() - t0
+    per_step = budget_s / max(1, steps + warm)
+    n_tok = int(n_max * per_step / max(t_full, 1e-9)) // P * P
+    n_tok = max(P, min(n_max, n_tok))
+    for _ in range(warm):
+        run(n_tok)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        run(n_tok)
+    el = time.perf_counter() - t0
+    value = steps * n_tok / el
+    return value, el / steps * 1e3, _blas_threads(), _sample_text(cfg, n_tok, f"{steps} timed steps in {el:.1f} s")
 
 
 # ---------------------------------------------------------------------------
@@ -304,7 +351,11 @@ def run_gpu(args, rank, world):
     value = tok_per_step / (ms_per_step / 1e3) * world
     e2e_value = tok_per_step / (e2e_ms / 1e3) * world
 
-    # roofline: packed bytes the decode reads per layer
+    # roofline: packed bytes the decode reads per layer.  traffic: DRAM bytes
+    # (read + write) of one split_kernel launch per algorithmic byte, from one ncu
+    # capture of the 1-layer Llama-shaped case at 32k context (33,888,768 B for
+    # 32,772 tokens x 1,024 B); only workloads with a capture of the current kernel
+    # have one, else traffic is null.
     bytes_per_tok_all_heads = codecs[0].page_bytes / P
     dec_bytes = B * len_after * bytes_per_tok_all_heads
     dec_avg_ms = dec_ms
@@ -338,7 +389,9 @@ def run_gpu(args, rank, world):
             "kernel": "split_kernel (latent flash-decode over the packed pages), timed with its fold and combine "
                       "launches chained by programmatic dependent launch",
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "frac": achieved / peaks["hbm_gbs"],
+            "traffic": (TRAFFIC_PER_ALGO_BYTE[args.workload] * dec_bytes
+                        if args.workload in TRAFFIC_PER_ALGO_BYTE else None),
             "peak_src": peaks["src"], "avg_launch_us": dec_avg_ms * 1e3,
             "algorithmic_bytes_per_launch": dec_bytes,
         },
@@ -368,11 +421,12 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        value, cores, sample = cpu_oracle_sample(cfg, target_s=max(3.0, min(30.0, 2.0 * args.steps)))
+        value, ms, cores, sample = cpu_oracle_steps(cfg, args.steps, args.warmup)
         L = args.layers or MODEL_LAYERS[args.workload]
         out = {
             "impl": "reference", "metric": "latent-KV decode attention: cache tokens/s/head", "value": value,
             "unit": "tokens/s/head", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": _workload_name(cfg, L)},
             "cpu_baseline": {"value": value, "unit": "tokens/s/head", "cores": cores, "kind": "oracle",

@@ -44,14 +44,14 @@ def test_quantize_append_bit_exact(name):
     import spectral_transform_coding_b200 as st
     s = _setup(name)
     codec, P = s["codec"], s["P"]
-    cache = st.LatentCache(codec, batch=2, max_pages_per_seq=6, device=dev())
+    table = np.arange(12, dtype=np.int32)[::-1].reshape(2, 6).copy()  # host-built page table
+    cache = st.LatentCache(codec, batch=2, max_pages_per_seq=6, device=dev(), page_table=torch.from_numpy(table))
     # sequence 0 gets 150 tokens, sequence 1 gets 37, then a second call appends
     # 21 + 5 more at unaligned positions
     seqs1 = np.array([0] * 150 + [1] * 37, np.int32)
     seqs2 = np.array([0] * 21 + [1] * 5, np.int32)
     lat1 = synthetic_latents(len(seqs1), codec.n_eff, seed=1)
     lat2 = synthetic_latents(len(seqs2), codec.n_eff, seed=2, scale=30.0)
-    table = cache.page_table.cpu().numpy()
     ref = None
     lengths = np.zeros(2, np.int64)
     for seqs, lat in ((seqs1, lat1), (seqs2, lat2)):
@@ -71,8 +71,8 @@ def test_single_token_decode_steps_bit_exact():
     s = _setup("llama4x")
     codec, P = s["codec"], s["P"]
     B = 3
-    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=2, device=dev())
-    table = cache.page_table.cpu().numpy()
+    table = np.arange(B * 2, dtype=np.int32).reshape(B, 2)
+    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=2, device=dev(), page_table=torch.from_numpy(table))
     ref = np.zeros(cache.pool.numel(), np.uint8)
     lengths = np.zeros(B, np.int64)
     seqs = np.arange(B, dtype=np.int32)
@@ -136,16 +136,22 @@ def _decode_case(name, lengths, seed=0, peaked=False, P_pages=None):
     cache = st.LatentCache(codec, batch=B, max_pages_per_seq=maxp, device=dev(),
                            page_table=torch.from_numpy(perm))
     seqs = np.concatenate([np.full(L, b, np.int32) for b, L in enumerate(lengths)])
+    # the oracle builds its own pool from the same latents; the GPU pool must
+    # equal it byte for byte, and the oracle attends over its own copy
+    pool_ref = np.zeros(cache.pool.numel(), np.uint8)
+    lay = oracle.page_layout(oracle_widths(s["widths"]), s["group"], P)
     if seqs.size:
         lat = synthetic_latents(seqs.size, codec.n_eff, seed=seed + 11, decay=0.5, scale=2.0)
         codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+        pool_ref, _, lay = oracle_pool_after({"group": s["group"]}, s["widths"], cache.pool.numel(),
+                                             codec.page_bytes, perm, np.zeros(B), seqs, lat, P)
     q = rng.standard_normal((B, s["n_q"], s["d_h"])).astype(np.float32) * 0.6
     if peaked:
         q *= 6.0
     out = codec.decode_attend(cache, torch.from_numpy(q).to(dev()))
     codec.device_status()
-    lay = oracle.page_layout(oracle_widths(s["widths"]), s["group"], P)
-    ref = oracle.decode_reference(cache.pool.cpu().numpy(), codec.page_bytes, lay, s["group"], P, perm,
+    assert np.array_equal(cache.pool.cpu().numpy(), pool_ref), "packed cache differs from the oracle's"
+    ref = oracle.decode_reference(pool_ref, codec.page_bytes, lay, s["group"], P, perm,
                                   np.array(lengths), q, kept_wup(s["W_up"], s["widths"], s["group"]),
                                   s["n_q"], s["n_kv"])
     got = out.cpu().numpy()
@@ -180,8 +186,15 @@ def test_decode_many_sequences_stress_shape():
 
 
 def test_toy_end_to_end_calibrate_encode_decode():
-    """fp32 calibration on the toy layer, bf16 encode, decode; codes bit-exact vs
-    the oracle's quantisation of the GPU latents; calibration close to the oracle's."""
+    """Toy layer end to end, each side on its own from the same H, W_K, W_V, q.
+
+    The library calibrates (fp32), encodes (bf16 projection, quantise, pack) and
+    decodes.  The oracle runs its own calibration, projects through its W_down
+    rounded to bf16 (the precision the library stores it in), quantises and
+    attends exactly.  Calibration and latents must agree closely (latents within
+    1e-3).  Codes may differ where the two sides' latents straddle a rounding
+    boundary, so the attention bound here is an integration bound of 1e-2; the
+    strict 2e-3 on identical caches is held by the decode parity tests."""
     torch = torch_mod()
     import spectral_transform_coding_b200 as st
     cfgw = get_config("toy")
@@ -199,28 +212,29 @@ def test_toy_end_to_end_calibrate_encode_decode():
         V_gpu = state["W_up"][0, sidx].T.astype(np.float64)
         # leading directions agree (sign fixed)
         assert np.abs(V_gpu[:, :8] - hs["V"][:, :8]).max() < 1e-3
-    # encode + decode through the C ABI
-    n = cfgw.cache_len
+    widths_or = np.array([[ref["heads"][0]["K"]["widths"], ref["heads"][0]["V"]["widths"]]], np.int32)
+    # encode through the C ABI
+    n, P = cfgw.cache_len, cfgw.page_tokens
     h = bf16_round(make_activations(cfgw, n, stream=3))
-    cache = st.LatentCache(codec, batch=1, max_pages_per_seq=n // cfgw.page_tokens, device=dev())
+    table = np.arange(n // P, dtype=np.int32).reshape(1, n // P)
+    cache = st.LatentCache(codec, batch=1, max_pages_per_seq=n // P, device=dev(),
+                           page_table=torch.from_numpy(table))
     lat = torch.empty((n, codec.n_eff), dtype=torch.float32, device=dev())
     codec.encode_append(cache, torch.from_numpy(h).to(dev()).to(torch.bfloat16),
                         torch.zeros(n, dtype=torch.int32, device=dev()), latents_out=lat)
     codec.device_status()
-    lat_np = lat.cpu().numpy()
-    s = dict(n_kv=1, group=cfgw.group, widths=state["widths"])
-    _check_latents(lat_np, h.astype(np.float64) @ state["W_down"].astype(np.float64), s)
-    table = cache.page_table.cpu().numpy()
-    pool_ref, _, lay = oracle_pool_after({"group": cfgw.group}, state["widths"], cache.pool.numel(),
-                                         codec.page_bytes, table, np.zeros(1), np.zeros(n, np.int64), lat_np,
-                                         cfgw.page_tokens)
-    assert np.array_equal(cache.pool.cpu().numpy(), pool_ref)
+    # the oracle's own encode
+    lat_or = h.astype(np.float64) @ bf16_round(ref["W_down"].astype(np.float32)).astype(np.float64)
+    _check_latents(lat.cpu().numpy(), lat_or, dict(n_kv=1, group=cfgw.group, widths=widths_or))
+    pool_or, _, lay = oracle_pool_after({"group": cfgw.group}, widths_or, cache.pool.numel(), codec.page_bytes,
+                                        table, np.zeros(1), np.zeros(n, np.int64), lat_or.astype(np.float32), P)
+    # decode on both sides
     q = make_queries(cfgw, 1)
     out = codec.decode_attend(cache, torch.from_numpy(q).to(dev())).cpu().numpy()
-    ref_o = oracle.decode_reference(pool_ref, codec.page_bytes, lay, cfgw.group, cfgw.page_tokens, table,
-                                    np.array([n]), q, kept_wup(state["W_up"], state["widths"], cfgw.group),
-                                    cfgw.n_q_heads, 1)
-    assert attention_rel_err(out, ref_o) <= 2e-3
+    W_up_or = [[ref["heads"][0]["K"]["W_up"], ref["heads"][0]["V"]["W_up"]]]
+    ref_o = oracle.decode_reference(pool_or, codec.page_bytes, lay, cfgw.group, P, table, np.array([n]), q,
+                                    W_up_or, cfgw.n_q_heads, 1)
+    assert attention_rel_err(out, ref_o) <= 1e-2
 
 
 def test_calibrate_bf16_llama_shaped_head():

@@ -12,5 +12,7 @@ from .synthetic import (  # noqa: F401
     make_layer,
     make_queries,
     make_weights,
+    random_factors,
     spawn,
+    synthetic_latents,
 )

@@ -146,3 +146,35 @@ def make_layer(cfg: WorkloadConfig, calib_tokens: int | None = None) -> dict:
     n = cfg.calib_tokens if calib_tokens is None else calib_tokens
     w["H_calib"] = make_activations(cfg, n, STREAM_CALIB)
     return w
+
+
+# ----------------------------------------------------------------------------
+# Inputs of the library-level parity checks: codec factors and latents drawn
+# directly (no calibration), so both sides start from identical numbers.
+# ----------------------------------------------------------------------------
+
+def random_factors(d_model, n_kv, d_h, rank, group, widths, seed=0, w_std=0.02):
+    """Seeded W_down (bf16 values) for the kept columns and orthonormal W_up rows."""
+    rng = np.random.default_rng(seed)
+    ng = rank // group
+    widths = np.asarray(widths, np.int32).reshape(n_kv, 2, ng)
+    n_eff = int(sum(group for a in range(n_kv) for s in range(2) for b in widths[a, s] if b > 0))
+    W_down = bf16_round((rng.standard_normal((d_model, max(n_eff, 1))) * w_std).astype(np.float32))
+    W_down = W_down[:, :n_eff]
+    W_up = np.zeros((n_kv, 2, rank, d_h), np.float32)
+    for a in range(n_kv):
+        for s in range(2):
+            q, _ = np.linalg.qr(rng.standard_normal((d_h, d_h)))
+            W_up[a, s] = q[:, :rank].T.astype(np.float32)
+    return widths, W_down, W_up
+
+
+def synthetic_latents(T, n_eff, seed, decay=0.7, scale=1.0):
+    """fp32 latents with a decaying per-column scale and a few exact ties/constants."""
+    rng = np.random.default_rng(seed)
+    col_scale = scale * (np.arange(n_eff) % 128 + 1.0) ** -decay
+    x = (rng.standard_normal((T, n_eff)) * col_scale[None, :]).astype(np.float32)
+    if T > 3 and n_eff >= 16:
+        x[1, :16] = 0.25   # a constant group (scale 0)
+        x[2, :16] = np.float32(1e-8) * np.arange(16, dtype=np.float32)  # a subnormal-scale group
+    return x
