@@ -37,26 +37,30 @@
  * codes are appended per token with one width per group):
  *   A page holds P = page_tokens tokens of one sequence for every KV head.
  *   page = head sections a = 0..n_kv_heads-1; head section = K side then V side;
- *   side section = for each group j with b_j > 0, ascending:
- *       b_j bit-planes (plane p = bit p of every code, p = 0 first), each
- *       P*g/8 bytes, then P/2 records of 8 bytes:
- *       fp16 {s[2u], s[2u+1], z[2u], z[2u+1]} (little-endian).
- *   A bit-plane is a run of 256-bit blocks (8 little-endian uint32 words), one
- *   per 256/g consecutive tokens.  Entry (token tau of the block, coordinate k
- *   of the group) sits at word `word`, bit `4*slot + t4`, where
+ *   side section = for each group j with b_j > 0, ascending: its code blocks
+ *   (P*g*b_j/8 bytes), then its P/2 scale/zero records of 8 bytes.
+ *   Code blocks: one block per 256/g consecutive tokens, 8*b_j little-endian
+ *   uint32 words.  Entry (token tau of the block, coordinate k of the group) has
+ *   a fragment position (gid, t4, slot), gid 0..7, t4 0..3, slot 0..7:
  *     g = 16: K side row = tau/2 (tau even) or 8 + tau/2 (tau odd), col = k;
  *             V side row = k, col = tau;
- *             word = row % 8, t4 = (col % 8)/2,
- *             slot = row/8 + 2*(col/8) + 4*(col % 2);
+ *             gid = row % 8, t4 = (col % 8)/2, slot = row/8 + 2*(col/8) + 4*(col % 2);
  *     g = 8 (32-token blocks; mi = tau/16, tl = tau%16):
- *             K side row from tl as above, word = row % 8, t4 = k/2,
+ *             K side row from tl as above, gid = row % 8, t4 = k/2,
  *                    slot = row/8 + 2*mi + 4*(k % 2);
- *             V side word = k, t4 = (tl % 8)/2,
- *                    slot = mi + 2*(tl/8) + 4*(tl % 2).
- *   (This places, after one rotate per plane, each lane's codes of an
- *   mma.sync A fragment into 4-bit fields.)  A page therefore takes exactly
- *   P * sum over kept groups of (g*b_j + 32)/8 bytes; all offsets are multiples
- *   of 16 bytes.
+ *             V side gid = k, t4 = (tl % 8)/2, slot = mi + 2*(tl/8) + 4*(tl % 2).
+ *   Code bit p of the entry sits at (word, bit):
+ *     b = 4: word 4*gid + t4, bit 4*slot + p;
+ *     b = 2: word 2*gid + t4/2, bit 4*slot + 2*(t4 % 2) + p;
+ *     b = 1: word gid, bit 4*slot + t4;
+ *     b = 3: bits 0-1 as for b = 2 (words 0..15), bit 2 as for b = 1 in word 16 + gid;
+ *     b = 8: word 2*(4*gid + t4) + (slot/2) % 2, bit 8*((slot % 2) + 2*(slot/4)) + p.
+ *   (Lane gid*4 + t4 of an mma.sync A fragment thus finds its 8 codes in one or
+ *   two words; slot r and r+4 form fragment register r.)
+ *   Records: fp16 {s[2u], s[2u+1], z[2u], z[2u+1]} (little-endian) of the token
+ *   pair u (tokens 2u, 2u+1 of the page) at record index (u % 8)*(P/16) + u/8.
+ *   A page therefore takes exactly P * sum over kept groups of (g*b_j + 32)/8
+ *   bytes; all offsets are multiples of 16 bytes.
  *
  * Quantiser (per token, per kept group of g fp32 latents, every step one IEEE
  * fp32 operation): s = fp16_rn(sat((max - min) / (2^b - 1))), z = fp16_rn(sat(min)),
@@ -303,7 +307,7 @@ SPECTRA_API spectra_status spectra_sym_eigen(const double* M, int32_t n, double*
 
 /* Page size and group placement for given widths ([n_kv_heads][2][rank/group]).
  * offsets (may be NULL) receives, per (head, side, group), the byte offset of
- * the group's first bit-plane in the page (-1 for dropped groups), followed by
+ * the group's first code block in the page (-1 for dropped groups), followed by
  * the same count of record offsets. */
 SPECTRA_API spectra_status spectra_page_layout(const spectra_config* cfg, const int32_t* widths,
                                    int64_t* page_bytes, int64_t* offsets);

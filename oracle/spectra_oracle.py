@@ -336,12 +336,26 @@ def quantize_side(c: np.ndarray, widths, g: int) -> list:
 #
 # A page holds P tokens of one sequence for every KV head.  Page = head sections
 # a = 0..H_kv-1; head section = K section then V section; a side section = for
-# each group with b > 0, in ascending group order: b bit-planes (plane p holds
-# bit p of every code; p = 0 first), each P*g/8 bytes, then P/2 records of 8
-# bytes (fp16 s[2u], s[2u+1], z[2u], z[2u+1]).  A bit-plane is a run of blocks
-# of 256 bits (8 little-endian uint32 words) covering 256/g consecutive tokens;
-# ``block_bit_address`` places entry (token tau in the block, coordinate k in
-# the group) at (word, bit).
+# each group with b > 0, in ascending group order: its code blocks, then its
+# scale/zero records.
+#
+# Code blocks.  A block holds the codes of 256/g consecutive tokens of one group
+# (256 entries, b*32 bytes = 8*b little-endian uint32 words); blocks follow token
+# order, P*g/256 of them per page.  Entry (token tau of the block, coordinate k)
+# has a fragment position (gid, t4, slot): 32 "lanes" gid*4 + t4 (gid 0..7,
+# t4 0..3) with 8 slots each (``fragment_position``).  Its code bit p is stored
+# at (word, bit) = ``code_bit_address``:
+#   b = 4: word 4*gid + t4, bit 4*slot + p (each lane's 8 codes are one word
+#          of nibbles);
+#   b = 2: word 2*gid + t4//2, bit 4*slot + 2*(t4 % 2) + p;
+#   b = 1: word gid, bit 4*slot + t4;
+#   b = 3: bits 0-1 as for b = 2 (words 0..15), bit 2 as for b = 1 in words
+#          16 + gid;
+#   b = 8: word 2*(4*gid + t4) + (slot // 2) % 2, bit 8*((slot % 2) + 2*(slot // 4)) + p.
+#
+# Records.  P/2 records of 8 bytes, fp16 {s[2u], s[2u+1], z[2u], z[2u+1]} for the
+# token pair u (tokens 2u, 2u+1 of the page).  With 16-token tiles, pair u is
+# pair u % 8 of tile u // 8 and sits at record index (u % 8) * (P/16) + u // 8.
 
 def tokens_per_block(g: int) -> int:
     if g not in (8, 16):
@@ -349,40 +363,65 @@ def tokens_per_block(g: int) -> int:
     return 256 // g
 
 
-def block_bit_address(g: int, side: str, tau: int, k: int) -> tuple[int, int]:
-    """(word, bit) of entry (token tau, group coordinate k) inside a 256-bit block."""
+def fragment_position(g: int, side: str, tau: int, k: int) -> tuple[int, int, int]:
+    """(gid, t4, slot) of entry (token tau in the block, coordinate k in the group)."""
     if g == 16:
         if side == "K":
             row = tau // 2 if tau % 2 == 0 else 8 + tau // 2
             col = k
         else:
             row, col = k, tau
-        word, hh = row % 8, row // 8
+        gid, hh = row % 8, row // 8
         t4, cp, ch = (col % 8) // 2, col % 2, col // 8
         slot = hh + 2 * ch + 4 * cp
     elif g == 8:
         mi, tl = tau // 16, tau % 16
         if side == "K":
             row = tl // 2 if tl % 2 == 0 else 8 + tl // 2
-            word, hh = row % 8, row // 8
+            gid, hh = row % 8, row // 8
             t4, cp = k // 2, k % 2
             slot = hh + 2 * mi + 4 * cp
         else:
-            word = k
+            gid = k
             t4, cp, ch = (tl % 8) // 2, tl % 2, tl // 8
             slot = mi + 2 * ch + 4 * cp
     else:
         raise ValueError("group must be 8 or 16")
-    return word, 4 * slot + t4
+    return gid, t4, slot
 
 
-def _address_table(g: int, side: str) -> tuple[np.ndarray, np.ndarray]:
+def code_bit_address(g: int, side: str, b: int, tau: int, k: int, p: int) -> tuple[int, int]:
+    """(word, bit) inside a block of code bit p of entry (tau, k) of a width-b group."""
+    if not 0 <= p < b:
+        raise ValueError("bit index out of range")
+    gid, t4, slot = fragment_position(g, side, tau, k)
+    if b == 4:
+        return 4 * gid + t4, 4 * slot + p
+    if b == 2 or (b == 3 and p < 2):
+        return 2 * gid + t4 // 2, 4 * slot + 2 * (t4 % 2) + p
+    if b == 1:
+        return gid, 4 * slot + t4
+    if b == 3:
+        return 16 + gid, 4 * slot + t4
+    if b == 8:
+        return 2 * (4 * gid + t4) + (slot // 2) % 2, 8 * ((slot % 2) + 2 * (slot // 4)) + p
+    raise ValueError("width must be 1, 2, 3, 4 or 8")
+
+
+def record_index(P: int, tau: int) -> int:
+    """Record index of page token tau's pair (see the layout statement above)."""
+    u = tau // 2
+    return (u % 8) * (P // 16) + u // 8
+
+
+def _address_table(g: int, side: str, b: int) -> tuple[np.ndarray, np.ndarray]:
     tb = tokens_per_block(g)
-    words = np.zeros((tb, g), dtype=np.int64)
-    bits = np.zeros((tb, g), dtype=np.int64)
-    for tau in range(tb):
-        for k in range(g):
-            words[tau, k], bits[tau, k] = block_bit_address(g, side, tau, k)
+    words = np.zeros((b, tb, g), dtype=np.int64)
+    bits = np.zeros((b, tb, g), dtype=np.int64)
+    for p in range(b):
+        for tau in range(tb):
+            for k in range(g):
+                words[p, tau, k], bits[p, tau, k] = code_bit_address(g, side, b, tau, k, p)
     return words, bits
 
 
@@ -395,7 +434,7 @@ def page_layout(codec_widths, g: int, P: int) -> dict:
 
     ``codec_widths[a][side_index]`` is the width vector of head a, side K (0) or
     V (1).  Returns dict(page_bytes, groups) with groups[(a, s)] = list of
-    (b, plane_offset, sz_offset, latent_col) for the non-empty groups.
+    (b, block_offset, record_offset, latent_col) for the non-empty groups.
     """
     if P % 32:
         raise ValueError("page_tokens must be a multiple of 32")
@@ -427,38 +466,40 @@ def pack_group_into_page(page: np.ndarray, g: int, side: str, P: int, b: int,
     Bits of those tokens are cleared first, then set; other tokens are untouched.
     """
     tb = tokens_per_block(g)
-    wtab, btab = _address_table(g, side)
-    words = page[plane_off: plane_off + b * P * g // 8].view("<u4").reshape(b, P // tb, 8)
+    wtab, btab = _address_table(g, side, b)
+    words = page[plane_off: plane_off + b * P * g // 8].view("<u4").reshape(P // tb, 8 * b)
     t = np.asarray(tokens, dtype=np.int64)
     blk = np.repeat((t // tb)[:, None], g, axis=1)
-    w = wtab[t % tb]
-    bit = btab[t % tb].astype(np.uint32)
-    one = np.left_shift(np.uint32(1), bit)
     c = np.asarray(codes, dtype=np.uint32)
     for p in range(b):
-        np.bitwise_and.at(words[p], (blk, w), np.invert(one))
+        w = wtab[p][t % tb]
+        bit = btab[p][t % tb].astype(np.uint32)
+        one = np.left_shift(np.uint32(1), bit)
+        np.bitwise_and.at(words, (blk, w), np.invert(one))
         v = (np.right_shift(c, np.uint32(p)) & np.uint32(1)) << bit
-        np.bitwise_or.at(words[p], (blk, w), v.astype(np.uint32))
+        np.bitwise_or.at(words, (blk, w), v.astype(np.uint32))
     rec = page[sz_off: sz_off + 4 * P].view("<f2").reshape(P // 2, 4)
-    rec[t // 2, t % 2] = np.asarray(s16, dtype=np.float16)
-    rec[t // 2, 2 + t % 2] = np.asarray(z16, dtype=np.float16)
+    ridx = ((t // 2) % 8) * (P // 16) + (t // 2) // 8  # record_index, vectorised
+    rec[ridx, t % 2] = np.asarray(s16, dtype=np.float16)
+    rec[ridx, 2 + t % 2] = np.asarray(z16, dtype=np.float16)
 
 
 def unpack_group_from_page(page: np.ndarray, g: int, side: str, P: int, b: int,
                            plane_off: int, sz_off: int, n_tokens: int):
     """Read codes[n_tokens, g], s[n_tokens], z[n_tokens] of a group back from a page."""
     tb = tokens_per_block(g)
-    wtab, btab = _address_table(g, side)
-    words = page[plane_off: plane_off + b * P * g // 8].view("<u4").reshape(b, P // tb, 8)
+    wtab, btab = _address_table(g, side, b)
+    words = page[plane_off: plane_off + b * P * g // 8].view("<u4").reshape(P // tb, 8 * b)
     t = np.arange(n_tokens)
     blk, tau = t // tb, t % tb
     codes = np.zeros((n_tokens, g), dtype=np.int64)
     for p in range(b):
-        wsel = words[p][blk[:, None], wtab[tau]]
-        codes |= ((wsel.astype(np.int64) >> btab[tau]) & 1) << p
+        wsel = words[blk[:, None], wtab[p][tau]]
+        codes |= ((wsel.astype(np.int64) >> btab[p][tau]) & 1) << p
     rec = page[sz_off: sz_off + 4 * P].view("<f2").reshape(P // 2, 4)
-    s = np.where(t % 2 == 0, rec[t // 2, 0], rec[t // 2, 1]).astype(np.float16)
-    z = np.where(t % 2 == 0, rec[t // 2, 2], rec[t // 2, 3]).astype(np.float16)
+    ridx = ((t // 2) % 8) * (P // 16) + (t // 2) // 8  # record_index, vectorised
+    s = rec[ridx, t % 2].astype(np.float16) if n_tokens else np.zeros(0, np.float16)
+    z = rec[ridx, 2 + t % 2].astype(np.float16) if n_tokens else np.zeros(0, np.float16)
     return codes.astype(np.uint8), s, z
 
 

@@ -40,20 +40,20 @@ namespace {
 constexpr int kDecWarps = 4;
 constexpr int kMaxG = 8;          // kept groups per side handled by the decode kernels
 constexpr int kMaxKept = 128;     // kept coordinates per side
-constexpr int kChunk = 4;         // 16-token tiles per softmax chunk
 constexpr int kMaxSplit = 256;    // context splits per (sequence, KV head)
 constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // bounded mbarrier waits
 constexpr float kPScaleLog2 = 8.f;   // p = 2^(s - m + 8): fp16 keeps small weights normal
 constexpr float kTwo24 = 16777216.f; // undo the 2^-24 of subnormal codes
+constexpr float kTwo20 = 1048576.f;  // the same for codes held at nibble bits 4-7 (x16)
 constexpr int kFragWords = (kMaxG * 2 + 2) * 32;  // uint2 per (sequence, KV head): bq[j][nt], bz[nt]
 
 // split kernel shared-memory carve-up (bytes)
 constexpr int kSmBars = 0;                                   // 4 warps x 8 mbarriers
 constexpr int kSmBq = 512;                                   // fragments [kMaxG*2 + 2][32] uint2
-constexpr int kSmGrp = kSmBq + kFragWords * 8;               // int4 {plane, rec, b, -} x (K 8, V 8)
-constexpr int kSmMisc = kSmGrp + 2 * kMaxG * 16;             // 32 ints
-constexpr int kSmAcc = kSmMisc + 128;                        // value accumulators [warp][kMaxG][32] float4
+constexpr int kSmGrp = kSmBq + kFragWords * 8;               // group tables (448 B)
+constexpr int kSmAcc = kSmGrp + 512;                         // value accumulators [warp][kMaxG][32] float4
 constexpr int kSmStages = kSmAcc + kDecWarps * kMaxG * 32 * 16;
+constexpr int kMergeBytes = (kDecWarps * kMaxGQ * (2 + kMaxKept) + kMaxGQ * (kDecWarps + 2)) * 4;
 
 struct DecodeArgs {
   const CodecDev* cd;
@@ -97,53 +97,12 @@ __device__ __forceinline__ void mma_m16n8k8_z(float d[4], const uint32_t a[2], u
       : "r"(a[0]), "r"(a[1]), "r"(b), "f"(z));
 }
 
-// Codes of one group into 4-bit fields: rotating plane p's word right by
-// (t4 - p mod 4) places this lane's 8 bits of the block at bits 4*slot + p mod 4;
-// planes 0-3 fill `lo`, planes 4-7 fill `hi`.
-template <int B>
-__device__ __forceinline__ void gather_fixed(const uint8_t* pw, int stride, const uint32_t (&rot)[4],
-                                             uint32_t& lo, uint32_t& hi) {
-  lo = 0u;
-  hi = 0u;
-#pragma unroll
-  for (int p = 0; p < B; ++p) {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(pw + p * stride);
-    const uint32_t r = __funnelshift_r(w, w, rot[p & 3]);
-    if (p < 4) lo |= r & (0x11111111u << p);
-    else hi |= r & (0x11111111u << (p - 4));
-  }
-}
-
-// Element pair (slot i, slot i+4) as two 16-bit integers: as fp16 bit patterns
-// these are the subnormals code * 2^-24.
-__device__ __forceinline__ uint32_t slot_pair(uint32_t lo, uint32_t hi, int i, bool wide) {
-  uint32_t v = (lo >> (4 * i)) & 0x000F000Fu;
-  if (wide) v |= ((hi >> (4 * i)) & 0x000F000Fu) << 4;
-  return v;
-}
-
-template <int G>
-__device__ __forceinline__ void code_frag_k(uint32_t lo, uint32_t hi, bool wide, int mi, uint32_t (&av)[4]) {
-  if (G == 16) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = slot_pair(lo, hi, i, wide);
-  } else {  // m16n8k8: rows (gid, gid+8) of half mi
-    av[0] = slot_pair(lo, hi, 2 * mi, wide);
-    av[1] = slot_pair(lo, hi, 2 * mi + 1, wide);
-  }
-}
-
-template <int G>
-__device__ __forceinline__ void code_frag_v(uint32_t lo, uint32_t hi, bool wide, int mi, uint32_t (&av)[4]) {
-  if (G == 16) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = slot_pair(lo, hi, i, wide);
-  } else {  // m16n8k16 with coordinate rows 8..15 padded with zeros
-    av[0] = slot_pair(lo, hi, mi, wide);
-    av[1] = 0u;
-    av[2] = slot_pair(lo, hi, mi + 2, wide);
-    av[3] = 0u;
-  }
+// 2^x for x <= 0 (and up to 2^8 for the scaled softmax weights); flushes
+// results below 2^-126 to zero.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
@@ -233,66 +192,240 @@ __global__ void __launch_bounds__(256) fold_kernel(const DecodeArgs A) {
 // split: one context split of one (sequence, KV head)
 // ---------------------------------------------------------------------------
 
-// Keys of one group for the tiles of a chunk: s_j (q_lat,j . code_j) accumulated
-// into acc[tt][nt][hi/lo of token 2gid, hi/lo of token 2gid+1].
-template <int G, int NT, int B>
-__device__ __forceinline__ void key_group(const uint8_t* __restrict__ pbase, const uint8_t* __restrict__ rbase,
-                                          const uint2 (&bqj)[NT], int t0, int ntile, int plane_stride,
-                                          const uint32_t (&rot)[4], float (&acc)[kChunk][NT][4]) {
-#pragma unroll
-  for (int tt = 0; tt < kChunk; ++tt) {
-    if (tt < ntile) {
-      const int t = t0 + tt;
-      const int blk = (G == 16) ? t : (t >> 1);
-      const int mi = (G == 16) ? 0 : (t & 1);
-      uint32_t lo, hi;
-      gather_fixed<B>(pbase + blk * 32, plane_stride, rot, lo, hi);
-      const uint32_t s2 = *reinterpret_cast<const uint32_t*>(rbase + t * 64);
-      const float sA = half_lo(s2), sB = half_hi(s2);
-      uint32_t av[4];
-      code_frag_k<G>(lo, hi, B > 4, mi, av);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float d[4];
-        const uint32_t bb[2] = {bqj[nt].x, bqj[nt].y};
-        if (G == 16) mma_m16n8k16_z(d, av, bb);
-        else mma_m16n8k8_z(d, av, bb[0]);
-        acc[tt][nt][0] = fmaf(sA, d[0], acc[tt][nt][0]);
-        acc[tt][nt][1] = fmaf(sA, d[1], acc[tt][nt][1]);
-        acc[tt][nt][2] = fmaf(sB, d[2], acc[tt][nt][2]);
-        acc[tt][nt][3] = fmaf(sB, d[3], acc[tt][nt][3]);
-      }
-    }
-  }
+// Fragment registers of one 256-entry block of a group with width B.  The
+// block's bytes hold, for every MMA lane, its 8 codes (slots 0..7, see the page
+// layout): B = 4: word `lane` holds them as nibbles; B = 2: word 2*gid + t4/2,
+// bits 2*(t4%2) + {0,1} of each nibble; B = 1: word gid, bit t4 of each nibble;
+// B = 3: a B = 2 part (16 words, code bits 0-1) then a B = 1 part (8 words,
+// code bit 2); B = 8: words 2*lane, 2*lane+1 hold bytes [s0 s1 s4 s5] [s2 s3 s6 s7].
+// A nibble-held code is used in place: as an fp16 bit pattern, bits 0-3 of a
+// 16-bit lane are the subnormal code * 2^-24 and bits 4-7 are code * 16 * 2^-24.
+// So registers a1, a3 (MMA rows gid+8) carry a factor 16 for B <= 4.
+template <int B>
+__device__ __forceinline__ uint32_t nibble_codes(const uint8_t* __restrict__ p, const uint8_t* __restrict__ p1,
+                                                 uint32_t sh, uint32_t rot1) {
+  if (B == 4) return *reinterpret_cast<const uint32_t*>(p);
+  if (B == 2 || B == 1) return *reinterpret_cast<const uint32_t*>(p) >> sh;
+  // B == 3: code bits 0-1 from the 2-bit part, bit 2 from the 1-bit part (rotated
+  // from nibble bit t4 to nibble bit 2); bit 3 of each nibble is left as junk and
+  // cleared by the fragment masks
+  const uint32_t lo = *reinterpret_cast<const uint32_t*>(p) >> sh;
+  const uint32_t w1 = *reinterpret_cast<const uint32_t*>(p1);
+  const uint32_t hi = __funnelshift_r(w1, w1, rot1);
+  return (lo & 0x33333333u) | (hi & 0xCCCCCCCCu);
 }
 
-// Values of one group for the tiles of a chunk: va += code^T (p s) (codes as
-// subnormals, so va carries a factor 2^-24).
+template <int B>
+__device__ __forceinline__ constexpr uint32_t frag_mask() {
+  return B >= 4 ? 0x000F000Fu : (B == 3 ? 0x00070007u : (B == 2 ? 0x00030003u : 0x00010001u));
+}
+
+// K side, A = codes (rows: tokens, cols: coordinates).  G = 16: m16n8k16, four
+// registers; G = 8: m16n8k8, two registers for half `mi` of a 32-token block.
 template <int G, int B>
-__device__ __forceinline__ void value_group(const uint8_t* __restrict__ pbase, const uint8_t* __restrict__ rbase,
-                                            const uint32_t (&pb)[kChunk][2], const uint32_t (&msk)[kChunk][2],
-                                            int t0, int ntile, int plane_stride, const uint32_t (&rot)[4],
-                                            float (&va)[4]) {
-#pragma unroll
-  for (int tt = 0; tt < kChunk; ++tt) {
-    if (tt < ntile) {
-      const int t = t0 + tt;
-      const int blk = (G == 16) ? t : (t >> 1);
-      const int mi = (G == 16) ? 0 : (t & 1);
-      uint32_t lo, hi;
-      gather_fixed<B>(pbase + blk * 32, plane_stride, rot, lo, hi);
-      const uint8_t* rb = rbase + t * 64;
-      const uint32_t s0 = *reinterpret_cast<const uint32_t*>(rb) & msk[tt][0];
-      const uint32_t s1 = *reinterpret_cast<const uint32_t*>(rb + 32) & msk[tt][1];
-      const uint32_t bj[2] = {hmul2_u32(pb[tt][0], s0), hmul2_u32(pb[tt][1], s1)};
-      uint32_t av[4];
-      code_frag_v<G>(lo, hi, B > 4, mi, av);
-      mma_m16n8k16(va, av, bj);
+__device__ __forceinline__ void frag_k(const uint8_t* __restrict__ p, const uint8_t* __restrict__ p1, uint32_t sh,
+                                       uint32_t rot1, int mi, uint32_t (&av)[4]) {
+  if (B == 8) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    if (G == 16) {
+      av[0] = w.x & 0x00FF00FFu;
+      av[1] = (w.x >> 8) & 0x00FF00FFu;
+      av[2] = w.y & 0x00FF00FFu;
+      av[3] = (w.y >> 8) & 0x00FF00FFu;
+    } else {
+      const uint32_t x = mi ? w.y : w.x;
+      av[0] = x & 0x00FF00FFu;
+      av[1] = (x >> 8) & 0x00FF00FFu;
+    }
+  } else {
+    constexpr uint32_t M = frag_mask<B>();
+    const uint32_t x = nibble_codes<B>(p, p1, sh, rot1);
+    if (G == 16) {
+      const uint32_t y = x >> 8;
+      av[0] = x & M;
+      av[1] = x & (M << 4);
+      av[2] = y & M;
+      av[3] = y & (M << 4);
+    } else {
+      const uint32_t y = mi ? (x >> 8) : x;
+      av[0] = y & M;
+      av[1] = y & (M << 4);
     }
   }
 }
 
-template <int G, int NT>
+// V side, A = codes transposed (rows: coordinates, cols: tokens), m16n8k16.
+// G = 8: rows 8..15 are zero; no factor 16 (shifts instead).
+template <int G, int B>
+__device__ __forceinline__ void frag_v(const uint8_t* __restrict__ p, const uint8_t* __restrict__ p1, uint32_t sh,
+                                       uint32_t rot1, int mi, uint32_t (&av)[4]) {
+  if (B == 8) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    if (G == 16) {
+      av[0] = w.x & 0x00FF00FFu;
+      av[1] = (w.x >> 8) & 0x00FF00FFu;
+      av[2] = w.y & 0x00FF00FFu;
+      av[3] = (w.y >> 8) & 0x00FF00FFu;
+    } else {
+      av[0] = (mi ? (w.x >> 8) : w.x) & 0x00FF00FFu;
+      av[1] = 0u;
+      av[2] = (mi ? (w.y >> 8) : w.y) & 0x00FF00FFu;
+      av[3] = 0u;
+    }
+  } else {
+    constexpr uint32_t M = frag_mask<B>();
+    const uint32_t x = nibble_codes<B>(p, p1, sh, rot1);
+    if (G == 16) {
+      const uint32_t y = x >> 8;
+      av[0] = x & M;
+      av[1] = x & (M << 4);
+      av[2] = y & M;
+      av[3] = y & (M << 4);
+    } else {
+      const uint32_t xs = mi ? (x >> 4) : x;
+      av[0] = xs & M;
+      av[1] = 0u;
+      av[2] = (xs >> 8) & M;
+      av[3] = 0u;
+    }
+  }
+}
+
+// Lane-constant addressing of a width class: byte offset of this lane's word in
+// a block (and of its 1-bit-part word for B = 3), shift and rotation.
+struct LaneAddr {
+  int off4, off2, off1, off8;
+  uint32_t sh2, sh1, rot1;
+};
+
+template <int B>
+__device__ __forceinline__ int lane_off(const LaneAddr& L) {
+  return B == 4 ? L.off4 : (B == 8 ? L.off8 : ((B == 2 || B == 3) ? L.off2 : L.off1));
+}
+template <int B>
+__device__ __forceinline__ uint32_t lane_sh(const LaneAddr& L) {
+  return B == 1 ? L.sh1 : L.sh2;
+}
+
+// Keys of one kept group for the CH tiles of a chunk: acc[tt][nt] +=
+// s * (q_lat,j . code) for (token row gid, token row gid+8) x (hi, lo).
+// Rows gid+8 carry the factor 16 (B = 8 scales s instead).
+template <int G, int NT, int CH, int B>
+__device__ __forceinline__ void key_group(const uint8_t* __restrict__ blocks, const uint8_t* __restrict__ rec,
+                                          const LaneAddr& L, const uint2 (&bqj)[NT], float (&acc)[CH][NT][4]) {
+  const uint8_t* p = blocks + lane_off<B>(L);
+  const uint8_t* p1 = blocks + 64 + L.off1;
+  uint32_t sp[CH];
+#pragma unroll
+  for (int h = 0; h < CH / 2; ++h) {
+    const uint4 r = *reinterpret_cast<const uint4*>(rec + 16 * h);  // {s, z} of 2 tiles
+    sp[2 * h] = r.x;
+    sp[2 * h + 1] = r.z;
+  }
+#pragma unroll
+  for (int tt = 0; tt < CH; ++tt) {
+    constexpr int kBlockTiles = G == 16 ? 1 : 2;
+    const int blk = tt / kBlockTiles;
+    uint32_t av[4];
+    frag_k<G, B>(p + blk * (B * 32), p1 + blk * (B * 32), lane_sh<B>(L), L.rot1, tt & 1, av);
+    const float sA = __half2float(__ushort_as_half((unsigned short)(sp[tt] & 0xffffu)));
+    float sB = __half2float(__ushort_as_half((unsigned short)(sp[tt] >> 16)));
+    if (B == 8) sB *= 16.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float d[4];
+      const uint32_t bb[2] = {bqj[nt].x, bqj[nt].y};
+      if (G == 16) mma_m16n8k16_z(d, av, bb);
+      else mma_m16n8k8_z(d, av, bb[0]);
+      acc[tt][nt][0] = fmaf(sA, d[0], acc[tt][nt][0]);
+      acc[tt][nt][1] = fmaf(sA, d[1], acc[tt][nt][1]);
+      acc[tt][nt][2] = fmaf(sB, d[2], acc[tt][nt][2]);
+      acc[tt][nt][3] = fmaf(sB, d[3], acc[tt][nt][3]);
+    }
+  }
+}
+
+// Values of one kept group for the CH tiles of a chunk: va += code^T (p s).
+// recA / recB: this lane's records of token pairs t4 and t4+4.
+template <int G, int CH, int B, bool kMask>
+__device__ __forceinline__ void value_group(const uint8_t* __restrict__ blocks, const uint8_t* __restrict__ recA,
+                                            const uint8_t* __restrict__ recB, const LaneAddr& L,
+                                            const uint32_t (&pb)[CH][2], const uint32_t (&msk)[CH][2],
+                                            float (&va)[4]) {
+  const uint8_t* p = blocks + lane_off<B>(L);
+  const uint8_t* p1 = blocks + 64 + L.off1;
+  uint32_t s0[CH], s1[CH];
+#pragma unroll
+  for (int h = 0; h < CH / 2; ++h) {
+    const uint4 ra = *reinterpret_cast<const uint4*>(recA + 16 * h);
+    const uint4 rb = *reinterpret_cast<const uint4*>(recB + 16 * h);
+    s0[2 * h] = ra.x;
+    s0[2 * h + 1] = ra.z;
+    s1[2 * h] = rb.x;
+    s1[2 * h + 1] = rb.z;
+  }
+#pragma unroll
+  for (int tt = 0; tt < CH; ++tt) {
+    constexpr int kBlockTiles = G == 16 ? 1 : 2;
+    const int blk = tt / kBlockTiles;
+    uint32_t av[4];
+    frag_v<G, B>(p + blk * (B * 32), p1 + blk * (B * 32), lane_sh<B>(L), L.rot1, tt & 1, av);
+    const uint32_t a0 = kMask ? (s0[tt] & msk[tt][0]) : s0[tt];
+    const uint32_t a1 = kMask ? (s1[tt] & msk[tt][1]) : s1[tt];
+    const uint32_t bj[2] = {hmul2_u32(pb[tt][0], a0), hmul2_u32(pb[tt][1], a1)};
+    mma_m16n8k16(va, av, bj);
+  }
+}
+
+// Group tables in shared memory: per side, kept groups ordered by width class
+// (4, 2, 1, 3, 8), each entry {block offset, record offset, group index, width}
+// relative to the head section; class bounds; record offsets by group index.
+struct GroupTables {
+  int4 ord[2][kMaxG];
+  int cls[2][8];
+  int rec[2][kMaxG];
+  int wid[2][kMaxG];
+};
+
+template <int G, int NT, int CH, int B>
+__device__ __forceinline__ void key_class(const GroupTables& T, const uint8_t* sec, int chunk_blk_bytes_unit,
+                                          int rec_lane, const LaneAddr& L, const uint2* bq_s, int lane,
+                                          int ci, float (&acc)[CH][NT][4]) {
+  const int c1 = T.cls[0][ci + 1];
+#pragma unroll 1
+  for (int c = T.cls[0][ci]; c < c1; ++c) {
+    const int4 g = T.ord[0][c];
+    uint2 bqj[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) bqj[nt] = bq_s[(g.z * NT + nt) * 32 + lane];
+    key_group<G, NT, CH, B>(sec + g.x + chunk_blk_bytes_unit * B, sec + g.y + rec_lane, L, bqj, acc);
+  }
+}
+
+template <int G, int CH, int B, bool kMask>
+__device__ __forceinline__ void value_class(const GroupTables& T, const uint8_t* sec, int chunk_blk_bytes_unit,
+                                            int recA_lane, int recB_lane, const LaneAddr& L, float4* vacc,
+                                            int lane, int ci, bool grew, float ae, float ao,
+                                            const uint32_t (&pb)[CH][2], const uint32_t (&msk)[CH][2]) {
+  const int c1 = T.cls[1][ci + 1];
+#pragma unroll 1
+  for (int c = T.cls[1][ci]; c < c1; ++c) {
+    const int4 g = T.ord[1][c];
+    float4 v4 = vacc[g.z * 32 + lane];
+    if (grew) {
+      v4.x *= ae;
+      v4.y *= ao;
+      v4.z *= ae;
+      v4.w *= ao;
+    }
+    float va[4] = {v4.x, v4.y, v4.z, v4.w};
+    value_group<G, CH, B, kMask>(sec + g.x + chunk_blk_bytes_unit * B, sec + g.y + recA_lane, sec + g.y + recB_lane,
+                                 L, pb, msk, va);
+    vacc[g.z * 32 + lane] = make_float4(va[0], va[1], va[2], va[3]);
+  }
+}
+
+template <int G, int NT, int CH>
 __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs A) {
   const CodecDev* __restrict__ cd = A.cd;
   const int split = blockIdx.x, a = blockIdx.y, b = blockIdx.z;
@@ -301,19 +434,16 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmBars) + warp * 8;
-  uint2* bq_s = reinterpret_cast<uint2*>(smem + kSmBq);              // [row][lane]
-  int4* grp_s = reinterpret_cast<int4*>(smem + kSmGrp);              // [0..7] K, [8..15] V
-  int* misc_s = reinterpret_cast<int*>(smem + kSmMisc);
-  float4* vacc_s = reinterpret_cast<float4*>(smem + kSmAcc) + warp * kMaxG * 32;  // [j][lane]
+  uint2* bq_s = reinterpret_cast<uint2*>(smem + kSmBq);
+  GroupTables& T = *reinterpret_cast<GroupTables*>(smem + kSmGrp);
+  float4* vacc_s = reinterpret_cast<float4*>(smem + kSmAcc) + warp * kMaxG * 32;
   uint8_t* region = smem + kSmStages;
   uint8_t* my_stages = region + (size_t)warp * A.stages * A.stage_bytes;
 
   const int P = cd->P, gq = cd->gq;
+  const int tpp = P / 16;  // tiles per page
   const HeadDev* hd = &cd->head[a];
   const int sec_off = hd->sec_off, sec_bytes = hd->sec_bytes;
-  const int plane_stride = P * G / 8;
-  // the cache (written by the preceding encode) is complete once this grid runs:
-  // the fold it depends on started only after the encode finished
   const int len = A.lengths[b];
   const int n_pages = (len + P - 1) / P;
   const int per = (n_pages + A.n_split - 1) / A.n_split;
@@ -349,16 +479,23 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   if (lane == 0)
     for (int i = 0; i < min(S, my_count); ++i) issue(i);
 
-  if (tid < 2 * kMaxG) {
-    const bool isv = tid >= kMaxG;
-    const int j = tid & (kMaxG - 1);
-    const SideDev* sd = isv ? sv : sk;
-    int4 g = make_int4(0, 0, 0, 0);
-    if (j < sd->n_groups) {
-      const GroupDev gd = sd->grp[j];
-      g = make_int4(gd.plane_off - sec_off, gd.plane_off - sec_off + gd.b * plane_stride, gd.b, 0);
+  // group tables (one thread per side)
+  if (tid < 2) {
+    const SideDev* sd = tid ? sv : sk;
+    constexpr int kOrder[5] = {4, 2, 1, 3, 8};
+    int n = 0;
+    for (int ci = 0; ci < 5; ++ci) {
+      T.cls[tid][ci] = n;
+      for (int j = 0; j < sd->n_groups; ++j) {
+        const GroupDev gd = sd->grp[j];
+        if (gd.b == kOrder[ci]) T.ord[tid][n++] = make_int4(gd.plane_off - sec_off, gd.sz_off - sec_off, j, gd.b);
+      }
     }
-    grp_s[tid] = g;
+    T.cls[tid][5] = n;
+    for (int j = 0; j < kMaxG; ++j) {
+      T.rec[tid][j] = j < sd->n_groups ? sd->grp[j].sz_off - sec_off : -1;
+      T.wid[tid][j] = j < sd->n_groups ? sd->grp[j].b : 0;
+    }
   }
   for (int j = 0; j < kMaxG; ++j) vacc_s[j * 32 + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
 
@@ -369,8 +506,6 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
     for (int e = tid; e < kFragWords; e += blockDim.x) bq_s[e] = src[e];
   }
   __syncthreads();
-  if (tid < kMaxG) misc_s[tid] = (tid < nV) ? grp_s[kMaxG + tid].y : -1;  // V record offsets by group
-  __syncthreads();
   uint32_t bz[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -378,12 +513,22 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
     bz[nt][0] = v.x;
     bz[nt][1] = v.y;
   }
-  uint32_t rot[4];
-#pragma unroll
-  for (int p = 0; p < 4; ++p) rot[p] = (uint32_t)(t4 - p) & 31u;
-  const int vrec_mine = misc_s[gid];  // record offset of V group `gid` (-1 if none)
-  const int krecA = (2 * t4 < nK) ? grp_s[2 * t4].y : -1;          // K groups 2*t4, 2*t4+1
-  const int krecB = (2 * t4 + 1 < nK) ? grp_s[2 * t4 + 1].y : -1;
+  LaneAddr L;
+  L.off4 = lane * 4;
+  L.off8 = lane * 8;
+  L.off2 = (2 * gid + (t4 >> 1)) * 4;
+  L.off1 = gid * 4;
+  L.sh2 = 2u * (uint32_t)(t4 & 1);
+  L.sh1 = (uint32_t)t4;
+  L.rot1 = (uint32_t)(t4 - 2) & 31u;
+  // record offsets (within a group's records) of this lane for chunk 0: K rows
+  // use token pair gid; V uses pairs t4 and t4 + 4; the K z term uses groups
+  // 2*t4 and 2*t4+1 at pair gid; the V z term group gid at pairs t4, t4+4
+  const int recK = gid * tpp * 8, recVa = t4 * tpp * 8, recVb = (t4 + 4) * tpp * 8;
+  const int zkA = T.rec[0][min(2 * t4, kMaxG - 1)], zkB = T.rec[0][min(2 * t4 + 1, kMaxG - 1)];
+  const bool hasA = 2 * t4 < nK, hasB = 2 * t4 + 1 < nK;
+  const int zv = T.rec[1][gid];
+  const bool hasV = gid < nV;
 
   float m_run[NT], l_run[NT];
 #pragma unroll
@@ -393,7 +538,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   }
   float dz[4] = {0.f, 0.f, 0.f, 0.f};
 
-  // ---- 3. stream this warp's pages in chunks of 64 tokens -------------------
+  // ---- 3. stream this warp's pages, CH tiles (16 tokens each) at a time ------
   bool timed_out = false;
   int i = 0;
   for (; i < my_count; ++i) {
@@ -406,83 +551,81 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
     const uint8_t* sec = my_stages + (size_t)s * A.stage_bytes;
     const int pg = p0 + warp + kDecWarps * i;
     const int n_valid = min(P, len - pg * P);
-    const int n_tiles = (n_valid + 15) >> 4;
 #pragma unroll 1
-    for (int t0 = 0; t0 < n_tiles; t0 += kChunk) {
-      const int ntile = min(kChunk, n_tiles - t0);
+    for (int c0 = 0; c0 < tpp; c0 += CH) {
+      const int tok0 = c0 * 16;
+      const bool partial = n_valid < tok0 + CH * 16;  // warp-uniform
+      const int unit = c0 * 32 / (G == 16 ? 1 : 2);   // chunk's block bytes per code bit
       // keys
-      float acc[kChunk][NT][4];
+      float acc[CH][NT][4];
 #pragma unroll
-      for (int tt = 0; tt < kChunk; ++tt)
+      for (int tt = 0; tt < CH; ++tt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int r = 0; r < 4; ++r) acc[tt][nt][r] = 0.f;
-#pragma unroll 1
-      for (int j = 0; j < nK; ++j) {
-        const int4 g = grp_s[j];
-        uint2 bqj[NT];
+      const int rk = recK + c0 * 8;
+      key_class<G, NT, CH, 4>(T, sec, unit, rk, L, bq_s, lane, 0, acc);
+      key_class<G, NT, CH, 2>(T, sec, unit, rk, L, bq_s, lane, 1, acc);
+      key_class<G, NT, CH, 1>(T, sec, unit, rk, L, bq_s, lane, 2, acc);
+      key_class<G, NT, CH, 3>(T, sec, unit, rk, L, bq_s, lane, 3, acc);
+      key_class<G, NT, CH, 8>(T, sec, unit, rk, L, bq_s, lane, 4, acc);
+      // z term of the keys (k = group index) and the scores (log2 units)
+      uint32_t zA[CH], zB[CH];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) bqj[nt] = bq_s[(j * NT + nt) * 32 + lane];
-        const uint8_t* pbase = sec + g.x + gid * 4;
-        const uint8_t* rbase = sec + g.y + gid * 8;
-        switch (g.z) {
-          case 1: key_group<G, NT, 1>(pbase, rbase, bqj, t0, ntile, plane_stride, rot, acc); break;
-          case 2: key_group<G, NT, 2>(pbase, rbase, bqj, t0, ntile, plane_stride, rot, acc); break;
-          case 3: key_group<G, NT, 3>(pbase, rbase, bqj, t0, ntile, plane_stride, rot, acc); break;
-          case 4: key_group<G, NT, 4>(pbase, rbase, bqj, t0, ntile, plane_stride, rot, acc); break;
-          default: key_group<G, NT, 8>(pbase, rbase, bqj, t0, ntile, plane_stride, rot, acc); break;
+      for (int h = 0; h < CH / 2; ++h) {
+        const uint4 ra = hasA ? *reinterpret_cast<const uint4*>(sec + zkA + rk + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint4 rb = hasB ? *reinterpret_cast<const uint4*>(sec + zkB + rk + 16 * h) : make_uint4(0, 0, 0, 0);
+        zA[2 * h] = ra.y;
+        zA[2 * h + 1] = ra.w;
+        zB[2 * h] = rb.y;
+        zB[2 * h + 1] = rb.w;
+      }
+      float sc[CH][NT][2];
+#pragma unroll
+      for (int tt = 0; tt < CH; ++tt) {
+        const uint32_t az[4] = {__byte_perm(zA[tt], zB[tt], 0x5410), __byte_perm(zA[tt], zB[tt], 0x7632), 0u, 0u};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float d[4];
+          mma_m16n8k16_z(d, az, bz[nt]);
+          sc[tt][nt][0] = fmaf(acc[tt][nt][0] + acc[tt][nt][1], kTwo24, d[0] + d[1]);
+          sc[tt][nt][1] = fmaf(acc[tt][nt][2] + acc[tt][nt][3], kTwo20, d[2] + d[3]);
         }
       }
-      // z term of the keys (k = group index) and the scores
-      float sc[kChunk][NT][2];
+      if (partial) {
 #pragma unroll
-      for (int tt = 0; tt < kChunk; ++tt) {
-        const int t = t0 + tt;
-        const int nv = n_valid - t * 16;
-        if (tt < ntile) {
-          const uint32_t zA = krecA >= 0 ? *reinterpret_cast<const uint32_t*>(sec + krecA + (t * 8 + gid) * 8 + 4) : 0u;
-          const uint32_t zB = krecB >= 0 ? *reinterpret_cast<const uint32_t*>(sec + krecB + (t * 8 + gid) * 8 + 4) : 0u;
-          const uint32_t az[4] = {__byte_perm(zA, zB, 0x5410), __byte_perm(zA, zB, 0x7632), 0u, 0u};
+        for (int tt = 0; tt < CH; ++tt) {
+          const int nv = n_valid - tok0 - tt * 16;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            float d[4];
-            mma_m16n8k16_z(d, az, bz[nt]);
-            sc[tt][nt][0] = fmaf(acc[tt][nt][0] + acc[tt][nt][1], kTwo24, d[0] + d[1]);
-            sc[tt][nt][1] = fmaf(acc[tt][nt][2] + acc[tt][nt][3], kTwo24, d[2] + d[3]);
             if (2 * gid >= nv) sc[tt][nt][0] = -CUDART_INF_F;
             if (2 * gid + 1 >= nv) sc[tt][nt][1] = -CUDART_INF_F;
           }
-        } else {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) sc[tt][nt][0] = sc[tt][nt][1] = -CUDART_INF_F;
         }
       }
       // online softmax (log2 units); rescale only when a running max grows
-      float mt[NT];
       bool grow = false;
+      float alpha[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float mx = -CUDART_INF_F;
 #pragma unroll
-        for (int tt = 0; tt < kChunk; ++tt) mx = fmaxf(mx, fmaxf(sc[tt][nt][0], sc[tt][nt][1]));
+        for (int tt = 0; tt < CH; ++tt) mx = fmaxf(mx, fmaxf(sc[tt][nt][0], sc[tt][nt][1]));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        mt[nt] = mx;
-        grow |= mx > m_run[nt];
+        alpha[nt] = 1.f;
+        if (mx > m_run[nt]) {
+          alpha[nt] = ex2_approx(m_run[nt] - mx);
+          m_run[nt] = mx;
+          l_run[nt] *= alpha[nt];
+          grow = true;
+        }
       }
       const bool grew = __any_sync(0xffffffffu, grow);
       float ae = 1.f, ao = 1.f;
       if (grew) {
-        float alpha[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float m_new = fmaxf(m_run[nt], mt[nt]);
-          alpha[nt] = exp2f(m_run[nt] - m_new);
-          m_run[nt] = m_new;
-          l_run[nt] *= alpha[nt];
-        }
         // value accumulators hold heads 2*t4 and 2*t4+1
         ae = __shfl_sync(0xffffffffu, alpha[0], (2 * t4) & 3);
         ao = __shfl_sync(0xffffffffu, alpha[0], (2 * t4 + 1) & 3);
@@ -499,16 +642,16 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
       }
       // p as the B operand (tokens x heads): lane (gid, t4) needs head gid,
       // tokens (2t4, 2t4+1) and (2t4+8, 2t4+9)
-      uint32_t pb[kChunk][2];
-      uint32_t msk[kChunk][2];
+      uint32_t pb[CH][2];
+      uint32_t msk[CH][2];
       const int src0 = (t4 << 2) | (gid & 3), src1 = ((t4 + 4) << 2) | (gid & 3);
 #pragma unroll
-      for (int tt = 0; tt < kChunk; ++tt) {
+      for (int tt = 0; tt < CH; ++tt) {
         uint32_t p01[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const float pa = exp2f(sc[tt][nt][0] - m_run[nt] + kPScaleLog2);
-          const float pv = exp2f(sc[tt][nt][1] - m_run[nt] + kPScaleLog2);
+          const float pa = ex2_approx(sc[tt][nt][0] - m_run[nt] + kPScaleLog2);
+          const float pv = ex2_approx(sc[tt][nt][1] - m_run[nt] + kPScaleLog2);
           l_run[nt] += pa + pv;
           p01[nt] = pack_half2(pa, pv);
         }
@@ -523,41 +666,45 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
           }
         }
         if (gid >= gq) pb[tt][0] = pb[tt][1] = 0u;
-        // tokens past the end: their records may hold anything; zero their s and z
-        const int nv = n_valid - (t0 + tt) * 16;
         msk[tt][0] = msk[tt][1] = 0xffffffffu;
-        if (nv < 16) {
+        if (partial) {
+          // tokens past the end: their records may hold anything; zero their s and z
+          const int nv = n_valid - tok0 - tt * 16;
           msk[tt][0] = ((2 * t4 < nv) ? 0x0000ffffu : 0u) | ((2 * t4 + 1 < nv) ? 0xffff0000u : 0u);
           msk[tt][1] = ((2 * t4 + 8 < nv) ? 0x0000ffffu : 0u) | ((2 * t4 + 9 < nv) ? 0xffff0000u : 0u);
         }
       }
       // values: per group, sum_t (p_t s_t,j) code_t,j ...
-#pragma unroll 1
-      for (int j = 0; j < nV; ++j) {
-        const int4 g = grp_s[kMaxG + j];
-        const float4 v4 = vacc_s[j * 32 + lane];
-        float va[4] = {v4.x * ae, v4.y * ao, v4.z * ae, v4.w * ao};
-        const uint8_t* pbase = sec + g.x + gid * 4;
-        const uint8_t* rbase = sec + g.y + t4 * 8;
-        switch (g.z) {
-          case 1: value_group<G, 1>(pbase, rbase, pb, msk, t0, ntile, plane_stride, rot, va); break;
-          case 2: value_group<G, 2>(pbase, rbase, pb, msk, t0, ntile, plane_stride, rot, va); break;
-          case 3: value_group<G, 3>(pbase, rbase, pb, msk, t0, ntile, plane_stride, rot, va); break;
-          case 4: value_group<G, 4>(pbase, rbase, pb, msk, t0, ntile, plane_stride, rot, va); break;
-          default: value_group<G, 8>(pbase, rbase, pb, msk, t0, ntile, plane_stride, rot, va); break;
-        }
-        vacc_s[j * 32 + lane] = make_float4(va[0], va[1], va[2], va[3]);
+      const int ra = recVa + c0 * 8, rb = recVb + c0 * 8;
+      if (!partial) {
+        value_class<G, CH, 4, false>(T, sec, unit, ra, rb, L, vacc_s, lane, 0, grew, ae, ao, pb, msk);
+        value_class<G, CH, 2, false>(T, sec, unit, ra, rb, L, vacc_s, lane, 1, grew, ae, ao, pb, msk);
+        value_class<G, CH, 1, false>(T, sec, unit, ra, rb, L, vacc_s, lane, 2, grew, ae, ao, pb, msk);
+        value_class<G, CH, 3, false>(T, sec, unit, ra, rb, L, vacc_s, lane, 3, grew, ae, ao, pb, msk);
+        value_class<G, CH, 8, false>(T, sec, unit, ra, rb, L, vacc_s, lane, 4, grew, ae, ao, pb, msk);
+      } else {
+        value_class<G, CH, 4, true>(T, sec, unit, ra, rb, L, vacc_s, lane, 0, grew, ae, ao, pb, msk);
+        value_class<G, CH, 2, true>(T, sec, unit, ra, rb, L, vacc_s, lane, 1, grew, ae, ao, pb, msk);
+        value_class<G, CH, 1, true>(T, sec, unit, ra, rb, L, vacc_s, lane, 2, grew, ae, ao, pb, msk);
+        value_class<G, CH, 3, true>(T, sec, unit, ra, rb, L, vacc_s, lane, 3, grew, ae, ao, pb, msk);
+        value_class<G, CH, 8, true>(T, sec, unit, ra, rb, L, vacc_s, lane, 4, grew, ae, ao, pb, msk);
       }
-      // ... plus sum_t p_t z_t,j for all groups (rows = groups)
+      // ... plus sum_t p_t z_t,j for all groups (rows = groups).  Lanes of
+      // absent groups load nothing, but every lane executes the MMA.
+      {
+        uint32_t za[CH], zb[CH];
 #pragma unroll
-      for (int tt = 0; tt < kChunk; ++tt) {
-        if (tt < ntile) {
-          uint32_t az[4] = {0u, 0u, 0u, 0u};
-          if (vrec_mine >= 0) {
-            const uint8_t* rb = sec + vrec_mine + (t0 + tt) * 64;
-            az[0] = *reinterpret_cast<const uint32_t*>(rb + t4 * 8 + 4) & msk[tt][0];
-            az[2] = *reinterpret_cast<const uint32_t*>(rb + (t4 + 4) * 8 + 4) & msk[tt][1];
-          }
+        for (int h = 0; h < CH / 2; ++h) {
+          const uint4 x = hasV ? *reinterpret_cast<const uint4*>(sec + zv + ra + 16 * h) : make_uint4(0, 0, 0, 0);
+          const uint4 y = hasV ? *reinterpret_cast<const uint4*>(sec + zv + rb + 16 * h) : make_uint4(0, 0, 0, 0);
+          za[2 * h] = x.y;
+          za[2 * h + 1] = x.w;
+          zb[2 * h] = y.y;
+          zb[2 * h + 1] = y.w;
+        }
+#pragma unroll
+        for (int tt = 0; tt < CH; ++tt) {
+          const uint32_t az[4] = {za[tt] & msk[tt][0], 0u, zb[tt] & msk[tt][1], 0u};
           mma_m16n8k16(dz, az, pb[tt]);
         }
       }
@@ -588,10 +735,13 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   }
 
   // ---- 4. merge the warps of this CTA into one partial record per q head ----
+  // latent accumulator of (head h, coordinate j*G + k) = 2^24 * f * vacc + the
+  // z term of group j; f = 1/16 for rows k >= 8 of a G = 16 group of width <= 4
   __syncthreads();
   const int nkv = sv->n_kept;
-  const int rec = 2 + kMaxKept;
-  float* wsm = reinterpret_cast<float*>(region);
+  constexpr int rec = 2 + kMaxKept;
+  float* wsm = reinterpret_cast<float*>(region);              // [warp][gq][rec]
+  float* wts = wsm + kDecWarps * kMaxGQ * rec;                // [gq][kDecWarps + 2]
   if (gid == 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -602,39 +752,49 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
       }
     }
   }
+  const int h0 = 2 * t4, h1 = 2 * t4 + 1;
   for (int j = 0; j < nV; ++j) {
     const float4 v4 = vacc_s[j * 32 + lane];
-    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int hl = 2 * t4 + (c & 1);
-      const int coord = j * G + gid + ((c >> 1) ? 8 : 0);
-      if (hl < gq && (G == 16 || c < 2)) wsm[(warp * gq + hl) * rec + 2 + coord] = vv[c] * kTwo24;
+    const float z0 = __shfl_sync(0xffffffffu, dz[0], j * 4 + t4);
+    const float z1 = __shfl_sync(0xffffffffu, dz[1], j * 4 + t4);
+    const float f_hi = (G == 16 && T.wid[1][j] <= 4) ? kTwo20 : kTwo24;
+    float* r0 = wsm + (warp * gq + h0) * rec + 2 + j * G + gid;
+    float* r1 = wsm + (warp * gq + h1) * rec + 2 + j * G + gid;
+    if (h0 < gq) {
+      r0[0] = fmaf(v4.x, kTwo24, z0);
+      if (G == 16) r0[8] = fmaf(v4.z, f_hi, z0);
+    }
+    if (h1 < gq) {
+      r1[0] = fmaf(v4.y, kTwo24, z1);
+      if (G == 16) r1[8] = fmaf(v4.w, f_hi, z1);
     }
   }
-  __syncwarp();
-  if (gid < nV) {  // z term of group gid, heads 2*t4 and 2*t4+1
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int hl = 2 * t4 + c;
-      if (hl < gq)
-        for (int k = 0; k < G; ++k) wsm[(warp * gq + hl) * rec + 2 + gid * G + k] += dz[c];
+  __syncthreads();
+  if (tid < gq) {
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wsm[(w * gq + tid) * rec]);
+    float Lsum = 0.f;
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float mw = wsm[(w * gq + tid) * rec];
+      const float wt = (mw == -CUDART_INF_F) ? 0.f : ex2_approx(mw - M);
+      wts[tid * (kDecWarps + 2) + w] = wt;
+      Lsum = fmaf(wt, wsm[(w * gq + tid) * rec + 1], Lsum);
     }
+    wts[tid * (kDecWarps + 2) + kDecWarps] = M;
+    wts[tid * (kDecWarps + 2) + kDecWarps + 1] = Lsum;
   }
   __syncthreads();
   float* part = A.part + ((size_t)(b * A.n_q + a * gq) * A.n_split + split) * A.part_stride;
   for (int idx = tid; idx < gq * (2 + nkv); idx += blockDim.x) {
     const int hl = idx / (2 + nkv), c = idx % (2 + nkv);
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wsm[(w * gq + hl) * rec]);
-    float v = 0.f;
-    if (c == 0) {
-      v = M;
-    } else if (M != -CUDART_INF_F) {
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float mw = wsm[(w * gq + hl) * rec];
-        if (mw != -CUDART_INF_F) v += exp2f(mw - M) * wsm[(w * gq + hl) * rec + c];
-      }
+    const float* wt = wts + hl * (kDecWarps + 2);
+    float v;
+    if (c < 2) {
+      v = wt[kDecWarps + c];
+    } else {
+      v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) v = fmaf(wt[w], wsm[(w * gq + hl) * rec + c], v);
     }
     part[(size_t)hl * A.n_split * A.part_stride + c] = v;
   }
@@ -743,19 +903,29 @@ cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, int s
   return cudaGetLastError();
 }
 
-template <int G, int NT>
+template <int G, int NT, int CH>
 int split_occupancy(int smem) {
   int n = 0;
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(split_kernel<G, NT>), smem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<G, NT>, kDecWarps * 32, smem) != cudaSuccess ||
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(split_kernel<G, NT, CH>), smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<G, NT, CH>, kDecWarps * 32, smem) !=
+          cudaSuccess ||
       n <= 0)
     n = 1;
   return n;
 }
 
-int split_ctas_per_sm(int group, bool two_tiles, int smem) {
-  if (group == 16) return two_tiles ? split_occupancy<16, 2>(smem) : split_occupancy<16, 1>(smem);
-  return two_tiles ? split_occupancy<8, 2>(smem) : split_occupancy<8, 1>(smem);
+// Tiles (16 tokens) per softmax chunk: 4 when a page holds a multiple of 64
+// tokens, else 2 (pages hold a multiple of 32).
+int chunk_tiles(int P) { return (P / 16) % 4 == 0 ? 4 : 2; }
+
+int split_ctas_per_sm(int group, bool two_tiles, int P, int smem) {
+  const bool c4 = chunk_tiles(P) == 4;
+  if (group == 16) {
+    if (two_tiles) return c4 ? split_occupancy<16, 2, 4>(smem) : split_occupancy<16, 2, 2>(smem);
+    return c4 ? split_occupancy<16, 1, 4>(smem) : split_occupancy<16, 1, 2>(smem);
+  }
+  if (two_tiles) return c4 ? split_occupancy<8, 2, 4>(smem) : split_occupancy<8, 2, 2>(smem);
+  return c4 ? split_occupancy<8, 1, 4>(smem) : split_occupancy<8, 1, 2>(smem);
 }
 
 int sm_count() {
@@ -768,11 +938,11 @@ int sm_count() {
   return n;
 }
 
-template <int G, int NT>
+template <int G, int NT, int CH>
 cudaError_t launch_all(const DecodeArgs& args, const DecodePlan& plan, int batch, int n_kv, int n_q, cudaStream_t st) {
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(fold_kernel<G, NT>), fold_smem_bytes());
   if (e != cudaSuccess) return e;
-  e = ensure_dynamic_smem(reinterpret_cast<const void*>(split_kernel<G, NT>), plan.smem_bytes);
+  e = ensure_dynamic_smem(reinterpret_cast<const void*>(split_kernel<G, NT, CH>), plan.smem_bytes);
   if (e != cudaSuccess) return e;
   const int csm = combine_smem_bytes(args.n_split, args.part_stride);
   e = ensure_dynamic_smem(reinterpret_cast<const void*>(combine_kernel), csm);
@@ -780,10 +950,17 @@ cudaError_t launch_all(const DecodeArgs& args, const DecodePlan& plan, int batch
   fold_kernel<G, NT><<<dim3(n_kv, batch), 256, fold_smem_bytes(), st>>>(args);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = launch_dependent(split_kernel<G, NT>, dim3(args.n_split, n_kv, batch), dim3(kDecWarps * 32), plan.smem_bytes,
-                       st, args);
+  e = launch_dependent(split_kernel<G, NT, CH>, dim3(args.n_split, n_kv, batch), dim3(kDecWarps * 32),
+                       plan.smem_bytes, st, args);
   if (e != cudaSuccess) return e;
   return launch_dependent(combine_kernel, dim3(n_q, batch), dim3(256), csm, st, args);
+}
+
+template <int G, int NT>
+cudaError_t launch_chunked(const DecodeArgs& args, const DecodePlan& plan, int P, int batch, int n_kv, int n_q,
+                           cudaStream_t st) {
+  return chunk_tiles(P) == 4 ? launch_all<G, NT, 4>(args, plan, batch, n_kv, n_q, st)
+                             : launch_all<G, NT, 2>(args, plan, batch, n_kv, n_q, st);
 }
 
 }  // namespace
@@ -811,13 +988,12 @@ DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq)
   // 2 stages per warp (more when sections are small) keep > 40 KB in flight per SM
   const int budget = 64 * 1024;
   p.stages = std::max(2, std::min(4, budget / (kDecWarps * p.stage_bytes)));
-  const int merge_bytes = kDecWarps * h.gq * (2 + kMaxKept) * 4;
-  p.smem_bytes = kSmStages + std::max(kDecWarps * p.stages * p.stage_bytes, merge_bytes);
+  p.smem_bytes = kSmStages + std::max(kDecWarps * p.stages * p.stage_bytes, kMergeBytes);
   // context splits: fill one wave of resident CTAs when that wastes < 15% of the
   // slots, else two waves; the count does not depend on the context length, so a
   // workspace sized once fits every call (the call clamps it to the cache's pages)
   const int units = std::max(1, batch * h.n_kv);
-  const int slots = split_ctas_per_sm(h.group, h.gq > 4, p.smem_bytes) * sm_count();
+  const int slots = split_ctas_per_sm(h.group, h.gq > 4, h.P, p.smem_bytes) * sm_count();
   int ns = std::max(1, slots / units);
   if ((double)units * ns / slots < 0.85) {
     const int ns2 = std::max(1, 2 * slots / units);
@@ -863,10 +1039,10 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
   args.q_scale = 1.4426950408889634f / sqrtf((float)h.d_h);
   const bool two = h.gq > 4;
   if (h.group == 16)
-    return two ? launch_all<16, 2>(args, plan, cache.batch, h.n_kv, h.n_q, st)
-               : launch_all<16, 1>(args, plan, cache.batch, h.n_kv, h.n_q, st);
-  return two ? launch_all<8, 2>(args, plan, cache.batch, h.n_kv, h.n_q, st)
-             : launch_all<8, 1>(args, plan, cache.batch, h.n_kv, h.n_q, st);
+    return two ? launch_chunked<16, 2>(args, plan, h.P, cache.batch, h.n_kv, h.n_q, st)
+               : launch_chunked<16, 1>(args, plan, h.P, cache.batch, h.n_kv, h.n_q, st);
+  return two ? launch_chunked<8, 2>(args, plan, h.P, cache.batch, h.n_kv, h.n_q, st)
+             : launch_chunked<8, 1>(args, plan, h.P, cache.batch, h.n_kv, h.n_q, st);
 }
 
 }  // namespace spectra

@@ -135,41 +135,91 @@ __global__ void __launch_bounds__(1024) append_plan_kernel(
 // Per token and group (every step one IEEE fp32 operation, no contraction):
 //   s = fp16(sat((max - min) / (2^b - 1))), z = fp16(sat(min)),
 //   code = clamp(rint((x - z) / s), 0, 2^b - 1), s == 0 -> 0.
-// Bits go to the page's bit-planes at the canonical (word, bit) addresses; the
-// token's bits are cleared then set with atomics, so tokens of one 256-bit block
-// written by different blocks of this grid (or by different calls) never race.
+// Code bits go to the group's block at the canonical (word, bit) addresses of
+// the page layout (fragment position of the entry, then the width rule); the
+// token's bits are cleared then set with atomics, so tokens of one block written
+// by different blocks of this grid (or by different calls) never race.
 // ---------------------------------------------------------------------------
 namespace {
 
 __device__ __forceinline__ float sat16(float x) { return fminf(fmaxf(x, -65504.f), 65504.f); }
 
+// Fragment position (gid, t4, slot) of entry (token tb of the block, coordinate k).
 template <int G>
-__device__ __forceinline__ void k_side_addr(int tb, int k, int* word, int* bit) {
+__device__ __forceinline__ void k_side_pos(int tb, int k, int* gid, int* t4, int* slot) {
   if (G == 16) {
     const int row = (tb & 1) ? 8 + (tb >> 1) : (tb >> 1);
-    const int slot = (row >> 3) + 2 * (k >> 3) + 4 * (k & 1);
-    *word = row & 7;
-    *bit = 4 * slot + ((k & 7) >> 1);
+    *slot = (row >> 3) + 2 * (k >> 3) + 4 * (k & 1);
+    *gid = row & 7;
+    *t4 = (k & 7) >> 1;
   } else {
     const int mi = tb >> 4, tl = tb & 15;
     const int row = (tl & 1) ? 8 + (tl >> 1) : (tl >> 1);
-    const int slot = (row >> 3) + 2 * mi + 4 * (k & 1);
-    *word = row & 7;
-    *bit = 4 * slot + (k >> 1);
+    *slot = (row >> 3) + 2 * mi + 4 * (k & 1);
+    *gid = row & 7;
+    *t4 = k >> 1;
   }
 }
 
 template <int G>
-__device__ __forceinline__ void v_side_addr(int tb, int k, int* word, int* bit) {
+__device__ __forceinline__ void v_side_pos(int tb, int k, int* gid, int* t4, int* slot) {
   if (G == 16) {
-    const int slot = (k >> 3) + 2 * (tb >> 3) + 4 * (tb & 1);
-    *word = k & 7;
-    *bit = 4 * slot + ((tb & 7) >> 1);
+    *slot = (k >> 3) + 2 * (tb >> 3) + 4 * (tb & 1);
+    *gid = k & 7;
+    *t4 = (tb & 7) >> 1;
   } else {
     const int mi = tb >> 4, tl = tb & 15;
-    const int slot = mi + 2 * (tl >> 3) + 4 * (tl & 1);
-    *word = k;
-    *bit = 4 * slot + ((tl & 7) >> 1);
+    *slot = mi + 2 * (tl >> 3) + 4 * (tl & 1);
+    *gid = k;
+    *t4 = (tl & 7) >> 1;
+  }
+}
+
+// Pending bits of one block word: consecutive entries that land in the same word
+// are merged and written with one atomicAnd/atomicOr pair.
+struct WordBits {
+  int w;
+  uint32_t mask, val;
+};
+
+__device__ __forceinline__ void flush_word(uint32_t* blk, WordBits& a) {
+  if (a.w >= 0) {
+    atomicAnd(blk + a.w, ~a.mask);
+    atomicOr(blk + a.w, a.val);
+  }
+  a.w = -1;
+  a.mask = a.val = 0u;
+}
+
+__device__ __forceinline__ void put_bits(uint32_t* blk, WordBits& a, int w, int shift, uint32_t width_mask,
+                                         uint32_t v) {
+  if (w != a.w) {
+    flush_word(blk, a);
+    a.w = w;
+  }
+  a.mask |= width_mask << shift;
+  a.val |= (v & width_mask) << shift;
+}
+
+// Writes one code (width b) of fragment position (gid, t4, slot) into a block:
+//   b = 4: word 4 gid + t4, nibble `slot`;
+//   b = 2: word 2 gid + t4/2, bits 4 slot + 2 (t4 % 2) + {0, 1};
+//   b = 1: word gid, bit 4 slot + t4;
+//   b = 3: bits 0-1 as b = 2, bit 2 as b = 1 in words 16 + gid (second pending word);
+//   b = 8: word 2 (4 gid + t4) + (slot / 2) % 2, byte (slot % 2) + 2 (slot / 4).
+__device__ __forceinline__ void put_code(uint32_t* blk, WordBits& a, WordBits& a1, int b, int gid, int t4,
+                                         int slot, uint32_t code) {
+  switch (b) {
+    case 4: put_bits(blk, a, 4 * gid + t4, 4 * slot, 0xFu, code); break;
+    case 2: put_bits(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code); break;
+    case 1: put_bits(blk, a, gid, 4 * slot + t4, 0x1u, code); break;
+    case 3:
+      put_bits(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code);
+      put_bits(blk, a1, 16 + gid, 4 * slot + t4, 0x1u, code >> 2);
+      break;
+    default:
+      put_bits(blk, a, 2 * (4 * gid + t4) + ((slot >> 1) & 1), 8 * ((slot & 1) + 2 * (slot >> 2)), 0xFFu, code);
+      break;
   }
 }
 
@@ -198,7 +248,6 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
   const int tau = p_tok % P;
   const int blk = tau / TB, tb = tau % TB;
   const float* crow = C + (size_t)i * ldc + sd.c_col0;
-  const int plane_stride = P * G / 8;
   const int n_groups = sd.n_groups;
   for (int j = warp * GROUPS_PER_WARP + lane / LANES_PER_TOKENSET; j < n_groups;
        j += 4 * GROUPS_PER_WARP) {
@@ -233,47 +282,20 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
       }
       code[k] = (uint32_t)c;
     }
-    uint32_t* plane0 = reinterpret_cast<uint32_t*>(page + gd.plane_off + blk * 32);
-    if (side == 0) {
-      int word = 0, bit;
-      uint32_t mask = 0;
+    uint32_t* blkw = reinterpret_cast<uint32_t*>(page + gd.plane_off + blk * (32 * b));
+    WordBits acc{-1, 0u, 0u}, acc1{-1, 0u, 0u};
 #pragma unroll
-      for (int k = 0; k < G; ++k) {
-        k_side_addr<G>(tb, k, &word, &bit);
-        mask |= 1u << bit;
-      }
-      for (int p = 0; p < b; ++p) {
-        uint32_t val = 0;
-#pragma unroll
-        for (int k = 0; k < G; ++k) {
-          k_side_addr<G>(tb, k, &word, &bit);
-          val |= ((code[k] >> p) & 1u) << bit;
-        }
-        uint32_t* w = plane0 + p * (plane_stride / 4) + word;
-        atomicAnd(w, ~mask);
-        atomicOr(w, val);
-      }
-    } else {
-      for (int p = 0; p < b; ++p) {
-        uint32_t m8[8], v8[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) m8[w] = v8[w] = 0;
-#pragma unroll
-        for (int k = 0; k < G; ++k) {
-          int word, bit;
-          v_side_addr<G>(tb, k, &word, &bit);
-          m8[word] |= 1u << bit;
-          v8[word] |= ((code[k] >> p) & 1u) << bit;
-        }
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          uint32_t* wp = plane0 + p * (plane_stride / 4) + w;
-          atomicAnd(wp, ~m8[w]);
-          atomicOr(wp, v8[w]);
-        }
-      }
+    for (int k = 0; k < G; ++k) {
+      int gid, t4, slot;
+      if (side == 0) k_side_pos<G>(tb, k, &gid, &t4, &slot);
+      else v_side_pos<G>(tb, k, &gid, &t4, &slot);
+      put_code(blkw, acc, acc1, b, gid, t4, slot, code[k]);
     }
-    __half* rec = reinterpret_cast<__half*>(page + gd.sz_off + 8 * (tau >> 1));
+    flush_word(blkw, acc);
+    flush_word(blkw, acc1);
+    // record of the token pair u = tau/2: index (u % 8) * (P/16) + u / 8
+    const int u = tau >> 1;
+    __half* rec = reinterpret_cast<__half*>(page + gd.sz_off + 8 * ((u & 7) * (P >> 4) + (u >> 3)));
     rec[tau & 1] = s_h;
     rec[2 + (tau & 1)] = z_h;
   }

@@ -11,22 +11,51 @@ import oracle
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-def test_addresses_are_a_bijection():
+def _golden_rows():
+    with open(os.path.join(GOLDEN, "layout_bits.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                yield [x.strip() for x in line.split("|")]
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 8])
+def test_addresses_are_a_bijection(b):
     for g in (8, 16):
         for side in ("K", "V"):
             tb = oracle.tokens_per_block(g)
-            seen = {oracle.block_bit_address(g, side, t, k) for t in range(tb) for k in range(g)}
+            seen = {oracle.code_bit_address(g, side, b, t, k, p)
+                    for t in range(tb) for k in range(g) for p in range(b)}
+            assert len(seen) == 256 * b
+            assert all(0 <= w < 8 * b and 0 <= bit < 32 for w, bit in seen)
+
+
+def test_fragment_positions_are_a_bijection():
+    for g in (8, 16):
+        for side in ("K", "V"):
+            tb = oracle.tokens_per_block(g)
+            seen = {oracle.fragment_position(g, side, t, k) for t in range(tb) for k in range(g)}
             assert len(seen) == 256
-            assert all(0 <= w < 8 and 0 <= b < 32 for w, b in seen)
+            assert all(0 <= gid < 8 and 0 <= t4 < 4 and 0 <= sl < 8 for gid, t4, sl in seen)
 
 
 def test_hand_derived_addresses():
-    with open(os.path.join(GOLDEN, "layout_bits.txt")) as f:
-        rows = [l.split("|") for l in f if l.strip() and not l.startswith("#")]
+    rows = [r for r in _golden_rows() if r[0] != "rec"]
+    assert len(rows) >= 10
+    for r in rows:
+        g, side, b, tau, k, p, word, bit = int(r[0]), r[1], *map(int, r[2:])
+        assert oracle.code_bit_address(g, side, b, tau, k, p) == (word, bit), r
+
+
+def test_hand_derived_record_indices():
+    rows = [r for r in _golden_rows() if r[0] == "rec"]
     assert rows
     for r in rows:
-        g, side, tau, k, word, bit = int(r[0]), r[1].strip(), int(r[2]), int(r[3]), int(r[4]), int(r[5])
-        assert oracle.block_bit_address(g, side, tau, k) == (word, bit), r
+        P, tau, idx = map(int, r[1:])
+        assert oracle.record_index(P, tau) == idx, r
+    # the records of a page are a permutation of its token pairs
+    for P in (32, 64, 96):
+        assert sorted(oracle.record_index(P, 2 * u) for u in range(P // 2)) == list(range(P // 2))
 
 
 @pytest.mark.parametrize("g", [8, 16])
@@ -58,9 +87,11 @@ def test_round_trip(g, b, side):
 
 
 def test_one_token_bytes_by_hand():
-    """g=16, K side, b=2, token 1 with code 3 at coordinate 0 and code 1 at
-    coordinate 8: token 1 is row 8 (hh=1); coordinate 0 -> slot 1 -> bit 4,
-    coordinate 8 -> slot 3 -> bit 12; plane 0 gets bits 4 and 12, plane 1 bit 4."""
+    """g=16, K side, b=2, P=32, token 1 with code 3 at coordinate 0 and code 1 at
+    coordinate 8.  Token 1 is row 8 (gid 0, hh 1); coordinate 0 has t4 0, ch 0 ->
+    slot 1; coordinate 8 has t4 0, ch 1 -> slot 3.  b=2 puts lane (0, 0) in word 0
+    at nibble bits 0-1: code 3 -> bits 4, 5; code 1 -> bit 12.  Token 1 is in pair
+    0, record 0: s at fp16 index 1, z at index 3."""
     P, g, b = 32, 16, 2
     page = np.zeros(b * P * g // 8 + 4 * P, dtype=np.uint8)
     codes = np.zeros((1, 16), np.uint8)
@@ -68,12 +99,11 @@ def test_one_token_bytes_by_hand():
     oracle.pack_group_into_page(page, g, "K", P, b, 0, b * P * g // 8, np.array([1]), codes,
                                 np.array([1.0], np.float16), np.array([-2.0], np.float16))
     words = page[: b * P * g // 8].view("<u4")
-    plane_words = P * g // 32
-    assert words[0] == (1 << 4) | (1 << 12)
-    assert words[plane_words + 0] == (1 << 4)
-    assert np.count_nonzero(words) == 2
+    assert words[0] == (1 << 4) | (1 << 5) | (1 << 12)
+    assert np.count_nonzero(words) == 1
     rec = page[b * P * g // 8:].view("<f2")
     assert rec[1] == 1.0 and rec[3] == -2.0 and rec[0] == 0 and rec[2] == 0
+    assert np.count_nonzero(rec) == 2
 
 
 def test_section_bytes_equal_budget_accounting():
@@ -103,37 +133,45 @@ def _rotr(x, n):
     return ((x >> n) | (x << (32 - n))) & 0xFFFFFFFF
 
 
-def _nibbles(words_by_plane, gid, t4, b):
-    """Kernel recipe: R = OR_p rotr(W_p[gid], t4 - p) & (0x11111111 << p) per
-    nibble plane group (planes 0-3 low accumulator, 4-7 high accumulator)."""
-    lo = hi = 0
-    for p in range(b):
-        w = int(words_by_plane[p][gid])
-        pp = p % 4
-        v = _rotr(w, t4 - pp) & (0x11111111 << pp)
-        if p < 4:
-            lo |= v
-        else:
-            hi |= v
-    return [((lo >> (4 * s)) & 0xF) | (((hi >> (4 * s)) & 0xF) << 4) for s in range(8)]
+def _slot_codes(block_words, gid, t4, b):
+    """Kernel recipe: this lane's 8 codes (slot order) from one block, by width.
+    b <= 4: one 32-bit word of nibbles, x; slot s is (x >> 4 s) & (2^b - 1)."""
+    w = [int(v) for v in block_words]
+    lane = 4 * gid + t4
+    if b == 8:
+        w0, w1 = w[2 * lane], w[2 * lane + 1]
+        byte = lambda x, i: (x >> (8 * i)) & 0xFF
+        return [byte(w0, 0), byte(w0, 1), byte(w1, 0), byte(w1, 1),
+                byte(w0, 2), byte(w0, 3), byte(w1, 2), byte(w1, 3)]
+    if b == 4:
+        x = w[lane]
+    elif b == 2:
+        x = w[2 * gid + t4 // 2] >> (2 * (t4 % 2))
+    elif b == 1:
+        x = w[gid] >> t4
+    else:  # b == 3
+        lo = w[2 * gid + t4 // 2] >> (2 * (t4 % 2))
+        hi = _rotr(w[16 + gid], t4 - 2)
+        x = (lo & 0x33333333) | (hi & 0xCCCCCCCC)
+    return [(x >> (4 * s)) & ((1 << b) - 1) for s in range(8)]
 
 
 @pytest.mark.parametrize("g", [8, 16])
 @pytest.mark.parametrize("side", ["K", "V"])
-@pytest.mark.parametrize("b", [1, 3, 8])
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 8])
 def test_layout_feeds_mma_fragments(g, side, b):
     rng = np.random.default_rng(7 * g + b + (side == "V"))
     tb = oracle.tokens_per_block(g)
-    P = 32
+    P = 64
     page = np.zeros(b * P * g // 8 + 4 * P, dtype=np.uint8)
     codes = rng.integers(0, 2 ** b, size=(P, g)).astype(np.uint8)
     oracle.pack_group_into_page(page, g, side, P, b, 0, b * P * g // 8, np.arange(P), codes,
                                 np.zeros(P, np.float16), np.zeros(P, np.float16))
-    words = page[: b * P * g // 8].view("<u4").reshape(b, P // tb, 8)
+    words = page[: b * P * g // 8].view("<u4").reshape(P // tb, 8 * b)
     for blk in range(P // tb):
         for lane in range(32):
             gid, t4 = lane >> 2, lane & 3
-            nib = _nibbles([words[p, blk] for p in range(b)], gid, t4, b)
+            nib = _slot_codes(words[blk], gid, t4, b)
             # register r holds the element pair (slot r, slot r + 4); see layout rules
             for mi in range(2 if g == 8 else 1):
                 n_elem = 8 if (g == 16 or side == "V") else 4
@@ -157,3 +195,20 @@ def test_layout_feeds_mma_fragments(g, side, b):
                         slot = mi + 2 * (i >> 2) + 4 * (i & 1)
                         tok, coord = 16 * mi + col, row
                     assert nib[slot] == codes[blk * tb + tok, coord]
+
+
+def test_records_feed_the_kernels_lanes():
+    """With P/16 tiles per page, the lane reading token pair j of tiles
+    t0 .. t0+3 finds them in 4 consecutive records starting at j*(P/16) + t0."""
+    P = 64
+    blocks = P * 16 // 8  # b = 1
+    page = np.zeros(blocks + 4 * P, dtype=np.uint8)
+    s = (np.arange(P) + 1).astype(np.float16)
+    oracle.pack_group_into_page(page, 16, "K", P, 1, 0, blocks, np.arange(P), np.zeros((P, 16), np.uint8), s,
+                                -s)
+    rec = page[blocks:].view("<f2").reshape(P // 2, 4)
+    for j in range(8):
+        for t in range(P // 16):
+            r = rec[j * (P // 16) + t]
+            tok = 16 * t + 2 * j
+            assert (r[0], r[1], r[2], r[3]) == (s[tok], s[tok + 1], -s[tok], -s[tok + 1])
