@@ -41,6 +41,7 @@ constexpr int kDecWarps = 4;
 constexpr int kMaxG = 8;          // kept groups per side handled by the decode kernels
 constexpr int kMaxKept = 128;     // kept coordinates per side
 constexpr int kMaxSplit = 256;    // context splits per (sequence, KV head)
+constexpr int kMaxSmemPerBlock = 227 * 1024;  // opt-in dynamic shared memory per CTA (sm_100)
 constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // bounded mbarrier waits
 constexpr float kPScaleLog2 = 8.f;   // p = 2^(s - m + 8): fp16 keeps small weights normal
 constexpr float kTwo24 = 16777216.f; // undo the 2^-24 of subnormal codes
@@ -73,11 +74,11 @@ struct DecodeArgs {
   int part_stride;
   int n_q;
   int n_kv;
+  int max_kept_v;
+  int d_h;
   float q_scale;
 };
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 // mma with a zero accumulator input (no register moves for C)
 __device__ __forceinline__ void mma_m16n8k16_z(float d[4], const uint32_t a[4], const uint32_t b[2]) {
@@ -105,6 +106,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 16-byte asynchronous global -> shared copy (both addresses 16-byte aligned)
+// and the wait for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
@@ -116,75 +124,95 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 // nt*4 + n/2, part n&1 (0: fp16(q_lat), 1: fp16(q_lat - fp16(q_lat))); rows
 // k = 2*(lane%4) + {0,1} (+8).  bz[nt][lane] likewise over group sums.
 // ---------------------------------------------------------------------------
+//
+// One CTA per (KV head, sequence, quarter z of the kept K coordinates): lane c
+// of each warp owns coordinate 32 z + c, warp w heads w and w + 4.  A quarter
+// holds whole groups (2 of 16 or 4 of 8), so the CTA writes every fragment of
+// its groups, and the bz lanes whose rows (2 t4, 2 t4 + 1) are its groups.
+// ---------------------------------------------------------------------------
+constexpr int kFoldThreads = 128;
+
 template <int G, int NT>
-__global__ void __launch_bounds__(256) fold_kernel(const DecodeArgs A) {
+__global__ void __launch_bounds__(kFoldThreads) fold_kernel(const DecodeArgs A) {
   const CodecDev* __restrict__ cd = A.cd;
-  const int a = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int a = blockIdx.x, b = blockIdx.y, z = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-  float* qlat_s = reinterpret_cast<float*>(smem + 128);            // [kMaxGQ][kMaxKept]
-  float* qsum_s = qlat_s + kMaxGQ * kMaxKept;                      // [kMaxGQ][kMaxG]
-  float* q_s = qsum_s + kMaxGQ * kMaxG;                            // [kMaxGQ][kMaxDHead]
-  float* w_s = q_s + kMaxGQ * kMaxDHead;                           // [d_h][n_kept]
+  __shared__ float q_s[kMaxGQ * kMaxDHead];
+  __shared__ float qlat_s[kMaxGQ][33];
+  __shared__ __align__(16) float w_s[kMaxDHead * 32];  // this quarter's columns of W_up^K
   const int gq = cd->gq, d_h = cd->d_h;
   const SideDev* sk = &cd->head[a].side[0];
   const int nk = sk->n_kept, nK = sk->n_groups;
-  const uint32_t wbytes = (uint32_t)nk * d_h * 4;
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-    if (wbytes) {
-      mbar_arrive_expect_tx(bar, wbytes);
-      bulk_copy_g2s(w_s, cd->w_up + sk->wup_off, wbytes, bar);
-    }
+  const float* w = cd->w_up + sk->wup_off;  // [d_h][nk]; nk is a multiple of 8
+  // all 16-byte pieces of the quarter in flight at once
+  for (int e = tid; e < d_h * 8; e += kFoldThreads) {
+    const int d = e >> 3, c4 = 32 * z + 4 * (e & 7);
+    if (c4 < nk) cp_async16(w_s + d * 32 + 4 * (e & 7), w + (size_t)d * nk + c4);
   }
   const float* qb = A.q + ((size_t)b * A.n_q + (size_t)a * gq) * d_h;
-  for (int e = tid; e < gq * d_h; e += blockDim.x) q_s[(e / d_h) * kMaxDHead + e % d_h] = qb[e];
+  for (int e = tid; e < gq * d_h; e += kFoldThreads) q_s[e] = qb[e];
+  cp_async_wait_all();
   __syncthreads();
-  bool ok = true;
-  if (wbytes) ok = mbar_wait_bounded(bar, 0, kWaitLimitNs);
-  if (!ok && tid == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
-  for (int idx = tid; idx < nk * gq; idx += blockDim.x) {
-    const int c = idx % nk, h = idx / nk;
-    float acc = 0.f;
-    for (int d = 0; d < d_h; ++d) acc = fmaf(q_s[h * kMaxDHead + d], w_s[d * nk + c], acc);
-    qlat_s[h * kMaxKept + c] = ok ? acc * A.q_scale : 0.f;
+  const int c = 32 * z + lane;
+  float acc0 = 0.f, acc1 = 0.f;
+  const int h0 = warp, h1 = warp + 4;
+  if (c < nk) {
+    const float* q0 = q_s + h0 * d_h;
+    const float* q1 = q_s + (h1 < gq ? h1 : h0) * d_h;
+#pragma unroll 8
+    for (int d = 0; d < d_h; ++d) {
+      const float wv = w_s[d * 32 + lane];
+      acc0 = fmaf(q0[d], wv, acc0);
+      acc1 = fmaf(q1[d], wv, acc1);
+    }
   }
+  qlat_s[h0][lane] = acc0 * A.q_scale;
+  qlat_s[h1][lane] = acc1 * A.q_scale;
   __syncthreads();
-  if (tid < gq * kMaxG) {
-    const int h = tid / kMaxG, j = tid % kMaxG;
-    float s = 0.f;
-    if (j < nK)
-      for (int k = 0; k < G; ++k) s += qlat_s[h * kMaxKept + j * G + k];
-    qsum_s[h * kMaxG + j] = s;
-  }
-  __syncthreads();
+  pdl_wait();  // the fragment buffer may still be read by an earlier decode's split kernel
+  // fragments of this quarter's groups
+  constexpr int kGroupsPerQ = 32 / G;
   uint2* out = A.frag + ((size_t)b * A.n_kv + a) * kFragWords;
-  for (int idx = tid; idx < (kMaxG + 1) * NT * 32; idx += blockDim.x) {
-    const int lane = idx % 32, row = idx / 32;  // row < kMaxG*NT: bq[j][nt]; then bz[nt]
-    const int gid = lane >> 2, t4 = lane & 3;
-    const bool is_bz = row >= kMaxG * NT;
-    const int j = is_bz ? 0 : row / NT, nt = is_bz ? row - kMaxG * NT : row % NT;
-    const int hl = nt * 4 + (gid >> 1);
-    const int part = gid & 1;
+  for (int idx = tid; idx < kGroupsPerQ * NT * 32; idx += kFoldThreads) {
+    const int ln = idx % 32, r = idx / 32;
+    const int jl = r / NT, nt = r % NT;
+    const int j = z * kGroupsPerQ + jl;
+    if (j >= kMaxG) continue;
+    const int gid = ln >> 2, t4 = ln & 3;
+    const int hl = nt * 4 + (gid >> 1), part = gid & 1;
     auto split_h = [&](float x) -> float {
       const float hi = __half2float(__float2half_rn(x));
       return part ? (x - hi) : hi;
     };
     uint2 v = make_uint2(0u, 0u);
-    if (hl < gq) {
-      if (is_bz) {
-        const float* qs = qsum_s + hl * kMaxG;
-        v.x = pack_half2(split_h(qs[2 * t4]), split_h(qs[2 * t4 + 1]));
-      } else if (j < nK) {
-        const float* base = qlat_s + hl * kMaxKept + j * G;
-        v.x = pack_half2(split_h(base[2 * t4]), split_h(base[2 * t4 + 1]));
-        if (G == 16) v.y = pack_half2(split_h(base[2 * t4 + 8]), split_h(base[2 * t4 + 9]));
-      }
+    if (hl < gq && j < nK) {
+      const float* base = &qlat_s[hl][jl * G];
+      v.x = pack_half2(split_h(base[2 * t4]), split_h(base[2 * t4 + 1]));
+      if (G == 16) v.y = pack_half2(split_h(base[2 * t4 + 8]), split_h(base[2 * t4 + 9]));
     }
-    out[(is_bz ? kMaxG * 2 + nt : j * NT + nt) * 32 + lane] = v;
+    out[(j * NT + nt) * 32 + ln] = v;
+  }
+  // bz rows k = 2 t4, 2 t4 + 1 are groups; lanes whose groups lie in this quarter
+  for (int idx = tid; idx < NT * 32; idx += kFoldThreads) {
+    const int ln = idx % 32, nt = idx / 32;
+    const int gid = ln >> 2, t4 = ln & 3;
+    const int j0 = 2 * t4;
+    if (j0 / kGroupsPerQ != z) continue;
+    const int hl = nt * 4 + (gid >> 1), part = gid & 1;
+    auto gsum = [&](int j) -> float {
+      float s = 0.f;
+      if (j < nK)
+        for (int k = 0; k < G; ++k) s += qlat_s[hl][(j - z * kGroupsPerQ) * G + k];
+      return s;
+    };
+    auto split_h = [&](float x) -> float {
+      const float hi = __half2float(__float2half_rn(x));
+      return part ? (x - hi) : hi;
+    };
+    uint2 v = make_uint2(0u, 0u);
+    if (hl < gq) v.x = pack_half2(split_h(gsum(j0)), split_h(gsum(j0 + 1)));
+    out[(kMaxG * 2 + nt) * 32 + ln] = v;
   }
 }
 
@@ -377,24 +405,14 @@ __device__ __forceinline__ void value_group(const uint8_t* __restrict__ blocks, 
   }
 }
 
-// Group tables in shared memory: per side, kept groups ordered by width class
-// (4, 2, 1, 3, 8), each entry {block offset, record offset, group index, width}
-// relative to the head section; class bounds; record offsets by group index.
-struct GroupTables {
-  int4 ord[2][kMaxG];
-  int cls[2][8];
-  int rec[2][kMaxG];
-  int wid[2][kMaxG];
-};
-
 template <int G, int NT, int CH, int B>
-__device__ __forceinline__ void key_class(const GroupTables& T, const uint8_t* sec, int chunk_blk_bytes_unit,
+__device__ __forceinline__ void key_class(const DecodeTables& T, const uint8_t* sec, int chunk_blk_bytes_unit,
                                           int rec_lane, const LaneAddr& L, const uint2* bq_s, int lane,
                                           int ci, float (&acc)[CH][NT][4]) {
   const int c1 = T.cls[0][ci + 1];
 #pragma unroll 1
   for (int c = T.cls[0][ci]; c < c1; ++c) {
-    const int4 g = T.ord[0][c];
+    const int4 g = *reinterpret_cast<const int4*>(T.ord[0][c]);
     uint2 bqj[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) bqj[nt] = bq_s[(g.z * NT + nt) * 32 + lane];
@@ -403,14 +421,14 @@ __device__ __forceinline__ void key_class(const GroupTables& T, const uint8_t* s
 }
 
 template <int G, int CH, int B, bool kMask>
-__device__ __forceinline__ void value_class(const GroupTables& T, const uint8_t* sec, int chunk_blk_bytes_unit,
+__device__ __forceinline__ void value_class(const DecodeTables& T, const uint8_t* sec, int chunk_blk_bytes_unit,
                                             int recA_lane, int recB_lane, const LaneAddr& L, float4* vacc,
                                             int lane, int ci, bool grew, float ae, float ao,
                                             const uint32_t (&pb)[CH][2], const uint32_t (&msk)[CH][2]) {
   const int c1 = T.cls[1][ci + 1];
 #pragma unroll 1
   for (int c = T.cls[1][ci]; c < c1; ++c) {
-    const int4 g = T.ord[1][c];
+    const int4 g = *reinterpret_cast<const int4*>(T.ord[1][c]);
     float4 v4 = vacc[g.z * 32 + lane];
     if (grew) {
       v4.x *= ae;
@@ -435,7 +453,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmBars) + warp * 8;
   uint2* bq_s = reinterpret_cast<uint2*>(smem + kSmBq);
-  GroupTables& T = *reinterpret_cast<GroupTables*>(smem + kSmGrp);
+  DecodeTables& T = *reinterpret_cast<DecodeTables*>(smem + kSmGrp);
   float4* vacc_s = reinterpret_cast<float4*>(smem + kSmAcc) + warp * kMaxG * 32;
   uint8_t* region = smem + kSmStages;
   uint8_t* my_stages = region + (size_t)warp * A.stages * A.stage_bytes;
@@ -446,7 +464,9 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   const int sec_off = hd->sec_off, sec_bytes = hd->sec_bytes;
   const int len = A.lengths[b];
   const int n_pages = (len + P - 1) / P;
-  const int per = (n_pages + A.n_split - 1) / A.n_split;
+  // pages per split: a multiple of the warp count, so the warps of a CTA get
+  // equal shares (trailing splits may get fewer pages or none)
+  const int per = ((n_pages + A.n_split - 1) / A.n_split + kDecWarps - 1) / kDecWarps * kDecWarps;
   const int p0 = min(split * per, n_pages), p1 = min(p0 + per, n_pages);
   const int count = (p1 - p0 > warp) ? (p1 - p0 - warp + kDecWarps - 1) / kDecWarps : 0;
   const SideDev* sk = &hd->side[0];
@@ -479,23 +499,12 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   if (lane == 0)
     for (int i = 0; i < min(S, my_count); ++i) issue(i);
 
-  // group tables (one thread per side)
-  if (tid < 2) {
-    const SideDev* sd = tid ? sv : sk;
-    constexpr int kOrder[5] = {4, 2, 1, 3, 8};
-    int n = 0;
-    for (int ci = 0; ci < 5; ++ci) {
-      T.cls[tid][ci] = n;
-      for (int j = 0; j < sd->n_groups; ++j) {
-        const GroupDev gd = sd->grp[j];
-        if (gd.b == kOrder[ci]) T.ord[tid][n++] = make_int4(gd.plane_off - sec_off, gd.sz_off - sec_off, j, gd.b);
-      }
-    }
-    T.cls[tid][5] = n;
-    for (int j = 0; j < kMaxG; ++j) {
-      T.rec[tid][j] = j < sd->n_groups ? sd->grp[j].sz_off - sec_off : -1;
-      T.wid[tid][j] = j < sd->n_groups ? sd->grp[j].b : 0;
-    }
+  // group tables (built on the host with the page layout)
+  {
+    static_assert(sizeof(DecodeTables) % 16 == 0, "DecodeTables must copy as int4");
+    const int4* src = reinterpret_cast<const int4*>(&hd->dec);
+    int4* dst = reinterpret_cast<int4*>(&T);
+    for (int e = tid; e < (int)(sizeof(DecodeTables) / 16); e += blockDim.x) dst[e] = src[e];
   }
   for (int j = 0; j < kMaxG; ++j) vacc_s[j * 32 + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
 
@@ -816,8 +825,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs A) {
   float* red = reinterpret_cast<float*>(smem + 64);      // 32 floats
   float* olat = red + 32;                                // [kMaxKept]
   float* wgt = olat + kMaxKept;                          // [kMaxSplit]
-  float* w_s = wgt + kMaxSplit;                          // [nkv][d_h]
-  float* p_s = w_s + kMaxKept * kMaxDHead;               // [ns][stride]
+  float* half_s = wgt + kMaxSplit;                       // [2][kMaxDHead]
+  float* w_s = half_s + 2 * kMaxDHead;                   // [max_kept_v][d_h]
+  float* p_s = w_s + A.max_kept_v * d_h;                 // [ns][stride]
   const uint32_t wbytes = (uint32_t)nkv * d_h * 4;
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -828,12 +838,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs A) {
     }
   }
   pdl_wait();  // the split partials are complete from here on
-  const float* pr = A.part + ((size_t)b * A.n_q + h) * ns * stride;
-  for (int e = tid; e < ns * stride; e += blockDim.x) p_s[e] = pr[e];
+  {
+    const float* src = A.part + ((size_t)b * A.n_q + h) * ns * stride;  // stride % 4 == 0
+    for (int e = tid; e < ns * stride / 4; e += blockDim.x) cp_async16(p_s + 4 * e, src + 4 * e);
+    cp_async_wait_all();
+  }
   __syncthreads();
+  const float* pr = p_s;
   const int warp = tid >> 5, lane = tid & 31;
   float mloc = -CUDART_INF_F;
-  for (int s = tid; s < ns; s += blockDim.x) mloc = fmaxf(mloc, p_s[s * stride]);
+  for (int s = tid; s < ns; s += blockDim.x) mloc = fmaxf(mloc, pr[(size_t)s * stride]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
   if (lane == 0) red[warp] = mloc;
@@ -843,10 +857,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs A) {
   __syncthreads();
   float lloc = 0.f;
   for (int s = tid; s < ns; s += blockDim.x) {
-    const float ms = p_s[s * stride];
+    const float ms = pr[(size_t)s * stride];
     const float w = (M == -CUDART_INF_F || ms == -CUDART_INF_F) ? 0.f : exp2f(ms - M);
     wgt[s] = w;
-    lloc += w * p_s[s * stride + 1];
+    lloc += w * pr[(size_t)s * stride + 1];
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, o);
@@ -855,52 +869,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs A) {
   float L = 0.f;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) L += red[w];
   const float invL = L > 0.f ? 1.f / L : 0.f;
-  for (int c = tid; c < nkv; c += blockDim.x) {
+  // latent output: each coordinate's sum over the splits in two halves
+  const int hs = (ns + 1) / 2;
+  for (int idx = tid; idx < 2 * nkv; idx += blockDim.x) {
+    const int c = idx % nkv, hf = idx / nkv;
     float acc = 0.f;
-    for (int s = 0; s < ns; ++s) acc = fmaf(wgt[s], p_s[s * stride + 2 + c], acc);
-    olat[c] = acc * invL;
+    for (int s = hf * hs; s < min(ns, hf * hs + hs); ++s) acc = fmaf(wgt[s], pr[(size_t)s * stride + 2 + c], acc);
+    half_s[hf * kMaxDHead + c] = acc;
   }
+  __syncthreads();
+  for (int c = tid; c < nkv; c += blockDim.x) olat[c] = (half_s[c] + half_s[kMaxDHead + c]) * invL;
   __syncthreads();
   bool ok = true;
   if (wbytes) ok = mbar_wait_bounded(bar, 0, kWaitLimitNs);
   if (!ok && tid == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
-  float* orow = A.out + ((size_t)b * A.n_q + h) * d_h;
-  for (int d = tid; d < d_h; d += blockDim.x) {
+  // out = olat W_up^V, each output's sum over the coordinates in two halves
+  const int hc = (nkv + 1) / 2;
+  for (int idx = tid; idx < 2 * d_h; idx += blockDim.x) {
+    const int d = idx % d_h, hf = idx / d_h;
     float acc = 0.f;
-    for (int c = 0; c < nkv; ++c) acc = fmaf(olat[c], w_s[c * d_h + d], acc);
-    orow[d] = ok ? acc : 0.f;
+    for (int c = hf * hc; c < min(nkv, hf * hc + hc); ++c) acc = fmaf(olat[c], w_s[c * d_h + d], acc);
+    half_s[hf * kMaxDHead + d] = acc;
   }
+  __syncthreads();
+  float* orow = A.out + ((size_t)b * A.n_q + h) * d_h;
+  for (int d = tid; d < d_h; d += blockDim.x) orow[d] = ok ? half_s[d] + half_s[kMaxDHead + d] : 0.f;
 }
 
-int fold_smem_bytes() { return 128 + (kMaxGQ * kMaxKept + kMaxGQ * kMaxG + kMaxGQ * kMaxDHead) * 4 + kMaxKept * kMaxDHead * 4; }
-int combine_smem_bytes(int ns, int stride) {
-  return 64 + (32 + kMaxKept + kMaxSplit + kMaxKept * kMaxDHead) * 4 + ns * stride * 4;
-}
-
-// Launch with programmatic stream serialisation (the kernel may start while the
-// previous one in the stream finishes; it waits with griddepcontrol.wait).  If
-// the attribute is refused, launch plainly: griddepcontrol.wait is then a no-op.
-template <typename... Args>
-cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, int smem, cudaStream_t st, Args... args) {
-  static bool pdl_ok = true;
-  if (pdl_ok) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-    if (e == cudaSuccess) return e;
-    (void)cudaGetLastError();
-    pdl_ok = false;
-  }
-  kern<<<grid, block, smem, st>>>(args...);
-  return cudaGetLastError();
+// Shared memory of the combine kernel: barrier, reductions, W_up^V of the
+// largest V side (n_kept x d_head floats) and the partial records.
+int combine_smem_bytes(int max_kept_v, int d_h, int ns, int stride) {
+  return 64 + (32 + kMaxKept + kMaxSplit + 2 * kMaxDHead) * 4 + max_kept_v * d_h * 4 + ns * stride * 4;
 }
 
 template <int G, int NT, int CH>
@@ -940,15 +939,12 @@ int sm_count() {
 
 template <int G, int NT, int CH>
 cudaError_t launch_all(const DecodeArgs& args, const DecodePlan& plan, int batch, int n_kv, int n_q, cudaStream_t st) {
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(fold_kernel<G, NT>), fold_smem_bytes());
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(split_kernel<G, NT, CH>), plan.smem_bytes);
   if (e != cudaSuccess) return e;
-  e = ensure_dynamic_smem(reinterpret_cast<const void*>(split_kernel<G, NT, CH>), plan.smem_bytes);
-  if (e != cudaSuccess) return e;
-  const int csm = combine_smem_bytes(args.n_split, args.part_stride);
+  const int csm = combine_smem_bytes(args.max_kept_v, args.d_h, args.n_split, args.part_stride);
   e = ensure_dynamic_smem(reinterpret_cast<const void*>(combine_kernel), csm);
   if (e != cudaSuccess) return e;
-  fold_kernel<G, NT><<<dim3(n_kv, batch), 256, fold_smem_bytes(), st>>>(args);
-  e = cudaGetLastError();
+  e = launch_dependent(fold_kernel<G, NT>, dim3(n_kv, batch, kMaxG * G / 32), dim3(kFoldThreads), 0, st, args);
   if (e != cudaSuccess) return e;
   e = launch_dependent(split_kernel<G, NT, CH>, dim3(args.n_split, n_kv, batch), dim3(kDecWarps * 32),
                        plan.smem_bytes, st, args);
@@ -985,9 +981,10 @@ cudaError_t ensure_dynamic_smem(const void* kern, int bytes) {
 DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq) {
   DecodePlan p{};
   p.stage_bytes = std::max(16, ((h.max_sec_bytes + 15) / 16) * 16);
-  // 2 stages per warp (more when sections are small) keep > 40 KB in flight per SM
-  const int budget = 64 * 1024;
-  p.stages = std::max(2, std::min(4, budget / (kDecWarps * p.stage_bytes)));
+  // up to 32 KB of stages per CTA: one stage per warp for the largest sections
+  // (so 4 CTAs fit an SM), up to 4 when sections are small
+  const int budget = 32 * 1024;
+  p.stages = std::max(1, std::min(4, budget / (kDecWarps * p.stage_bytes)));
   p.smem_bytes = kSmStages + std::max(kDecWarps * p.stages * p.stage_bytes, kMergeBytes);
   // context splits: fill one wave of resident CTAs when that wastes < 15% of the
   // slots, else two waves; the count does not depend on the context length, so a
@@ -999,10 +996,11 @@ DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq)
     const int ns2 = std::max(1, 2 * slots / units);
     if ((double)units * ns2 / (2.0 * slots) > (double)units * ns / slots) ns = ns2;
   }
-  ns = std::min(ns, kMaxSplit);
+  p.part_stride = ((2 + h.max_kept_v) + 3) / 4 * 4;
+  const int ns_fit = (kMaxSmemPerBlock - combine_smem_bytes(h.max_kept_v, h.d_h, 0, 0)) / (p.part_stride * 4);
+  ns = std::max(1, std::min({ns, kMaxSplit, ns_fit}));
   (void)max_pages_per_seq;
   p.n_split = ns;
-  p.part_stride = ((2 + h.max_kept_v) + 3) / 4 * 4;
   size_t off = 0;
   auto carve = [&](size_t bytes) {
     const size_t o = off;
@@ -1036,6 +1034,8 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
   args.part_stride = plan.part_stride;
   args.n_q = h.n_q;
   args.n_kv = h.n_kv;
+  args.max_kept_v = h.max_kept_v;
+  args.d_h = h.d_h;
   args.q_scale = 1.4426950408889634f / sqrtf((float)h.d_h);
   const bool two = h.gq > 4;
   if (h.group == 16)

@@ -24,6 +24,18 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- programmatic dependent launch -----------------------------------------
+// A kernel launched with programmatic stream serialisation may start while the
+// previous kernel in the stream runs, once every CTA of that kernel has called
+// pdl_launch_dependents (or exited).  pdl_wait blocks until the previous kernel
+// has completed and its memory is visible.  Rule for every libspectra kernel:
+// before pdl_wait touch only read-only codec data and the caller's inputs; read
+// predecessor outputs and write any shared buffer after it; and call pdl_wait
+// before exiting, so that each kernel's completion implies all earlier ones'.
+// Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ---- mbarrier + bulk copy (TMA, non-tensor form) -----------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

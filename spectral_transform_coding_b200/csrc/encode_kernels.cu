@@ -12,13 +12,13 @@ namespace spectra {
 
 // ---------------------------------------------------------------------------
 // latents[t][n] = sum_k H[t][k] * W_down[k][n]   for small T (decode steps).
-// W_down is stored transposed (wt[n][k], bf16); each warp owns 4 columns and
-// streams their rows once with 16-byte loads; H rows (small) come from L2.
+// W_down is stored transposed (wt[n][k], bf16).  A warp owns CPW columns and
+// streams their rows with 16-byte loads, KC/256 per column and lane in flight;
+// each KC-wide slice of up to ROWS H rows is staged once per CTA in shared
+// memory (loaded after the warp's W loads are issued, so the two overlap).
 // bf16 x bf16 products are exact in fp32; accumulation is fp32.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr int kGemvCols = 4;   // columns per warp
-constexpr int kGemvRows = 8;   // H rows per pass
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float f[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -30,49 +30,75 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float f[8]) {
 }
 }  // namespace
 
+template <int CPW, int ROWS, int KC>
 __global__ void __launch_bounds__(256) project_gemv_kernel(const uint16_t* __restrict__ wt,
                                                            const uint16_t* __restrict__ H, int T,
                                                            int d_model, int n_eff,
                                                            float* __restrict__ C, int64_t ldc) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int n0 = warp * kGemvCols;
-  if (n0 >= n_eff) return;
-  for (int t0 = 0; t0 < T; t0 += kGemvRows) {
-    float acc[kGemvCols][kGemvRows];
+  constexpr int BATCH = KC / 256;  // 16-byte chunks per column and lane per slice
+  __shared__ __align__(16) uint16_t h_s[ROWS * KC];
+  const int tid = threadIdx.x;
+  const int warp = (blockIdx.x * blockDim.x + tid) >> 5;
+  const int lane = tid & 31;
+  const int n0 = warp * CPW;
+  const bool active = n0 < n_eff;  // every warp stages H and meets the barriers
+  pdl_launch_dependents();
+  for (int t0 = 0; t0 < T; t0 += ROWS) {
+    const int nr = min(ROWS, T - t0);
+    float acc[CPW][ROWS];
 #pragma unroll
-    for (int c = 0; c < kGemvCols; ++c)
+    for (int c = 0; c < CPW; ++c)
 #pragma unroll
-      for (int r = 0; r < kGemvRows; ++r) acc[c][r] = 0.f;
-    for (int k = lane * 8; k < d_model; k += 256) {
-      float w[kGemvCols][8];
+      for (int r = 0; r < ROWS; ++r) acc[c][r] = 0.f;
+    for (int kc0 = 0; kc0 < d_model; kc0 += KC) {
+      uint4 wv[CPW][BATCH];
 #pragma unroll
-      for (int c = 0; c < kGemvCols; ++c) {
-        const int n = min(n0 + c, n_eff - 1);
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(wt + (size_t)n * d_model + k));
-        bf16x8_to_f32(v, w[c]);
+      for (int i = 0; i < BATCH; ++i)
+#pragma unroll
+        for (int c = 0; c < CPW; ++c) {
+          const int k = kc0 + lane * 8 + 256 * i;
+          const int n = min(n0 + c, n_eff - 1);
+          wv[c][i] = (active && k < d_model)
+                         ? __ldg(reinterpret_cast<const uint4*>(wt + (size_t)n * d_model + k))
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+      pdl_wait();       // H may come from the previous kernel; W_down is read-only codec data
+      __syncthreads();  // the previous slice's readers are done
+      for (int e = tid; e < ROWS * KC / 8; e += blockDim.x) {
+        const int r = e / (KC / 8), col = (e % (KC / 8)) * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < nr && kc0 + col < d_model)
+          v = __ldg(reinterpret_cast<const uint4*>(H + (size_t)(t0 + r) * d_model + kc0 + col));
+        *reinterpret_cast<uint4*>(h_s + r * KC + col) = v;
       }
+      __syncthreads();
 #pragma unroll
-      for (int r = 0; r < kGemvRows; ++r) {
-        if (t0 + r < T) {
-          float h[8];
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(H + (size_t)(t0 + r) * d_model + k));
-          bf16x8_to_f32(v, h);
+      for (int i = 0; i < BATCH; ++i) {
+        const int kl = lane * 8 + 256 * i;
+        float w[CPW][8];
 #pragma unroll
-          for (int c = 0; c < kGemvCols; ++c)
+        for (int c = 0; c < CPW; ++c) bf16x8_to_f32(wv[c][i], w[c]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[c][r] = fmaf(w[c][e], h[e], acc[c][r]);
+        for (int r = 0; r < ROWS; ++r) {
+          if (r < nr) {
+            float h[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(h_s + r * KC + kl), h);
+#pragma unroll
+            for (int c = 0; c < CPW; ++c)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[c][r] = fmaf(w[c][e], h[e], acc[c][r]);
+          }
         }
       }
     }
 #pragma unroll
-    for (int c = 0; c < kGemvCols; ++c)
+    for (int c = 0; c < CPW; ++c)
 #pragma unroll
-      for (int r = 0; r < kGemvRows; ++r) {
+      for (int r = 0; r < ROWS; ++r) {
         float v = acc[c][r];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0 && n0 + c < n_eff && t0 + r < T) C[(size_t)(t0 + r) * ldc + n0 + c] = v;
+        if (lane == 0 && active && n0 + c < n_eff && r < nr) C[(size_t)(t0 + r) * ldc + n0 + c] = v;
       }
   }
 }
@@ -88,6 +114,8 @@ __global__ void __launch_bounds__(1024) append_plan_kernel(
     const int32_t* __restrict__ seq_ids, int T, int batch, int32_t* __restrict__ lengths,
     const int32_t* __restrict__ page_table, int max_pages, int64_t n_pool_pages, int P,
     int32_t* __restrict__ pos_out, int32_t* __restrict__ ok_flag, int32_t* __restrict__ err) {
+  pdl_launch_dependents();
+  pdl_wait();  // lengths, page table and seq_ids may come from earlier kernels
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
@@ -234,6 +262,8 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
   constexpr int TB = 256 / G;               // tokens per 256-bit block
   constexpr int LANES_PER_TOKENSET = TB;    // 16 or 32
   constexpr int GROUPS_PER_WARP = 32 / LANES_PER_TOKENSET;
+  pdl_launch_dependents();
+  pdl_wait();  // latents and the append plan come from the preceding kernels
   if (*ok_flag == 0) return;
   const int a = blockIdx.y >> 1, side = blockIdx.y & 1;
   const SideDev& sd = cd->head[a].side[side];
@@ -306,17 +336,25 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
 // ---------------------------------------------------------------------------
 cudaError_t launch_project_gemv(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
                                 float* C, int64_t ldc, cudaStream_t st) {
-  const int warps = (h.n_eff + kGemvCols - 1) / kGemvCols;
-  const int blocks = (warps * 32 + 255) / 256;
-  project_gemv_kernel<<<blocks, 256, 0, st>>>(wt, H, T, h.d_model, h.n_eff, C, ldc);
-  return cudaGetLastError();
+  // one column per warp for single-token steps (a whole 4096-wide row in flight
+  // per warp); two columns per warp and 16 H rows per pass for larger batches
+  if (T <= 1) {
+    const int blocks = (h.n_eff * 32 + 255) / 256;
+    return launch_dependent(project_gemv_kernel<1, 1, 4096>, dim3(blocks), dim3(256), 0, st, wt, H, T, h.d_model,
+                            h.n_eff, C, ldc);
+  } else {
+    const int warps = (h.n_eff + 1) / 2;
+    const int blocks = (warps * 32 + 255) / 256;
+    return launch_dependent(project_gemv_kernel<2, 16, 1024>, dim3(blocks), dim3(256), 0, st, wt, H, T,
+                            h.d_model, h.n_eff, C, ldc);
+  }
 }
 
 cudaError_t launch_append_plan(const int32_t* seq_ids, int T, const spectra_cache& cache, int P,
                                int32_t* pos, int32_t* ok_flag, int32_t* err, cudaStream_t st) {
-  append_plan_kernel<<<1, 1024, 0, st>>>(seq_ids, T, cache.batch, cache.lengths, cache.page_table,
-                                         cache.max_pages_per_seq, cache.n_pages, P, pos, ok_flag, err);
-  return cudaGetLastError();
+  return launch_dependent(append_plan_kernel, dim3(1), dim3(1024), 0, st, seq_ids, T, (int)cache.batch,
+                          cache.lengths, cache.page_table, (int)cache.max_pages_per_seq, (int64_t)cache.n_pages, P,
+                          pos, ok_flag, err);
 }
 
 cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const float* C, int64_t ldc,
@@ -325,14 +363,12 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
   const int tb = 256 / h.group;
   dim3 grid((T + tb - 1) / tb, h.n_kv * 2);
   if (h.group == 16)
-    quantize_append_kernel<16><<<grid, 128, 0, st>>>(d, C, ldc, seq_ids, pos, ok_flag, T,
-                                                     (uint8_t*)cache.pool, cache.page_table,
-                                                     cache.max_pages_per_seq);
-  else
-    quantize_append_kernel<8><<<grid, 128, 0, st>>>(d, C, ldc, seq_ids, pos, ok_flag, T,
-                                                    (uint8_t*)cache.pool, cache.page_table,
-                                                    cache.max_pages_per_seq);
-  return cudaGetLastError();
+    return launch_dependent(quantize_append_kernel<16>, grid, dim3(128), 0, st, d, C, ldc, seq_ids, pos,
+                            (const int32_t*)ok_flag, T, (uint8_t*)cache.pool, cache.page_table,
+                            (int)cache.max_pages_per_seq);
+  return launch_dependent(quantize_append_kernel<8>, grid, dim3(128), 0, st, d, C, ldc, seq_ids, pos,
+                          (const int32_t*)ok_flag, T, (uint8_t*)cache.pool, cache.page_table,
+                          (int)cache.max_pages_per_seq);
 }
 
 }  // namespace spectra

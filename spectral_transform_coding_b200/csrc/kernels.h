@@ -7,6 +7,31 @@
 
 namespace spectra {
 
+// Launch with programmatic stream serialisation (see pdl_wait in
+// device_common.cuh); if the attribute is refused, launch plainly.
+template <typename... Args>
+cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, int smem, cudaStream_t st, Args... args) {
+  static bool pdl_ok = true;
+  if (pdl_ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e == cudaSuccess) return e;
+    (void)cudaGetLastError();
+    pdl_ok = false;
+  }
+  kern<<<grid, block, smem, st>>>(args...);
+  return cudaGetLastError();
+}
+
 // encode_kernels.cu
 cudaError_t launch_project_gemv(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
                                 float* C, int64_t ldc, cudaStream_t st);
