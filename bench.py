@@ -403,19 +403,130 @@ def run_gpu(args, rank, world):
     return result
 
 
+def run_prefill(args):
+    """Prefill encode (one 65,536-token bf16 chunk for all KV heads, 4x and 8x
+    budgets), then one decode step: encode tokens/s, the tensor-core projection's
+    TFLOP/s and the quantise/pack kernel's GB/s.  One JSON line per budget."""
+    import torch
+
+    import spectral_transform_coding_b200 as st
+    from spectral_transform_coding_b200.codec import make_config
+    from workloads import get_config
+    from workloads.synthetic import _basis
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    out = []
+    for name in ("prefill", "prefill8"):
+        cfg = get_config(name)
+        T, P = args.prefill_tokens or cfg.prefill_tokens, cfg.page_tokens
+        gen = torch.Generator(device=dev)
+        basis = _basis(cfg.d_model, cfg.seed)
+        lam = torch.arange(1, cfg.d_model + 1, device=dev, dtype=torch.float32) ** (-cfg.spectrum_exp)
+        q1 = torch.from_numpy(basis[1]).to(dev, torch.float32)
+        q2 = torch.from_numpy(basis[2]).to(dev, torch.float32) if basis[0] == "kron" else None
+
+        def acts(n, seed):
+            gen.manual_seed(seed)
+            y = torch.randn((n, cfg.d_model), generator=gen, device=dev) * lam.sqrt()
+            if q2 is None:
+                h = y @ q1.T
+            else:
+                a_, b_ = q1.shape[0], q2.shape[0]
+                h = torch.einsum("ia,nab,jb->nij", q1, y.view(n, a_, b_), q2).reshape(n, a_ * b_)
+            return h.to(torch.bfloat16)
+
+        c = make_config(cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head, cfg.rank, cfg.group,
+                        cfg.budget_bits, cfg.count_overhead, P)
+        kvw = cfg.n_kv_heads * cfg.d_head
+        gen.manual_seed(1000 * cfg.seed)
+        W_K = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+        W_V = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+        codec = st.Codec.calibrate(c, acts(cfg.calib_tokens, 7000), W_K, W_V)
+        del W_K, W_V
+        H = acts(T, 12345)
+        cache = st.LatentCache(codec, batch=1, max_pages_per_seq=(T + P - 1) // P + 1, device=dev, zero=False)
+        seq = torch.zeros(T, dtype=torch.int32, device=dev)
+        ws = torch.empty(codec.encode_workspace_bytes(T), dtype=torch.uint8, device=dev)
+        lat = torch.empty((T, codec.n_eff), dtype=torch.float32, device=dev)
+        stream = torch.cuda.Stream(device=dev)
+        q = (torch.randn((1, cfg.n_q_heads, cfg.d_head), generator=gen, device=dev) * 0.5).contiguous()
+        o = torch.empty_like(q)
+        dws = torch.zeros(codec.decode_workspace_bytes(1, cache.capacity), dtype=torch.uint8, device=dev)
+
+        def timed(fn, reps):
+            tot = 0.0
+            for r in range(reps + 2):
+                cache.lengths.zero_()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                torch.cuda.synchronize()
+                if r >= 2:
+                    tot += e0.elapsed_time(e1)
+            return tot / reps
+
+        reps = max(3, min(args.steps, 10))
+        t_enc = timed(lambda: codec.encode_append(cache, H, seq, workspace=ws, stream=stream), reps)
+        t_proj = timed(lambda: codec.project(H, out=lat, stream=stream), reps)
+        t_quant = timed(lambda: codec.quantize_append(cache, lat, seq, workspace=ws, stream=stream), reps)
+        cache.lengths.zero_()
+        codec.encode_append(cache, H, seq, workspace=ws, stream=stream)  # leave the cache full for decode
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                codec.decode_attend(cache, q, o, workspace=dws, stream=stream)
+            e0.record(stream)
+            for _ in range(10):
+                codec.decode_attend(cache, q, o, workspace=dws, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        t_dec = e0.elapsed_time(e1) / 10
+        codec.device_status(stream)
+        flops = 2.0 * cfg.d_model * codec.n_eff * T
+        qbytes = T * (4.0 * codec.n_eff + codec.page_bytes / P)
+        tfl = flops / (t_proj / 1e3) / 1e12
+        gbs = qbytes / (t_quant / 1e3) / 1e9
+        out.append({
+            "metric": "prefill encode-append tokens/s", "value": T / (t_enc / 1e3), "unit": "tokens/s",
+            "workload": f"{name}: {T} tokens x (d_model {cfg.d_model}, {cfg.n_kv_heads} kv heads, "
+                        f"{cfg.budget_bits} bits/side), one chunk, then one decode step",
+            "encode_ms": t_enc, "n_eff": codec.n_eff,
+            "projection": {"ms": t_proj, "tflops": tfl, "peak": peaks["bf16_tflops"],
+                           "frac": tfl / peaks["bf16_tflops"], "kernel": "gemm_tcgen05_kernel (bf16, fp32 out)"},
+            "quantize_pack": {"ms": t_quant, "gbs": gbs, "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+                              "bytes": qbytes},
+            "decode_after_us": t_dec * 1e3, "peak_src": peaks["src"],
+        })
+    for r in out:
+        print(json.dumps(r), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="llama", choices=sorted(MODEL_LAYERS))
+    ap.add_argument("--workload", default="llama", choices=sorted(MODEL_LAYERS) + ["prefill"])
     ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-tokens", type=int, default=0,
+                    help="prefill mode: tokens in the chunk (default: the workload's 65,536)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     from workloads import get_config
+    if args.workload == "prefill":
+        if args.impl == "reference" or rank != 0:
+            return 0
+        return run_prefill(args)
     cfg = get_config(args.workload)
 
     if args.impl == "reference":

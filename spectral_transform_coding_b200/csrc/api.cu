@@ -600,6 +600,12 @@ spectra_status spectra_encode_append(const spectra_codec* c, const spectra_cache
   s = check_device(c);
   if (s != SPECTRA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T <= kFusedMaxT) {
+    // decode steps: projection, quantisation and packing fused per kept group
+    CUDA_TRY(launch_encode_fused(c->h, c->d, static_cast<const uint16_t*>(H), seq_ids, (int)T, *cache,
+                                 latents_out, st));
+    return SPECTRA_OK;
+  }
   uint8_t* w = static_cast<uint8_t*>(workspace);
   const size_t lat_off = ((size_t)T * 4 + 255) / 256 * 256 + 256;
   float* C = latents_out ? latents_out : reinterpret_cast<float*>(w + lat_off);

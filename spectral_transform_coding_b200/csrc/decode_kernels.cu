@@ -113,10 +113,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
-  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
 
 // ---------------------------------------------------------------------------
 // fold: q_lat[h][c] = (q_h . W_up^K[c]) * log2(e)/sqrt(d_h) and group sums, as
@@ -356,8 +352,8 @@ __device__ __forceinline__ void key_group(const uint8_t* __restrict__ blocks, co
     const int blk = tt / kBlockTiles;
     uint32_t av[4];
     frag_k<G, B>(p + blk * (B * 32), p1 + blk * (B * 32), lane_sh<B>(L), L.rot1, tt & 1, av);
-    const float sA = __half2float(__ushort_as_half((unsigned short)(sp[tt] & 0xffffu)));
-    float sB = __half2float(__ushort_as_half((unsigned short)(sp[tt] >> 16)));
+    float sA, sB;
+    half2_to_floats(sp[tt], sA, sB);
     if (B == 8) sB *= 16.f;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -400,7 +396,7 @@ __device__ __forceinline__ void value_group(const uint8_t* __restrict__ blocks, 
     frag_v<G, B>(p + blk * (B * 32), p1 + blk * (B * 32), lane_sh<B>(L), L.rot1, tt & 1, av);
     const uint32_t a0 = kMask ? (s0[tt] & msk[tt][0]) : s0[tt];
     const uint32_t a1 = kMask ? (s1[tt] & msk[tt][1]) : s1[tt];
-    const uint32_t bj[2] = {hmul2_u32(pb[tt][0], a0), hmul2_u32(pb[tt][1], a1)};
+    const uint32_t bj[2] = {hmul2_bits(pb[tt][0], a0), hmul2_bits(pb[tt][1], a1)};
     mma_m16n8k16(va, av, bj);
   }
 }
@@ -511,8 +507,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   // ---- 2. the folded query (written by the fold grid) -----------------------
   pdl_wait();
   {
+    // rows j*NT + nt (j < kMaxG) and the bz rows kMaxG*2 + nt
     const uint2* src = A.frag + ((size_t)b * A.n_kv + a) * kFragWords;
-    for (int e = tid; e < kFragWords; e += blockDim.x) bq_s[e] = src[e];
+    for (int e = tid; e < kMaxG * NT * 32; e += blockDim.x) bq_s[e] = src[e];
+    for (int e = tid; e < NT * 32; e += blockDim.x) bq_s[kMaxG * 2 * 32 + e] = src[kMaxG * 2 * 32 + e];
   }
   __syncthreads();
   uint32_t bz[NT][2];
@@ -653,14 +651,17 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
       // tokens (2t4, 2t4+1) and (2t4+8, 2t4+9)
       uint32_t pb[CH][2];
       uint32_t msk[CH][2];
+      float off[NT];  // p = 2^(s - m + 8)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) off[nt] = kPScaleLog2 - m_run[nt];
       const int src0 = (t4 << 2) | (gid & 3), src1 = ((t4 + 4) << 2) | (gid & 3);
 #pragma unroll
       for (int tt = 0; tt < CH; ++tt) {
         uint32_t p01[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const float pa = ex2_approx(sc[tt][nt][0] - m_run[nt] + kPScaleLog2);
-          const float pv = ex2_approx(sc[tt][nt][1] - m_run[nt] + kPScaleLog2);
+          const float pa = ex2_approx(sc[tt][nt][0] + off[nt]);
+          const float pv = ex2_approx(sc[tt][nt][1] + off[nt]);
           l_run[nt] += pa + pv;
           p01[nt] = pack_half2(pa, pv);
         }
@@ -713,7 +714,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
         }
 #pragma unroll
         for (int tt = 0; tt < CH; ++tt) {
-          const uint32_t az[4] = {za[tt] & msk[tt][0], 0u, zb[tt] & msk[tt][1], 0u};
+          const uint32_t az[4] = {partial ? (za[tt] & msk[tt][0]) : za[tt], 0u,
+                                  partial ? (zb[tt] & msk[tt][1]) : zb[tt], 0u};
           mma_m16n8k16(dz, az, pb[tt]);
         }
       }
@@ -794,18 +796,20 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   }
   __syncthreads();
   float* part = A.part + ((size_t)(b * A.n_q + a * gq) * A.n_split + split) * A.part_stride;
-  for (int idx = tid; idx < gq * (2 + nkv); idx += blockDim.x) {
-    const int hl = idx / (2 + nkv), c = idx % (2 + nkv);
+  for (int hl = 0; hl < gq; ++hl) {
     const float* wt = wts + hl * (kDecWarps + 2);
-    float v;
-    if (c < 2) {
-      v = wt[kDecWarps + c];
-    } else {
-      v = 0.f;
+    float* dst = part + (size_t)hl * A.n_split * A.part_stride;
+    for (int c = tid; c < 2 + nkv; c += blockDim.x) {
+      float v;
+      if (c < 2) {
+        v = wt[kDecWarps + c];
+      } else {
+        v = 0.f;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) v = fmaf(wt[w], wsm[(w * gq + hl) * rec + c], v);
+        for (int w = 0; w < kDecWarps; ++w) v = fmaf(wt[w], wsm[(w * gq + hl) * rec + c], v);
+      }
+      dst[c] = v;
     }
-    part[(size_t)hl * A.n_split * A.part_stride + c] = v;
   }
 }
 

@@ -112,16 +112,35 @@ __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+// fp16x2 helpers on 32-bit registers (PTX: half extraction is free in the
+// conversion instruction; no round trip through __half objects)
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void half2_to_floats(uint32_t x, float& lo, float& hi) {
+  asm("{\n .reg .f16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(x));
 }
 
 __device__ __forceinline__ float half_lo(uint32_t x) {
-  return __half2float(__ushort_as_half((unsigned short)(x & 0xffffu)));
+  float lo, hi;
+  half2_to_floats(x, lo, hi);
+  return lo;
 }
 __device__ __forceinline__ float half_hi(uint32_t x) {
-  return __half2float(__ushort_as_half((unsigned short)(x >> 16)));
+  float lo, hi;
+  half2_to_floats(x, lo, hi);
+  return hi;
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 }  // namespace spectra

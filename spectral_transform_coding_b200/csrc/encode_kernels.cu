@@ -172,6 +172,33 @@ namespace {
 
 __device__ __forceinline__ float sat16(float x) { return fminf(fmaxf(x, -65504.f), 65504.f); }
 
+// One token's group of G fp32 latents at width b (every step one IEEE fp32
+// operation): s = fp16(sat((max - min) / (2^b - 1))), z = fp16(sat(min)),
+// code = clamp(rint((x - z) / s), 0, 2^b - 1), all codes 0 when s == 0.
+template <int G>
+__device__ __forceinline__ void quantize_group(const float (&x)[G], int b, __half& s_h, __half& z_h,
+                                               uint32_t (&code)[G]) {
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int k = 1; k < G; ++k) {
+    mn = fminf(mn, x[k]);
+    mx = fmaxf(mx, x[k]);
+  }
+  const float levels = (float)((1 << b) - 1);
+  s_h = __float2half_rn(sat16(__fdiv_rn(__fsub_rn(mx, mn), levels)));
+  z_h = __float2half_rn(sat16(mn));
+  const float sf = __half2float(s_h), zf = __half2float(z_h);
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    float c = 0.f;
+    if (sf > 0.f) {
+      const float t = __fdiv_rn(__fsub_rn(x[k], zf), sf);
+      c = fminf(fmaxf(rintf(t), 0.f), levels);
+    }
+    code[k] = (uint32_t)c;
+  }
+}
+
 // Fragment position (gid, t4, slot) of entry (token tb of the block, coordinate k).
 template <int G>
 __device__ __forceinline__ void k_side_pos(int tb, int k, int* gid, int* t4, int* slot) {
@@ -204,25 +231,29 @@ __device__ __forceinline__ void v_side_pos(int tb, int k, int* gid, int* t4, int
 }
 
 // Pending bits of one block word: consecutive entries that land in the same word
-// are merged and written with one atomicAnd/atomicOr pair.
+// are merged.  Global words (kShared = false) are written with one atomicAnd /
+// atomicOr pair (other tokens of the block may be written concurrently or may
+// hold stale bits); a zeroed shared-memory copy of the block only needs the OR.
 struct WordBits {
   int w;
   uint32_t mask, val;
 };
 
+template <bool kShared>
 __device__ __forceinline__ void flush_word(uint32_t* blk, WordBits& a) {
   if (a.w >= 0) {
-    atomicAnd(blk + a.w, ~a.mask);
+    if (!kShared) atomicAnd(blk + a.w, ~a.mask);
     atomicOr(blk + a.w, a.val);
   }
   a.w = -1;
   a.mask = a.val = 0u;
 }
 
+template <bool kShared>
 __device__ __forceinline__ void put_bits(uint32_t* blk, WordBits& a, int w, int shift, uint32_t width_mask,
                                          uint32_t v) {
   if (w != a.w) {
-    flush_word(blk, a);
+    flush_word<kShared>(blk, a);
     a.w = w;
   }
   a.mask |= width_mask << shift;
@@ -235,20 +266,45 @@ __device__ __forceinline__ void put_bits(uint32_t* blk, WordBits& a, int w, int 
 //   b = 1: word gid, bit 4 slot + t4;
 //   b = 3: bits 0-1 as b = 2, bit 2 as b = 1 in words 16 + gid (second pending word);
 //   b = 8: word 2 (4 gid + t4) + (slot / 2) % 2, byte (slot % 2) + 2 (slot / 4).
+template <bool kShared>
 __device__ __forceinline__ void put_code(uint32_t* blk, WordBits& a, WordBits& a1, int b, int gid, int t4,
                                          int slot, uint32_t code) {
   switch (b) {
-    case 4: put_bits(blk, a, 4 * gid + t4, 4 * slot, 0xFu, code); break;
-    case 2: put_bits(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code); break;
-    case 1: put_bits(blk, a, gid, 4 * slot + t4, 0x1u, code); break;
+    case 4: put_bits<kShared>(blk, a, 4 * gid + t4, 4 * slot, 0xFu, code); break;
+    case 2: put_bits<kShared>(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code); break;
+    case 1: put_bits<kShared>(blk, a, gid, 4 * slot + t4, 0x1u, code); break;
     case 3:
-      put_bits(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code);
-      put_bits(blk, a1, 16 + gid, 4 * slot + t4, 0x1u, code >> 2);
+      put_bits<kShared>(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code);
+      put_bits<kShared>(blk, a1, 16 + gid, 4 * slot + t4, 0x1u, code >> 2);
       break;
     default:
-      put_bits(blk, a, 2 * (4 * gid + t4) + ((slot >> 1) & 1), 8 * ((slot & 1) + 2 * (slot >> 2)), 0xFFu, code);
+      put_bits<kShared>(blk, a, 2 * (4 * gid + t4) + ((slot >> 1) & 1), 8 * ((slot & 1) + 2 * (slot >> 2)), 0xFFu,
+                        code);
       break;
   }
+}
+
+// Scale/zero of page token tau: record of its pair u = tau/2 at index
+// (u % 8) * (P/16) + u / 8, fp16 {s[2u], s[2u+1], z[2u], z[2u+1]}.
+__device__ __forceinline__ void put_record(uint8_t* recs, int P, int tau, __half s_h, __half z_h) {
+  const int u = tau >> 1;
+  __half* rec = reinterpret_cast<__half*>(recs + 8 * ((u & 7) * (P >> 4) + (u >> 3)));
+  rec[tau & 1] = s_h;
+  rec[2 + (tau & 1)] = z_h;
+}
+
+template <int G, bool kShared>
+__device__ __forceinline__ void put_codes(uint32_t* blk, int side, int tb, int b, const uint32_t (&code)[G]) {
+  WordBits acc{-1, 0u, 0u}, acc1{-1, 0u, 0u};
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    int gid, t4, slot;
+    if (side == 0) k_side_pos<G>(tb, k, &gid, &t4, &slot);
+    else v_side_pos<G>(tb, k, &gid, &t4, &slot);
+    put_code<kShared>(blk, acc, acc1, b, gid, t4, slot, code[k]);
+  }
+  flush_word<kShared>(blk, acc);
+  flush_word<kShared>(blk, acc1);
 }
 
 }  // namespace
@@ -268,7 +324,14 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
   const int a = blockIdx.y >> 1, side = blockIdx.y & 1;
   const SideDev& sd = cd->head[a].side[side];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * TB + (lane % TB);
+  // This CTA's TB input tokens fill one whole block when they exist, belong to
+  // one sequence and start at a block boundary (positions of one sequence are
+  // consecutive): then each group's block is assembled in shared memory and
+  // stored whole; otherwise tokens merge their bits into the page with atomics.
+  const int i0 = blockIdx.x * TB;
+  const bool full = i0 + TB <= T && seq_ids[i0] == seq_ids[i0 + TB - 1] && pos[i0] % TB == 0;
+  __shared__ __align__(16) uint32_t wbuf[4][GROUPS_PER_WARP][64];
+  const int i = i0 + (lane % TB);
   if (i >= T) return;
   const int P = cd->P;
   const int p_tok = pos[i];
@@ -292,43 +355,188 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
       x[4 * q + 2] = v.z;
       x[4 * q + 3] = v.w;
     }
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int k = 1; k < G; ++k) {
-      mn = fminf(mn, x[k]);
-      mx = fmaxf(mx, x[k]);
-    }
-    const float levels = (float)((1 << b) - 1);
-    const __half s_h = __float2half_rn(sat16(__fdiv_rn(__fsub_rn(mx, mn), levels)));
-    const __half z_h = __float2half_rn(sat16(mn));
-    const float sf = __half2float(s_h), zf = __half2float(z_h);
+    __half s_h, z_h;
     uint32_t code[G];
-#pragma unroll
-    for (int k = 0; k < G; ++k) {
-      float c = 0.f;
-      if (sf > 0.f) {
-        const float t = __fdiv_rn(__fsub_rn(x[k], zf), sf);
-        c = fminf(fmaxf(rintf(t), 0.f), levels);
-      }
-      code[k] = (uint32_t)c;
-    }
+    quantize_group<G>(x, b, s_h, z_h, code);
     uint32_t* blkw = reinterpret_cast<uint32_t*>(page + gd.plane_off + blk * (32 * b));
-    WordBits acc{-1, 0u, 0u}, acc1{-1, 0u, 0u};
-#pragma unroll
-    for (int k = 0; k < G; ++k) {
-      int gid, t4, slot;
-      if (side == 0) k_side_pos<G>(tb, k, &gid, &t4, &slot);
-      else v_side_pos<G>(tb, k, &gid, &t4, &slot);
-      put_code(blkw, acc, acc1, b, gid, t4, slot, code[k]);
+    if (full) {
+      // the TB lanes holding this group (one half-warp for G = 16) own the block
+      const unsigned hm = GROUPS_PER_WARP == 2 ? (0xFFFFu << (16 * (lane >> 4))) : 0xFFFFFFFFu;
+      const int sub = lane % LANES_PER_TOKENSET;
+      uint32_t* wb = wbuf[warp][lane / LANES_PER_TOKENSET];
+      for (int w = sub; w < 8 * b; w += LANES_PER_TOKENSET) wb[w] = 0u;
+      __syncwarp(hm);
+      put_codes<G, true>(wb, side, tb, b, code);
+      __syncwarp(hm);
+      for (int w4 = sub; w4 < 2 * b; w4 += LANES_PER_TOKENSET)
+        reinterpret_cast<uint4*>(blkw)[w4] = reinterpret_cast<const uint4*>(wb)[w4];
+      __syncwarp(hm);  // before the next group reuses the buffer
+    } else {
+      put_codes<G, false>(blkw, side, tb, b, code);
     }
-    flush_word(blkw, acc);
-    flush_word(blkw, acc1);
-    // record of the token pair u = tau/2: index (u % 8) * (P/16) + u / 8
-    const int u = tau >> 1;
-    __half* rec = reinterpret_cast<__half*>(page + gd.sz_off + 8 * ((u & 7) * (P >> 4) + (u >> 3)));
-    rec[tau & 1] = s_h;
-    rec[2 + (tau & 1)] = z_h;
+    put_record(page + gd.sz_off, P, tau, s_h, z_h);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Fused small-batch encode (decode steps, T <= kFusedMaxT tokens): one CTA per
+// kept group projects the step's tokens onto the group's G columns (W_down rows
+// streamed once, H slices staged in shared memory), quantises and packs them,
+// all in one kernel; the positions are computed and validated by every CTA the
+// same way from the current lengths, so a failed check writes nothing anywhere.
+// A one-block commit kernel then advances the lengths.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Cache position of token t of an append (seq_ids non-decreasing), or an error.
+__device__ __forceinline__ int append_position(const int32_t* __restrict__ seq_ids, int t,
+                                               const spectra_cache& c, int P, int64_t* pos) {
+  const int s = seq_ids[t];
+  if (s < 0 || s >= c.batch || (t > 0 && seq_ids[t - 1] > s)) return SPECTRA_ERR_ORDER;
+  int first = t;
+  while (first > 0 && seq_ids[first - 1] == s) --first;
+  const int64_t p = (int64_t)c.lengths[s] + (t - first);
+  if (p < 0 || p >= (int64_t)c.max_pages_per_seq * P) return SPECTRA_ERR_CAPACITY;
+  const int pid = c.page_table[(size_t)s * c.max_pages_per_seq + p / P];
+  if (pid < 0 || (int64_t)pid >= c.n_pages) return SPECTRA_ERR_CAPACITY;
+  *pos = p;
+  return 0;
+}
+
+}  // namespace
+
+template <int G, int ROWS, int KC>
+__global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __restrict__ cd,
+                                                           const uint16_t* __restrict__ H, int T,
+                                                           const int32_t* __restrict__ seq_ids,
+                                                           const spectra_cache cache,
+                                                           float* __restrict__ latents_out) {
+  constexpr int CPW = G / 8;       // columns per warp (8 warps cover the group)
+  constexpr int BATCH = KC / 256;  // 16-byte chunks per column and lane per slice
+  __shared__ __align__(16) uint16_t h_s[ROWS * KC];
+  __shared__ float x_s[ROWS][G];
+  __shared__ int worst;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_launch_dependents();
+  // this CTA's group: kept groups numbered head-major, K side then V side
+  int a = 0, sd_i = 0, g = blockIdx.x;
+  for (; a < cd->n_kv; ++a) {
+    int side = 0;
+    for (; side < 2; ++side) {
+      const int n = cd->head[a].side[side].n_groups;
+      if (g < n) break;
+      g -= n;
+    }
+    if (side < 2) {
+      sd_i = side;
+      break;
+    }
+  }
+  const SideDev& sd = cd->head[a].side[sd_i];
+  const GroupDev gd = sd.grp[g];
+  const int d_model = cd->d_model;
+  const int n0 = sd.c_col0 + gd.col + warp * CPW;  // latent columns of this warp
+  const uint16_t* wt = cd->wt_down;
+  float acc[CPW][ROWS];
+#pragma unroll
+  for (int c = 0; c < CPW; ++c)
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) acc[c][r] = 0.f;
+  const int nr = min(ROWS, T);
+  for (int kc0 = 0; kc0 < d_model; kc0 += KC) {
+    uint4 wv[CPW][BATCH];
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i)
+#pragma unroll
+      for (int c = 0; c < CPW; ++c) {
+        const int k = kc0 + lane * 8 + 256 * i;
+        wv[c][i] = k < d_model ? __ldg(reinterpret_cast<const uint4*>(wt + (size_t)(n0 + c) * d_model + k))
+                               : make_uint4(0u, 0u, 0u, 0u);
+      }
+    pdl_wait();       // H, lengths and the page table may come from earlier kernels
+    __syncthreads();  // the previous slice's readers are done
+    for (int e = tid; e < ROWS * KC / 8; e += blockDim.x) {
+      const int r = e / (KC / 8), col = (e % (KC / 8)) * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < nr && kc0 + col < d_model)
+        v = __ldg(reinterpret_cast<const uint4*>(H + (size_t)r * d_model + kc0 + col));
+      *reinterpret_cast<uint4*>(h_s + r * KC + col) = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int kl = lane * 8 + 256 * i;
+      float w[CPW][8];
+#pragma unroll
+      for (int c = 0; c < CPW; ++c) bf16x8_to_f32(wv[c][i], w[c]);
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        if (r < nr) {
+          float h[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(h_s + r * KC + kl), h);
+#pragma unroll
+          for (int c = 0; c < CPW; ++c)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[c][r] = fmaf(w[c][e], h[e], acc[c][r]);
+        }
+      }
+    }
+  }
+  if (tid == 0) worst = 0;
+#pragma unroll
+  for (int c = 0; c < CPW; ++c)
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      float v = acc[c][r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && r < nr) x_s[r][warp * CPW + c] = v;
+    }
+  // positions of the step's tokens; every CTA reaches the same verdict
+  int64_t pos = 0;
+  int code_err = 0;
+  if (tid < T) code_err = append_position(seq_ids, tid, cache, cd->P, &pos);
+  __syncthreads();
+  if (code_err) atomicMax(&worst, code_err);
+  __syncthreads();
+  if (worst) {
+    if (blockIdx.x == 0 && tid == 0) device_error(cd->err, worst);
+    return;
+  }
+  if (tid < T) {
+    float x[G];
+#pragma unroll
+    for (int k = 0; k < G; ++k) x[k] = x_s[tid][k];
+    if (latents_out) {
+      float* lo = latents_out + (size_t)tid * cd->n_eff + sd.c_col0 + gd.col;
+#pragma unroll
+      for (int k = 0; k < G; ++k) lo[k] = x[k];
+    }
+    const int P = cd->P, TB = 256 / G;
+    const int seq = seq_ids[tid];
+    const int pid = cache.page_table[(size_t)seq * cache.max_pages_per_seq + pos / P];
+    uint8_t* page = static_cast<uint8_t*>(cache.pool) + (size_t)pid * (size_t)cd->page_bytes;
+    const int tau = (int)(pos % P);
+    const int b = gd.b;
+    __half s_h, z_h;
+    uint32_t code[G];
+    quantize_group<G>(x, b, s_h, z_h, code);
+    uint32_t* blkw = reinterpret_cast<uint32_t*>(page + gd.plane_off + (tau / TB) * (32 * b));
+    put_codes<G, false>(blkw, sd_i, tau % TB, b, code);
+    put_record(page + gd.sz_off, P, tau, s_h, z_h);
+  }
+}
+
+// Advances the lengths after a fused encode (same checks, so the same verdict).
+__global__ void __launch_bounds__(32) encode_commit_kernel(const int32_t* __restrict__ seq_ids, int T,
+                                                           const spectra_cache cache, int P) {
+  pdl_launch_dependents();
+  pdl_wait();  // the fused encode read the lengths before this point
+  const int t = threadIdx.x;
+  int64_t pos = 0;
+  const int err = t < T ? append_position(seq_ids, t, cache, P, &pos) : 0;
+  if (__any_sync(0xffffffffu, err != 0)) return;
+  if (t < T && (t == T - 1 || seq_ids[t + 1] != seq_ids[t])) cache.lengths[seq_ids[t]] = (int32_t)(pos + 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -369,6 +577,28 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
   return launch_dependent(quantize_append_kernel<8>, grid, dim3(128), 0, st, d, C, ldc, seq_ids, pos,
                           (const int32_t*)ok_flag, T, (uint8_t*)cache.pool, cache.page_table,
                           (int)cache.max_pages_per_seq);
+}
+
+cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
+                                int T, const spectra_cache& cache, float* latents_out, cudaStream_t st) {
+  int n_groups = 0;
+  for (int a = 0; a < h.n_kv; ++a) n_groups += h.head[a].side[0].n_groups + h.head[a].side[1].n_groups;
+  cudaError_t e = cudaSuccess;
+  if (n_groups > 0) {
+    const dim3 grid(n_groups), block(256);
+    if (h.group == 16)
+      e = T <= 1 ? launch_dependent(encode_fused_kernel<16, 1, 2048>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                                    latents_out)
+                 : launch_dependent(encode_fused_kernel<16, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T,
+                                    seq_ids, cache, latents_out);
+    else
+      e = T <= 1 ? launch_dependent(encode_fused_kernel<8, 1, 4096>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                                    latents_out)
+                 : launch_dependent(encode_fused_kernel<8, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T, seq_ids,
+                                    cache, latents_out);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_dependent(encode_commit_kernel, dim3(1), dim3(32), 0, st, seq_ids, T, cache, h.P);
 }
 
 }  // namespace spectra

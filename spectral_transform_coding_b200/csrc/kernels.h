@@ -41,6 +41,12 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
                                    const int32_t* seq_ids, const int32_t* pos, const int32_t* ok_flag,
                                    int T, const spectra_cache& cache, cudaStream_t st);
 
+// Fused encode for decode steps: projection, quantisation and packing in one
+// kernel per kept group, then a commit kernel that advances the lengths.
+constexpr int kFusedMaxT = 16;
+cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
+                                int T, const spectra_cache& cache, float* latents_out, cudaStream_t st);
+
 // decode_kernels.cu
 // Raises `kern`'s dynamic shared-memory limit on the current device to at least
 // `bytes` (one record per kernel and device; the limit never shrinks).

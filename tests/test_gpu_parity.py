@@ -290,3 +290,63 @@ def test_wo_correction_matches_oracle():
                                ref_codec, 2, 1, 16)
     err = np.abs(W_Op - ref["W_O"]).max() / np.abs(ref["W_O"]).max()
     assert err < 2e-2, err
+
+
+# --- fused encode of decode steps (T <= 16) ---------------------------------------
+
+@pytest.mark.parametrize("name,seqs", [("llama4x", [0]), ("llama4x", [0, 1, 1, 2]), ("qwen8x", [0] * 16),
+                                       ("g8wide", [0, 0, 1]), ("allwidths", [0, 1, 2, 3, 4])])
+def test_fused_encode_matches_oracle_latents_and_unfused_codes(name, seqs):
+    """Latents within 1e-3 of the oracle's H W_down; the packed pages equal what
+    the separately parity-tested quantiser writes for those same latents; lengths
+    advance by each sequence's token count."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup(name, seed=4)
+    codec, P = s["codec"], s["P"]
+    B = max(seqs) + 1
+    seqs = np.array(seqs, np.int32)
+    rng = np.random.default_rng(21)
+    H = bf16_round(rng.standard_normal((len(seqs), s["d_model"])).astype(np.float32))
+    table = np.arange(B * 3, dtype=np.int32).reshape(B, 3)
+    c1 = st.LatentCache(codec, batch=B, max_pages_per_seq=3, device=dev(), page_table=torch.from_numpy(table))
+    c2 = st.LatentCache(codec, batch=B, max_pages_per_seq=3, device=dev(), page_table=torch.from_numpy(table))
+    # start mid-block, at different lengths per sequence
+    start = np.array([5 + 7 * b for b in range(B)], np.int32)
+    c1.lengths.copy_(torch.from_numpy(start))
+    c2.lengths.copy_(torch.from_numpy(start))
+    lat = torch.empty((len(seqs), codec.n_eff), dtype=torch.float32, device=dev())
+    codec.encode_append(c1, torch.from_numpy(H).to(dev()).to(torch.bfloat16), torch.from_numpy(seqs).to(dev()),
+                        latents_out=lat)
+    codec.device_status()
+    _check_latents(lat.cpu().numpy(), H.astype(np.float64) @ s["W_down"].astype(np.float64), s)
+    codec.quantize_append(c2, lat, torch.from_numpy(seqs).to(dev()))
+    codec.device_status()
+    assert np.array_equal(c1.pool.cpu().numpy(), c2.pool.cpu().numpy())
+    want = start + np.bincount(seqs, minlength=B)
+    np.testing.assert_array_equal(c1.lengths.cpu().numpy(), want)
+
+
+def test_fused_encode_rejects_overflow_and_disorder_writing_nothing():
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup("llama4x", seed=5)
+    codec, P = s["codec"], s["P"]
+    cache = st.LatentCache(codec, batch=2, max_pages_per_seq=1, device=dev())
+    H = torch.from_numpy(bf16_round(np.ones((2, s["d_model"]), np.float32))).to(dev()).to(torch.bfloat16)
+    cache.lengths.copy_(torch.tensor([P - 1, 0], dtype=torch.int32))
+    before = cache.pool.clone()
+    # two tokens for sequence 0 with one free slot: capacity
+    codec.encode_append(cache, H, torch.tensor([0, 0], dtype=torch.int32, device=dev()))
+    with pytest.raises(st.SpectraError) as e:
+        codec.device_status()
+    assert e.value.status == 3
+    assert torch.equal(cache.pool, before)
+    assert cache.lengths.cpu().tolist() == [P - 1, 0]
+    # unsorted sequence ids: order
+    codec.encode_append(cache, H, torch.tensor([1, 0], dtype=torch.int32, device=dev()))
+    with pytest.raises(st.SpectraError) as e:
+        codec.device_status()
+    assert e.value.status == 7
+    assert torch.equal(cache.pool, before)
+    assert cache.lengths.cpu().tolist() == [P - 1, 0]
