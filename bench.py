@@ -51,7 +51,7 @@ def _workload_name(cfg, layers):
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same workload)
 # ---------------------------------------------------------------------------
-TRAFFIC_PER_ALGO_BYTE = {"llama": 33_888_768 / (32_772 * 1024)}
+TRAFFIC_PER_ALGO_BYTE = {"llama": 33_707_520 / (32_772 * 1024)}
 
 
 def _oracle_decode_case(cfg, n_tok=8192):
@@ -353,7 +353,7 @@ def run_gpu(args, rank, world):
 
     # roofline: packed bytes the decode reads per layer.  traffic: DRAM bytes
     # (read + write) of one split_kernel launch per algorithmic byte, from one ncu
-    # capture of the 1-layer Llama-shaped case at 32k context (33,888,768 B for
+    # capture of the 1-layer Llama-shaped case at 32k context (33,707,520 B for
     # 32,772 tokens x 1,024 B); only workloads with a capture of the current kernel
     # have one, else traffic is null.
     bytes_per_tok_all_heads = codecs[0].page_bytes / P

@@ -985,9 +985,10 @@ cudaError_t ensure_dynamic_smem(const void* kern, int bytes) {
 DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq) {
   DecodePlan p{};
   p.stage_bytes = std::max(16, ((h.max_sec_bytes + 15) / 16) * 16);
-  // up to 32 KB of stages per CTA: one stage per warp for the largest sections
-  // (so 4 CTAs fit an SM), up to 4 when sections are small
-  const int budget = 32 * 1024;
+  // up to 40 KB of stages per CTA: one stage per warp for 8 KB sections (four
+  // CTAs fit an SM), deeper per-warp pipelines when sections are small (measured
+  // best for 8, 4 and 2.5 KB sections: 1, 2 and 4 stages)
+  const int budget = 40 * 1024;
   p.stages = std::max(1, std::min(4, budget / (kDecWarps * p.stage_bytes)));
   p.smem_bytes = kSmStages + std::max(kDecWarps * p.stages * p.stage_bytes, kMergeBytes);
   // context splits: fill one wave of resident CTAs when that wastes < 15% of the
@@ -1003,7 +1004,9 @@ DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq)
   p.part_stride = ((2 + h.max_kept_v) + 3) / 4 * 4;
   const int ns_fit = (kMaxSmemPerBlock - combine_smem_bytes(h.max_kept_v, h.d_h, 0, 0)) / (p.part_stride * 4);
   ns = std::max(1, std::min({ns, kMaxSplit, ns_fit}));
-  (void)max_pages_per_seq;
+  // at least two pages per warp for a full-length sequence: fewer, longer
+  // splits amortise each CTA's fixed work
+  ns = std::max(1, std::min(ns, max_pages_per_seq / (kDecWarps * 2)));
   p.n_split = ns;
   size_t off = 0;
   auto carve = [&](size_t bytes) {
