@@ -361,7 +361,9 @@ def run_gpu(args, rank, world):
     dec_avg_ms = dec_ms
     peaks = _peaks()
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
-    launches_per_layer = 3 + 3  # encode: projection, append plan, quantise/pack; decode: fold, split, combine
+    # encode: fused projection/quantise/pack + commit for steps of <= 16 tokens,
+    # else projection + append plan + quantise/pack; decode: fold, split, combine
+    launches_per_layer = (2 if B <= 16 else 3) + 3
     h2d = H_new.numel() * 2 + Q.numel() * 4
     d2h = OUT.numel() * 4
 
