@@ -156,6 +156,27 @@ SPECTRA_API spectra_status spectra_calibrate(const spectra_config* cfg, int32_t 
                                  int64_t n_tokens, const void* W_K, const void* W_V,
                                  spectra_codec** out, void* stream);
 
+/* Width allocation of spectra_calibrate_ex. */
+typedef enum spectra_allocation {
+  SPECTRA_ALLOC_WATERFILL = 0, /* spectra_allocate_widths (stage 2 reverse water-filling, grouped) */
+  SPECTRA_ALLOC_UNIFORM = 1    /* spectra_allocate_widths_uniform (one width for all kept groups) */
+} spectra_allocation;
+
+/* spectra_calibrate_ex -- spectra_calibrate with a choice of allocation and an
+ * optional energy threshold on the rank.
+ *   allocation        SPECTRA_ALLOC_WATERFILL (what spectra_calibrate does) or
+ *                     SPECTRA_ALLOC_UNIFORM.
+ *   energy_threshold  0: every group may get bits; in (0, 1]: per head and side
+ *                     only the groups holding the leading spectra_energy_rank
+ *                     coordinates (rounded up to whole groups) may get bits
+ *                     ("Spectral-KV: SVD-projection KV cache compression
+ *                     (28x)", technical principle 1; e.g. 0.95).
+ * Otherwise as spectra_calibrate; SPECTRA_ERR_INVALID for other values. */
+SPECTRA_API spectra_status spectra_calibrate_ex(const spectra_config* cfg, int32_t dtype, const void* H,
+                                                int64_t n_tokens, const void* W_K, const void* W_V,
+                                                int32_t allocation, double energy_threshold,
+                                                spectra_codec** out, void* stream);
+
 /* spectra_codec_create -- build a codec from given factors (no calibration).
  *   widths   host [n_kv_heads][2][rank/group], each in {0,1,2,3,4,8}.
  *   W_down   host fp32 [d_model][n_eff]; columns head-major, K then V, kept
@@ -281,6 +302,18 @@ SPECTRA_API spectra_status spectra_decode_attend_noalloc(const spectra_codec* co
                                                          const spectra_cache* cache, const float* q,
                                                          float* out, void* stream);
 
+/* spectra_reconstruct -- rebuild the keys and values of cached tokens (stage 3:
+ * the dequantised latents lifted back with W_up for standard attention):
+ *   k^ = c^_K W_up^K, v^ = c^_V W_up^V, c^ = code * s + z (fp32), zero-width
+ *   groups contributing 0, for tokens [t0, t0 + n) of sequence `seq`.
+ *   K_out, V_out device fp32 [n][n_kv_heads][d_head], caller-owned.
+ * Any group count and width.  A range beyond lengths[seq] (known only on the
+ * device) or a page id outside [0, n_pages) records SPECTRA_ERR_INVALID in the
+ * device error word and leaves the outputs unspecified. */
+SPECTRA_API spectra_status spectra_reconstruct(const spectra_codec* codec, const spectra_cache* cache,
+                                               int32_t seq, int64_t t0, int64_t n, float* K_out, float* V_out,
+                                               void* stream);
+
 /* Synchronises `stream`, then reads and clears the codec's device error word.
  * Returns the recorded device-side status (SPECTRA_OK if none). */
 SPECTRA_API spectra_status spectra_device_status(const spectra_codec* codec, void* stream);
@@ -299,6 +332,25 @@ SPECTRA_API spectra_status spectra_device_status(const spectra_codec* codec, voi
 SPECTRA_API spectra_status spectra_allocate_widths(const double* sigma2, int32_t rank, int32_t group,
                                        int32_t budget_bits, int32_t count_overhead,
                                        int32_t* widths_out, double* distortion_out);
+
+/* Uniform allocation (SpectralQuant with uniform allocation, "Ablation,
+ * Statistical Inference, and Validation for KV-Cache Compression", practical
+ * recommendations): the leading k of the first n_eligible_groups groups all get
+ * one width b in {1,2,3,4,8}, the others 0; (k, b) minimises the model
+ * sum_j S_j 4^-b_j of spectra_allocate_widths under the same budget (ties: fewer
+ * bits, then fewer groups; k = 0 when nothing fits).  widths_out [rank/group];
+ * distortion_out may be NULL. */
+SPECTRA_API spectra_status spectra_allocate_widths_uniform(const double* sigma2, int32_t rank, int32_t group,
+                                                           int32_t n_eligible_groups, int32_t budget_bits,
+                                                           int32_t count_overhead, int32_t* widths_out,
+                                                           double* distortion_out);
+
+/* Effective rank: the smallest r with sigma2_0 + .. + sigma2_{r-1} >= threshold *
+ * (sigma2_0 + .. + sigma2_{n-1}), sigma2 in decreasing order, threshold in
+ * (0, 1] ("Spectral-KV: SVD-projection KV cache compression (28x)", technical
+ * principle 1, spectral profiling). */
+SPECTRA_API spectra_status spectra_energy_rank(const double* sigma2, int32_t n, double threshold,
+                                               int32_t* rank_out);
 
 /* Continuous reverse water-filling: theta with sum_i max(0, 1/2 log2(sigma2_i/theta))
  * = rate_bits; rates_out [n] (may be NULL). */

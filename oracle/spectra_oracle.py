@@ -34,6 +34,9 @@ Readings of points the pages leave open (each listed in the design doc):
   every cached token, GQA map q head h -> KV head h // (H_q/H_kv).
 * W_O correction: per q head least squares mapping the rank-truncated attention
   output onto the exact one on calibration data (the pages give no formula).
+* Alternatives for the allocation ablation: uniform widths (the leading k groups
+  at one width, (k, b) minimising the same model) and an energy-threshold rank
+  limiting which groups may get bits.
 
 Pinned by the ``-m "not gpu"`` tests in tests/test_oracle_*.py, except where a
 function's docstring says "parity unpinned".
@@ -223,6 +226,49 @@ def allocate_widths(sigma2: np.ndarray, g: int, budget: int, count_overhead: boo
     return widths
 
 
+def allocate_widths_uniform(sigma2: np.ndarray, g: int, budget: int, count_overhead: bool,
+                            n_eligible: int | None = None) -> np.ndarray:
+    """One width for every kept group ([ABL] "Practical recommendations":
+    SpectralQuant with uniform allocation).
+
+    Reading: the kept groups are the leading k of the first n_eligible groups,
+    all at one width b in {1,2,3,4,8}; among all (k, b) with k * cost(b) <= budget
+    choose the least model distortion sum_j S_j 4^-b_j (k = 0 keeps nothing); ties
+    go to fewer bits, then to fewer groups.  Enumerates every (k, b).
+    """
+    S = group_mass(sigma2, g)
+    n = S.size
+    ne = n if n_eligible is None else max(0, min(int(n_eligible), n))
+    best = (float(sum(S)), 0, 0, 0)  # (distortion, bits, k, b)
+    for b in WIDTHS[1:]:
+        cost = group_cost(b, g, count_overhead)
+        for k in range(1, ne + 1):
+            if k * cost > budget:
+                break
+            w = [b] * k + [0] * (n - k)
+            cand = (allocation_distortion(sigma2, w, g), k * cost, k, b)
+            if cand[:3] < best[:3]:
+                best = cand
+    _, _, k, b = best
+    return np.array([b] * k + [0] * (n - k), dtype=np.int64)
+
+
+def energy_rank(sigma2: np.ndarray, threshold: float) -> int:
+    """Smallest r with sum_{i<r} sigma2_i >= threshold * sum_i sigma2_i ([SKV]
+    "Technical principle" 1: the effective rank at a target energy, e.g. 0.95);
+    sigma2 in decreasing order, threshold in (0, 1]."""
+    s2 = np.asarray(sigma2, dtype=np.float64)
+    if not 0.0 < threshold <= 1.0:
+        raise ValueError("threshold must be in (0, 1]")
+    total = float(s2.sum())
+    acc = 0.0
+    for i, v in enumerate(s2):
+        acc += float(v)
+        if acc >= threshold * total:
+            return i + 1
+    return s2.size
+
+
 def allocation_distortion(sigma2, widths, g) -> float:
     S = group_mass(sigma2, g)
     return float(sum(group_distortion(S[j], int(b)) for j, b in enumerate(widths)))
@@ -238,7 +284,8 @@ def nonzero_coords(widths: np.ndarray, g: int) -> np.ndarray:
                           ) if np.any(np.asarray(widths) > 0) else np.zeros(0, dtype=np.int64)
 
 
-def calibrate(cfg, H: np.ndarray, W_K: np.ndarray, W_V: np.ndarray, literal: bool = False) -> dict:
+def calibrate(cfg, H: np.ndarray, W_K: np.ndarray, W_V: np.ndarray, literal: bool = False,
+              allocation: str = "waterfill", energy_threshold: float = 0.0) -> dict:
     """Gram -> per (head, side) basis, sigma^2, widths, theta -> W_down / W_up.
 
     ``cfg`` needs d_model, n_kv_heads, d_head, rank, group, budget_bits,
@@ -255,7 +302,19 @@ def calibrate(cfg, H: np.ndarray, W_K: np.ndarray, W_V: np.ndarray, literal: boo
             Wa = np.asarray(W, dtype=np.float64)[:, a * cfg.d_head:(a + 1) * cfg.d_head]
             basis = whitened_svd(G, Wa, cfg.rank) if literal else latent_basis(G, Wa, cfg.rank)
             s2 = basis["sigma2"][: cfg.rank]
-            widths = allocate_widths(s2, cfg.group, cfg.budget_bits, cfg.count_overhead)
+            n_grp = cfg.rank // cfg.group
+            n_elig = n_grp
+            if energy_threshold > 0.0:
+                re = energy_rank(basis["sigma2"], energy_threshold)  # over all d_head coordinates
+                n_elig = min(n_grp, -(-re // cfg.group))
+            if allocation == "uniform":
+                widths = allocate_widths_uniform(s2, cfg.group, cfg.budget_bits, cfg.count_overhead, n_elig)
+            elif allocation == "waterfill":
+                widths = np.zeros(n_grp, dtype=np.int64)
+                widths[:n_elig] = allocate_widths(s2[: n_elig * cfg.group], cfg.group, cfg.budget_bits,
+                                                  cfg.count_overhead)
+            else:
+                raise ValueError("allocation must be 'waterfill' or 'uniform'")
             payload = int(sum(cfg.group * int(b) for b in widths))
             wf = reverse_water_fill(s2, payload)
             keep = nonzero_coords(widths, cfg.group)

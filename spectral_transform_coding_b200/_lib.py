@@ -15,6 +15,7 @@ if not os.path.exists(lib_path):
 lib = ctypes.CDLL(lib_path)
 
 SPECTRA_F32, SPECTRA_BF16 = 0, 1
+SPECTRA_ALLOC_WATERFILL, SPECTRA_ALLOC_UNIFORM = 0, 1
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID", 2: "ERR_CUDA", 3: "ERR_CAPACITY", 4: "ERR_NUMERIC",
                 5: "ERR_UNSUPPORTED", 6: "ERR_TIMEOUT", 7: "ERR_ORDER"}
 
@@ -50,6 +51,7 @@ _P = ctypes.POINTER
 
 _SIGS = {
     "spectra_calibrate": [_P(Config), _i32, _vp, _i64, _vp, _vp, _P(_vp), _vp],
+    "spectra_calibrate_ex": [_P(Config), _i32, _vp, _i64, _vp, _vp, _i32, ctypes.c_double, _P(_vp), _vp],
     "spectra_codec_create": [_P(Config), _vp, _vp, _vp, _vp, _P(_vp)],
     "spectra_codec_get_info": [_vp, _P(CodecInfo)],
     "spectra_codec_get_state": [_vp, _vp, _vp, _vp, _vp, _vp],
@@ -64,7 +66,10 @@ _SIGS = {
     "spectra_decode_attend": [_vp, _P(CacheDesc), _vp, _vp, _vp, _sz, _vp],
     "spectra_decode_attend_noalloc": [_vp, _P(CacheDesc), _vp, _vp, _vp],
     "spectra_device_status": [_vp, _vp],
+    "spectra_reconstruct": [_vp, _P(CacheDesc), _i32, _i64, _i64, _vp, _vp, _vp],
     "spectra_allocate_widths": [_vp, _i32, _i32, _i32, _i32, _vp, _vp],
+    "spectra_allocate_widths_uniform": [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp],
+    "spectra_energy_rank": [_vp, _i32, ctypes.c_double, _P(_i32)],
     "spectra_water_fill": [_vp, _i32, ctypes.c_double, _vp, _vp],
     "spectra_sym_eigen": [_vp, _i32, _vp, _vp],
     "spectra_page_layout": [_P(Config), _vp, _P(_i64), _vp],

@@ -55,13 +55,19 @@ class Codec:
 
     # -- construction ------------------------------------------------------
     @classmethod
-    def calibrate(cls, cfg: Config, H, W_K, W_V, stream=None) -> "Codec":
+    def calibrate(cls, cfg: Config, H, W_K, W_V, stream=None, allocation: str = "waterfill",
+                  energy_threshold: float = 0.0) -> "Codec":
+        """allocation: "waterfill" or "uniform"; energy_threshold: 0 (off) or in (0, 1]."""
         dt = _dtype_code(H)
         if _dtype_code(W_K) != dt or _dtype_code(W_V) != dt:
             raise TypeError("H, W_K, W_V must share one dtype")
+        modes = {"waterfill": 0, "uniform": 1}
+        if allocation not in modes:
+            raise ValueError("allocation must be 'waterfill' or 'uniform'")
         h = ctypes.c_void_p()
-        check(lib.spectra_calibrate(ctypes.byref(cfg), dt, _ptr(H), H.shape[0], _ptr(W_K), _ptr(W_V),
-                                    ctypes.byref(h), _stream(stream)), "spectra_calibrate")
+        check(lib.spectra_calibrate_ex(ctypes.byref(cfg), dt, _ptr(H), H.shape[0], _ptr(W_K), _ptr(W_V),
+                                       modes[allocation], float(energy_threshold), ctypes.byref(h),
+                                       _stream(stream)), "spectra_calibrate_ex")
         return cls(h)
 
     @classmethod
@@ -163,6 +169,17 @@ class Codec:
         check(lib.spectra_decode_attend(self._h, ctypes.byref(d), _ptr(q), _ptr(out), _ptr(ws), ws.numel(),
                                         _stream(stream)), "spectra_decode_attend")
         return out
+
+    def reconstruct(self, cache: "LatentCache", seq: int, t0: int, n: int, stream=None):
+        """Keys and values [n][n_kv][d_head] (fp32) of tokens [t0, t0+n) of sequence seq."""
+        torch = _torch()
+        c = self.cfg
+        K = torch.empty((n, c.n_kv_heads, c.d_head), dtype=torch.float32, device=cache.pool.device)
+        V = torch.empty_like(K)
+        d = cache.desc()
+        check(lib.spectra_reconstruct(self._h, ctypes.byref(d), int(seq), int(t0), int(n), _ptr(K), _ptr(V),
+                                      _stream(stream)), "spectra_reconstruct")
+        return K, V
 
     def device_status(self, stream=None):
         check(lib.spectra_device_status(self._h, _stream(stream)), "spectra_device_status")

@@ -326,7 +326,17 @@ spectra_status spectra_codec_deserialize(const void* buf, size_t bytes, spectra_
 spectra_status spectra_calibrate(const spectra_config* cfg, int32_t dtype, const void* H,
                                  int64_t n_tokens, const void* W_K, const void* W_V,
                                  spectra_codec** out, void* stream) {
+  return spectra_calibrate_ex(cfg, dtype, H, n_tokens, W_K, W_V, SPECTRA_ALLOC_WATERFILL, 0.0, out, stream);
+}
+
+spectra_status spectra_calibrate_ex(const spectra_config* cfg, int32_t dtype, const void* H,
+                                    int64_t n_tokens, const void* W_K, const void* W_V, int32_t allocation,
+                                    double energy_threshold, spectra_codec** out, void* stream) {
   if (!cfg || !H || !W_K || !W_V || !out) return fail(SPECTRA_ERR_INVALID, "null pointer");
+  if (allocation != SPECTRA_ALLOC_WATERFILL && allocation != SPECTRA_ALLOC_UNIFORM)
+    return fail(SPECTRA_ERR_INVALID, "unknown allocation");
+  if (!(energy_threshold >= 0.0) || energy_threshold > 1.0)
+    return fail(SPECTRA_ERR_INVALID, "energy_threshold must be 0 (off) or in (0, 1]");
   *out = nullptr;
   std::string why;
   if (!valid_config(*cfg, &why)) return fail(SPECTRA_ERR_INVALID, why);
@@ -400,8 +410,20 @@ spectra_status spectra_calibrate(const spectra_config* cfg, int32_t dtype, const
         if (vals[i] < 0) vals[i] = 0;
       }
       std::copy(vals.begin(), vals.begin() + r, sigma2.begin() + hs * r);
-      allocate_widths(vals.data(), r, g, cfg->budget_bits, cfg->count_overhead != 0,
-                      widths.data() + hs * ng, nullptr);
+      // groups eligible for bits: all, or those holding the leading coordinates
+      // up to the energy rank (rounded up to whole groups)
+      int n_elig = ng;
+      if (energy_threshold > 0.0) {
+        int re = dh;
+        energy_rank(vals.data(), dh, energy_threshold, &re);
+        n_elig = std::min(ng, (re + g - 1) / g);
+      }
+      int32_t* wj = widths.data() + hs * ng;
+      std::fill(wj, wj + ng, 0);
+      if (allocation == SPECTRA_ALLOC_UNIFORM)
+        allocate_widths_uniform(vals.data(), r, g, n_elig, cfg->budget_bits, cfg->count_overhead != 0, wj, nullptr);
+      else
+        allocate_widths(vals.data(), n_elig * g, g, cfg->budget_bits, cfg->count_overhead != 0, wj, nullptr);
       int payload = 0;
       for (int j = 0; j < ng; ++j) payload += g * widths[hs * ng + j];
       water_fill(vals.data(), r, (double)payload, &theta[hs], nullptr);
@@ -627,6 +649,20 @@ spectra_status spectra_decode_attend(const spectra_codec* c, const spectra_cache
   const DecodePlan plan = make_decode_plan(c->h, cache->batch, cache->max_pages_per_seq);
   if (workspace_bytes < plan.ws_bytes) return fail(SPECTRA_ERR_INVALID, "workspace too small");
   CUDA_TRY(launch_decode(c->h, c->d, *cache, q, out, workspace, plan, static_cast<cudaStream_t>(stream)));
+  return SPECTRA_OK;
+}
+
+spectra_status spectra_reconstruct(const spectra_codec* c, const spectra_cache* cache, int32_t seq, int64_t t0,
+                                   int64_t n, float* K_out, float* V_out, void* stream) {
+  if (!c || !K_out || !V_out) return fail(SPECTRA_ERR_INVALID, "null pointer");
+  spectra_status s = check_cache(c, cache);
+  if (s != SPECTRA_OK) return s;
+  if (seq < 0 || seq >= cache->batch) return fail(SPECTRA_ERR_INVALID, "seq out of range");
+  if (t0 < 0 || n < 0 || n > ((int64_t)1 << 26)) return fail(SPECTRA_ERR_INVALID, "token range out of range");
+  if (!aligned(K_out, 4) || !aligned(V_out, 4)) return fail(SPECTRA_ERR_INVALID, "misaligned buffer");
+  s = check_device(c);
+  if (s != SPECTRA_OK) return s;
+  CUDA_TRY(launch_reconstruct(c->h, c->d, *cache, seq, t0, n, K_out, V_out, static_cast<cudaStream_t>(stream)));
   return SPECTRA_OK;
 }
 

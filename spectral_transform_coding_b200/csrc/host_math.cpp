@@ -79,6 +79,70 @@ int allocate_widths(const double* sigma2, int rank, int group, int budget, bool 
   return 0;
 }
 
+// Uniform allocation ("SpectralQuant with uniform allocation" of "Ablation,
+// Statistical Inference, and Validation for KV-Cache Compression", practical
+// recommendations): every kept group gets the same width b and the kept groups
+// are the leading k of the first n_eligible; (k, b) minimises the same model
+// sum_j S_j 4^-b_j under the budget (ties: fewer bits, then fewer groups).
+int allocate_widths_uniform(const double* sigma2, int rank, int group, int n_eligible, int budget,
+                            bool overhead, int32_t* widths, double* distortion) {
+  if (group <= 0 || rank % group != 0 || budget < 0) return 1;
+  const int n = rank / group;
+  n_eligible = std::max(0, std::min(n_eligible, n));
+  std::vector<double> S(n, 0.0);
+  double total = 0.0;
+  for (int j = 0; j < n; ++j) {
+    double acc = 0.0;
+    for (int i = j * group; i < (j + 1) * group; ++i) acc += sigma2[i];
+    S[j] = acc;
+  }
+  for (int j = n - 1; j >= 0; --j) total = S[j] + total;
+  double best = total;
+  int best_k = 0, best_b = 0, best_bits = 0;
+  for (int wi = 1; wi < 6; ++wi) {
+    const int b = kWidths[wi];
+    const int cost = group_cost(b, group, overhead);
+    double kept = 0.0;  // sum_{j<k} S_j
+    for (int k = 1; k <= n_eligible; ++k) {
+      if ((int64_t)k * cost > budget) break;
+      kept += S[k - 1];
+      double rest = 0.0;
+      for (int j = n - 1; j >= k; --j) rest = S[j] + rest;
+      const double d = kept * std::ldexp(1.0, -2 * b) + rest;
+      const int bits = k * cost;
+      if (d < best || (d == best && bits < best_bits)) {
+        best = d;
+        best_k = k;
+        best_b = b;
+        best_bits = bits;
+      }
+    }
+  }
+  for (int j = 0; j < n; ++j) widths[j] = j < best_k ? best_b : 0;
+  if (distortion) *distortion = best;
+  return 0;
+}
+
+// Effective rank ("Spectral-KV: SVD-projection KV cache compression (28x)",
+// technical principle 1, spectral profiling): the smallest r with
+// sum_{i<r} sigma2_i >= threshold * sum_i sigma2_i (sigma2 descending).
+int energy_rank(const double* sigma2, int n, double threshold, int* r) {
+  if (n <= 0 || !(threshold > 0.0) || threshold > 1.0) return 1;
+  double total = 0.0;
+  for (int i = 0; i < n; ++i) total += sigma2[i];
+  double acc = 0.0;
+  int k = n;
+  for (int i = 0; i < n; ++i) {
+    acc += sigma2[i];
+    if (acc >= threshold * total) {
+      k = i + 1;
+      break;
+    }
+  }
+  *r = k;
+  return 0;
+}
+
 // Reverse water-filling in closed form: with the k largest second moments
 // active, log theta = (sum_{i<k} log s_i - 2 R ln 2) / k; the right k is the one
 // whose theta lies in [s_(k+1), s_k).
@@ -329,6 +393,32 @@ spectra_status spectra_allocate_widths(const double* sigma2, int32_t rank, int32
     if (!std::isfinite(sigma2[i]) || sigma2[i] < 0) return fail(SPECTRA_ERR_NUMERIC, "sigma2 must be finite and >= 0");
   if (allocate_widths(sigma2, rank, group, budget_bits, count_overhead != 0, widths_out, distortion_out))
     return fail(SPECTRA_ERR_INVALID, "allocation failed");
+  return SPECTRA_OK;
+}
+
+spectra_status spectra_allocate_widths_uniform(const double* sigma2, int32_t rank, int32_t group,
+                                               int32_t n_eligible_groups, int32_t budget_bits,
+                                               int32_t count_overhead, int32_t* widths_out,
+                                               double* distortion_out) {
+  if (!sigma2 || !widths_out) return fail(SPECTRA_ERR_INVALID, "null pointer");
+  if (group <= 0 || rank <= 0 || rank % group || budget_bits < 0 || budget_bits > (1 << 20))
+    return fail(SPECTRA_ERR_INVALID, "bad rank/group/budget");
+  for (int i = 0; i < rank; ++i)
+    if (!std::isfinite(sigma2[i]) || sigma2[i] < 0) return fail(SPECTRA_ERR_NUMERIC, "sigma2 must be finite and >= 0");
+  if (allocate_widths_uniform(sigma2, rank, group, n_eligible_groups, budget_bits, count_overhead != 0,
+                              widths_out, distortion_out))
+    return fail(SPECTRA_ERR_INVALID, "allocation failed");
+  return SPECTRA_OK;
+}
+
+spectra_status spectra_energy_rank(const double* sigma2, int32_t n, double threshold, int32_t* rank_out) {
+  if (!sigma2 || !rank_out || n <= 0) return fail(SPECTRA_ERR_INVALID, "bad arguments");
+  if (!(threshold > 0.0) || threshold > 1.0) return fail(SPECTRA_ERR_INVALID, "threshold must be in (0, 1]");
+  for (int i = 0; i < n; ++i)
+    if (!std::isfinite(sigma2[i]) || sigma2[i] < 0) return fail(SPECTRA_ERR_NUMERIC, "sigma2 must be finite and >= 0");
+  int r = n;
+  energy_rank(sigma2, n, threshold, &r);
+  *rank_out = r;
   return SPECTRA_OK;
 }
 

@@ -47,6 +47,11 @@ constexpr int kFusedMaxT = 16;
 cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
                                 int T, const spectra_cache& cache, float* latents_out, cudaStream_t st);
 
+// reconstruct_kernels.cu: k^ = (code s + z) W_up^K, v^ likewise, for tokens
+// [t0, t0 + n) of sequence b; out of range or bad page ids -> device error INVALID
+cudaError_t launch_reconstruct(const CodecDev& h, const CodecDev* d, const spectra_cache& cache, int b, int64_t t0,
+                               int64_t n, float* K_out, float* V_out, cudaStream_t st);
+
 // decode_kernels.cu
 // Raises `kern`'s dynamic shared-memory limit on the current device to at least
 // `bytes` (one record per kernel and device; the limit never shrinks).

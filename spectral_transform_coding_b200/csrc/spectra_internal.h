@@ -66,6 +66,9 @@ struct CodecDev {
 // ---- host math (host_math.cpp), no CUDA needed ------------------------------
 int allocate_widths(const double* sigma2, int rank, int group, int budget, bool overhead,
                     int32_t* widths, double* distortion);
+int allocate_widths_uniform(const double* sigma2, int rank, int group, int n_eligible, int budget,
+                            bool overhead, int32_t* widths, double* distortion);
+int energy_rank(const double* sigma2, int n, double threshold, int* r);
 int water_fill(const double* sigma2, int n, double rate, double* theta, double* rates);
 int sym_eigen(const double* M, int n, double* vals, double* vecs);
 // Fills the layout part of `cd` (head sections, group offsets, n_eff ...).

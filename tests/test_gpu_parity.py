@@ -350,3 +350,76 @@ def test_fused_encode_rejects_overflow_and_disorder_writing_nothing():
     assert e.value.status == 7
     assert torch.equal(cache.pool, before)
     assert cache.lengths.cpu().tolist() == [P - 1, 0]
+
+
+# --- reconstruction of keys and values --------------------------------------------
+
+@pytest.mark.parametrize("name", ["llama4x", "allwidths", "g8wide", "zeroside"])
+def test_reconstruct_matches_oracle(name):
+    """k^, v^ of a token range rebuilt on the GPU from the packed pages equal the
+    oracle's dequantise-and-lift over its own pool (same seeded latents)."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup(name, seed=6)
+    codec, P = s["codec"], s["P"]
+    lengths = [150, 61]
+    B, maxp = 2, -(-max(lengths) // P)
+    rng = np.random.default_rng(8)
+    perm = rng.permutation(B * maxp).astype(np.int32).reshape(B, maxp)
+    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=maxp, device=dev(), page_table=torch.from_numpy(perm))
+    seqs = np.concatenate([np.full(L, b, np.int32) for b, L in enumerate(lengths)])
+    lat = synthetic_latents(seqs.size, codec.n_eff, seed=31, decay=0.5, scale=2.0)
+    codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+    pool_ref, _, lay = oracle_pool_after({"group": s["group"]}, s["widths"], cache.pool.numel(), codec.page_bytes,
+                                         perm, np.zeros(B), seqs, lat, P)
+    W_up = kept_wup(s["W_up"], s["widths"], s["group"])
+    for b, (t0, n) in ((0, (3, 140)), (1, (0, 61)), (0, (149, 1))):
+        K, V = codec.reconstruct(cache, b, t0, n)
+        codec.device_status()
+        for a in range(s["n_kv"]):
+            for side, got in ((0, K), (1, V)):
+                c = oracle.read_side(pool_ref, codec.page_bytes, lay, s["group"], P, perm[b], lengths[b], a, side)
+                ref = c[t0:t0 + n] @ np.asarray(W_up[a][side], np.float64)
+                g = got[:, a].cpu().numpy().astype(np.float64)
+                scale = np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+                if W_up[a][side].shape[0] == 0:
+                    assert np.all(g == 0)
+                else:
+                    assert (np.linalg.norm(g - ref, axis=1) / scale).max() <= 1e-5
+
+
+def test_reconstruct_rejects_range_past_length():
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup("llama4x", seed=6)
+    codec = s["codec"]
+    cache = st.LatentCache(codec, batch=1, max_pages_per_seq=2, device=dev())
+    lat = synthetic_latents(10, codec.n_eff, seed=2)
+    codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.zeros(10, dtype=torch.int32, device=dev()))
+    codec.reconstruct(cache, 0, 5, 6)
+    with pytest.raises(st.SpectraError) as e:
+        codec.device_status()
+    assert e.value.status == 1
+    with pytest.raises(st.SpectraError):
+        codec.reconstruct(cache, 1, 0, 1)  # sequence out of range: host check
+
+
+# --- calibration options (allocation ablation) ---------------------------------------
+
+@pytest.mark.parametrize("allocation,thr", [("uniform", 0.0), ("waterfill", 0.9), ("uniform", 0.8)])
+def test_calibrate_options_match_oracle(allocation, thr):
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    cfgw = get_config("toy")
+    layer = make_layer(cfgw)
+    cfg = make_cfg(cfgw.d_model, cfgw.n_q_heads, cfgw.n_kv_heads, cfgw.d_head, cfgw.rank, cfgw.group,
+                   cfgw.budget_bits, cfgw.count_overhead, cfgw.page_tokens)
+    t = lambda x: torch.from_numpy(x).to(dev())
+    codec = st.Codec.calibrate(cfg, t(layer["H_calib"]), t(layer["W_K"]), t(layer["W_V"]), allocation=allocation,
+                               energy_threshold=thr)
+    state = codec.state()
+    ref = oracle.calibrate(cfgw, layer["H_calib"], layer["W_K"], layer["W_V"], allocation=allocation,
+                           energy_threshold=thr)
+    for sidx, side in enumerate("KV"):
+        np.testing.assert_array_equal(state["widths"][0, sidx], ref["heads"][0][side]["widths"])
+        np.testing.assert_allclose(state["sigma2"][0, sidx], ref["heads"][0][side]["sigma2"], rtol=1e-4, atol=1e-7)

@@ -119,3 +119,29 @@ def test_invalid_config_rejected(st):
     assert st.lib.spectra_page_layout(ctypes.byref(bad), w.ctypes.data, ctypes.byref(pb), None) == 1
     bad = make_config(256, 4, 1, 64, 32, 8, 64, False, 48)  # page_tokens not multiple of 32
     assert st.lib.spectra_page_layout(ctypes.byref(bad), w.ctypes.data, ctypes.byref(pb), None) == 1
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_uniform_widths_match_oracle(seed):
+    from spectral_transform_coding_b200._lib import lib
+    rng = np.random.default_rng(100 + seed)
+    s2 = np.ascontiguousarray(np.sort(rng.gamma(0.7, size=128))[::-1])
+    for budget, ov, ne in ((512, 1, 8), (256, 1, 8), (256, 1, 3), (170, 1, 8), (64, 0, 8)):
+        w = np.zeros(8, np.int32)
+        d = ctypes.c_double(0)
+        assert lib.spectra_allocate_widths_uniform(s2.ctypes.data, 128, 16, ne, budget, ov, w.ctypes.data,
+                                                   ctypes.byref(d)) == 0
+        ref = oracle.allocate_widths_uniform(s2, 16, budget, bool(ov), ne)
+        np.testing.assert_array_equal(w, ref)
+        assert abs(d.value - oracle.allocation_distortion(s2, ref, 16)) <= 1e-12 * max(1.0, d.value)
+
+
+def test_energy_rank_matches_oracle():
+    from spectral_transform_coding_b200._lib import lib
+    rng = np.random.default_rng(7)
+    s2 = np.ascontiguousarray(np.sort(rng.exponential(size=128))[::-1])
+    for thr in (0.5, 0.9, 0.95, 0.99, 1.0):
+        r = ctypes.c_int32(0)
+        assert lib.spectra_energy_rank(s2.ctypes.data, 128, thr, ctypes.byref(r)) == 0
+        assert r.value == oracle.energy_rank(s2, thr)
+    assert lib.spectra_energy_rank(s2.ctypes.data, 128, 0.0, ctypes.byref(r)) != 0

@@ -127,3 +127,61 @@ def test_more_energy_more_bits():
         for budget in (170, 256, 512):
             w = oracle.allocate_widths(s2, 16, budget, True)
             assert list(w) == sorted(w, reverse=True)
+
+
+# --- uniform allocation and the energy rank (allocation ablation) -------------------
+
+def test_uniform_allocation_worked_by_hand():
+    """Groups of 2, no overhead, budget 8 bits (cost of a group = 2 b).
+    sigma2 = [4,4,1,1,.25,.25,0,0]: S = [8,2,.5,0].  Candidates (k, b) -> model
+    distortion: b=1: k=3 or 4 -> 10.5/4 = 2.625; b=2: k=2 -> 10/16 + .5 = 1.125,
+    k=1 -> 3.0; b=3: k=1 -> 8/64 + 2.5 = 2.625; b=4: k=1 -> 2.53125.  Best (2, 2).
+    sigma2 = [8,8,.5 x 6]: S = [16,1,1,1].  b=2, k=2 -> 17/16 + 2 = 3.0625 and
+    b=4, k=1 -> 1/16 + 3 = 3.0625 with 8 bits each: fewer groups wins -> (1, 4);
+    the grouped water-filling optimum is 2.5 (e.g. [3,1,0,0])."""
+    s2 = np.array([4, 4, 1, 1, .25, .25, 0, 0.])
+    w = oracle.allocate_widths_uniform(s2, 2, 8, False)
+    assert list(w) == [2, 2, 0, 0]
+    assert oracle.allocation_distortion(s2, w, 2) == 1.125
+    s2 = np.array([8, 8] + [.5] * 6)
+    w = oracle.allocate_widths_uniform(s2, 2, 8, False)
+    assert list(w) == [4, 0, 0, 0]
+    assert oracle.allocation_distortion(s2, w, 2) == 3.0625
+    assert oracle.allocation_distortion(s2, oracle.allocate_widths(s2, 2, 8, False), 2) == 2.5
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_uniform_never_beats_grouped_water_filling(seed):
+    """The grouped optimum is taken over a superset of the uniform choices."""
+    rng = np.random.default_rng(seed)
+    s2 = np.sort(rng.gamma(0.5, size=64))[::-1]
+    for budget, ov in ((128, True), (256, True), (96, False)):
+        wu = oracle.allocate_widths_uniform(s2, 8, budget, ov)
+        wd = oracle.allocate_widths(s2, 8, budget, ov)
+        assert sum(oracle.group_cost(int(b), 8, ov) for b in wu) <= budget
+        assert len(set(int(b) for b in wu if b > 0)) <= 1
+        assert oracle.allocation_distortion(s2, wd, 8) <= oracle.allocation_distortion(s2, wu, 8) + 1e-15
+
+
+def test_uniform_respects_eligible_groups():
+    s2 = np.linspace(4, 1, 32)
+    w = oracle.allocate_widths_uniform(s2, 8, 1000, True, n_eligible=2)
+    assert list(w[2:]) == [0, 0] and w[0] == w[1] == 8
+
+
+def test_energy_rank_worked_by_hand():
+    """sigma2 = [4,3,2,1] (total 10): cumulative 4, 7, 9, 10 -> threshold .7 reached
+    at r = 2, .71 at r = 3, 1.0 at r = 4; [5,0,0] holds all energy at r = 1."""
+    assert oracle.energy_rank([4, 3, 2, 1], 0.7) == 2
+    assert oracle.energy_rank([4, 3, 2, 1], 0.71) == 3
+    assert oracle.energy_rank([4, 3, 2, 1], 1.0) == 4
+    assert oracle.energy_rank([4, 3, 2, 1], 0.1) == 1
+    assert oracle.energy_rank([5, 0, 0], 1.0) == 1
+    with pytest.raises(ValueError):
+        oracle.energy_rank([1, 1], 0.0)
+
+
+def test_energy_rank_monotone_in_threshold():
+    s2 = np.sort(np.random.default_rng(3).exponential(size=128))[::-1]
+    ranks = [oracle.energy_rank(s2, t) for t in np.linspace(0.05, 1.0, 20)]
+    assert ranks == sorted(ranks) and ranks[-1] <= 128
