@@ -42,6 +42,22 @@ def _peaks():
     return dict(FALLBACK_PEAKS, src="fallback")
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings over the process group (the job
+    takes as long as its slowest rank); NCCL needs device tensors, gloo host ones."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def replicas_throughput(units_per_step_per_rank, ms_per_step_max, world):
+    """Whole-job throughput of `world` independent replicas (weak scaling): the
+    units all ranks processed per step over the slowest rank's step time."""
+    return units_per_step_per_rank * world / (ms_per_step_max / 1e3)
+
+
 def _workload_name(cfg, layers):
     return (f"{cfg.name}: {layers} layers x (d_model {cfg.d_model}, {cfg.n_q_heads}q/{cfg.n_kv_heads}kv heads, "
             f"d_head {cfg.d_head}, groups of {cfg.group}, {cfg.budget_bits} bits/side), "
@@ -342,14 +358,11 @@ def run_gpu(args, rank, world):
         codec.device_status(stream)
     ms_per_step = total_ms / steps
     if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_per_step, e2e_ms, dec_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step, e2e_ms, dec_ms = float(t[0]), float(t[1]), float(t[2])
+        ms_per_step, e2e_ms, dec_ms = max_over_ranks([ms_per_step, e2e_ms, dec_ms], dev)
     mean_ctx = (len0 + len_after) / 2.0
     tok_per_step = L * B * mean_ctx * cfg.n_kv_heads
-    value = tok_per_step / (ms_per_step / 1e3) * world
-    e2e_value = tok_per_step / (e2e_ms / 1e3) * world
+    value = replicas_throughput(tok_per_step, ms_per_step, world)
+    e2e_value = replicas_throughput(tok_per_step, e2e_ms, world)
 
     # roofline: packed bytes the decode reads per layer.  traffic: DRAM bytes
     # (read + write) of one split_kernel launch per algorithmic byte, from one ncu
