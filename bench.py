@@ -6,7 +6,7 @@ quantise + pack + append) followed by spectra_decode_attend over the whole
 latent cache.  Caches and codec factors of all layers (> L2) are resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama|qwen|stress]
-                    [--impl ours|reference]
+                    [--impl ours|reference] [--decode latent|reconstruct] [--rope-theta T]
 
 Prints one JSON line (rank 0).  Metric: cache tokens/s/head = sum over layers of
 batch * context * n_kv_heads per second of step time.  ``roofline`` reports the
@@ -70,9 +70,11 @@ def _workload_name(cfg, layers):
 TRAFFIC_PER_ALGO_BYTE = {"llama": 33_707_520 / (32_772 * 1024)}
 
 
-def _oracle_decode_case(cfg, n_tok=8192):
+def _oracle_decode_case(cfg, n_tok=8192, rope_theta=None):
     """One KV head of the workload's layer for the CPU oracle: widths from the
-    workload's spectrum, a packed pool of ``n_tok`` seeded tokens, W_up, queries."""
+    workload's spectrum, a packed pool of ``n_tok`` seeded tokens, W_up, queries.
+    rope_theta None: the latent decode's reference; else reconstruct-then-attend
+    with that rotary base."""
     import numpy as np
 
     import oracle
@@ -94,8 +96,12 @@ def _oracle_decode_case(cfg, n_tok=8192):
     qs = rng.standard_normal((1, cfg.gq, cfg.d_head)).astype(np.float32)
 
     def run(tokens):
-        oracle.decode_reference(pool, lay["page_bytes"], lay, cfg.group, P, table, np.array([tokens]), qs,
-                                W_up, cfg.gq, 1)
+        if rope_theta is None:
+            oracle.decode_reference(pool, lay["page_bytes"], lay, cfg.group, P, table, np.array([tokens]), qs,
+                                    W_up, cfg.gq, 1)
+        else:
+            oracle.decode_reference_rope(pool, lay["page_bytes"], lay, cfg.group, P, table, np.array([tokens]), qs,
+                                         W_up, cfg.gq, 1, rope_theta)
     return run, n_tok
 
 
@@ -115,9 +121,9 @@ def _sample_text(cfg, tokens, what):
             f"{_blas_threads()} threads of {os.cpu_count()} host cores")
 
 
-def cpu_oracle_sample(cfg, target_s=12.0):
+def cpu_oracle_sample(cfg, target_s=12.0, rope_theta=None):
     """The oracle's decode throughput over a bounded sample (about ``target_s`` s)."""
-    run, n_tok = _oracle_decode_case(cfg)
+    run, n_tok = _oracle_decode_case(cfg, rope_theta=rope_theta)
     t0 = time.perf_counter()
     reps = 0
     while True:
@@ -127,7 +133,10 @@ def cpu_oracle_sample(cfg, target_s=12.0):
         if el >= target_s:
             break
     value = reps * n_tok / el  # tokens/s/head (one KV head per pass)
-    return value, _blas_threads(), _sample_text(cfg, n_tok, f"{reps} passes in {el:.1f} s")
+    what = f"{reps} passes in {el:.1f} s"
+    if rope_theta is not None:
+        what += f", reconstruct-then-attend with rotary base {rope_theta:g}"
+    return value, _blas_threads(), _sample_text(cfg, n_tok, what)
 
 
 def cpu_oracle_steps(cfg, steps, warm, budget_s=120.0):
@@ -280,15 +289,20 @@ def run_gpu(args, rank, world):
     OUT = torch.empty_like(Q)
     seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
     ews = [torch.empty(codecs[l].encode_workspace_bytes(B), dtype=torch.uint8, device=dev) for l in range(L)]
-    dws = [torch.zeros(codecs[l].decode_workspace_bytes(B, cap_tokens), dtype=torch.uint8, device=dev)
-           for l in range(L)]
+    rt = args.decode == "reconstruct"
+    ws_bytes = (codecs[0].decode_reconstruct_workspace_bytes if rt else codecs[0].decode_workspace_bytes)
+    dws = [torch.zeros(ws_bytes(B, cap_tokens), dtype=torch.uint8, device=dev) for l in range(L)]
     stream = torch.cuda.Stream(device=dev)
 
     def encode_layer(l):
         codecs[l].encode_append(caches[l], H_new[l], seq_ids, workspace=ews[l], stream=stream)
 
     def decode_layer(l):
-        codecs[l].decode_attend(caches[l], Q[l], OUT[l], workspace=dws[l], stream=stream)
+        if rt:
+            codecs[l].decode_attend_reconstruct(caches[l], Q[l], args.rope_theta, OUT[l], workspace=dws[l],
+                                                stream=stream)
+        else:
+            codecs[l].decode_attend(caches[l], Q[l], OUT[l], workspace=dws[l], stream=stream)
 
     def step():
         for l in range(L):
@@ -376,7 +390,8 @@ def run_gpu(args, rank, world):
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     # encode: fused projection/quantise/pack + commit for steps of <= 16 tokens,
     # else projection + append plan + quantise/pack; decode: fold, split, combine
-    launches_per_layer = (2 if B <= 16 else 3) + 3
+    # (reconstruct-then-attend: split, combine)
+    launches_per_layer = (2 if B <= 16 else 3) + (2 if rt else 3)
     h2d = H_new.numel() * 2 + Q.numel() * 4
     d2h = OUT.numel() * 4
 
@@ -415,6 +430,28 @@ def run_gpu(args, rank, world):
         "gpu_launches": launches_per_layer * L * steps,
         "clocks": clk,
     }
+    if rt:
+        # the rebuild of the keys is fp32 FMA work on the CUDA cores: FLOPs per
+        # (token, KV head) = 2 n_kept_K d_h (lift) + 2 gq d_h (scores) + 2 gq n_kept_V
+        # (probability-weighted V latents), summed over the KV heads of a layer
+        widths = codecs[0].state()["widths"]
+        gq = cfg.n_q_heads // cfg.n_kv_heads
+        flop_tok = sum(2 * cfg.group * int((w[0] > 0).sum()) * cfg.d_head + 2 * gq * cfg.d_head
+                       + 2 * gq * cfg.group * int((w[1] > 0).sum()) for w in widths)
+        flops = B * len_after * flop_tok
+        alu_peak = 148 * 128 * 2 * 1965e6 / 1e12
+        tflops = flops / (dec_avg_ms / 1e3) / 1e12
+        result["config"]["decode"] = f"reconstruct-then-attend, rotary base {args.rope_theta:g}"
+        result["dtype"] = "u8 codes, fp16 scale/zero, fp32 lift and accumulate"
+        result["roofline"] = {
+            "kernel": "rt_split_kernel (keys rebuilt per 64-token tile with fp32 FMAs, rotated, scored; V summed "
+                      "in the latent space), timed with its combine launch",
+            "bound": "alu", "achieved": tflops, "peak": alu_peak, "unit": "TFLOP/s", "frac": tflops / alu_peak,
+            "traffic": None,
+            "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm)",
+            "avg_launch_us": dec_avg_ms * 1e3, "algorithmic_flops_per_launch": flops,
+            "packed_bytes_per_launch": dec_bytes,
+        }
     return result
 
 
@@ -532,6 +569,10 @@ def main():
     ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", default="latent", choices=["latent", "reconstruct"],
+                    help="decode attention: in the latent space (default) or over keys rebuilt per tile")
+    ap.add_argument("--rope-theta", type=float, default=500000.0,
+                    help="reconstruct decode: rotary base (0 = no rotation)")
     ap.add_argument("--prefill-tokens", type=int, default=0,
                     help="prefill mode: tokens in the chunk (default: the workload's 65,536)")
     args = ap.parse_args()
@@ -569,7 +610,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(cfg)
+        cpu = cpu_oracle_sample(cfg, rope_theta=args.rope_theta if args.decode == "reconstruct" else None)
     res = run_gpu(args, rank, world)
     if rank == 0:
         if cpu is not None:

@@ -314,6 +314,33 @@ SPECTRA_API spectra_status spectra_reconstruct(const spectra_codec* codec, const
                                                int32_t seq, int64_t t0, int64_t n, float* K_out, float* V_out,
                                                void* stream);
 
+/* Workspace bytes for spectra_decode_attend_reconstruct with `batch` sequences
+ * of up to max_len tokens (a cache whose max_pages_per_seq * page_tokens is at
+ * most max_len). */
+SPECTRA_API spectra_status spectra_decode_reconstruct_workspace_bytes(const spectra_codec* codec, int32_t batch,
+                                                                      int64_t max_len, size_t* bytes);
+
+/* spectra_decode_attend_reconstruct -- one decode step of attention with the
+ * keys rebuilt from the cache ("SPECTRA pipeline" stage 3 as the pages
+ * integrate it: latents dequantised and lifted back with W_up, then standard
+ * attention), with optional rotary position embedding:
+ *   k^_t = R(t) (c^_K,t W_up^K) for t in [0, lengths[b]),  q' = R(lengths[b]-1) q,
+ *   out = softmax(q' k^^T / sqrt(d_head)) (c^_V W_up^V)
+ * where R(p) turns the pair (i, i + d_head/2) by p * rope_theta^(-2i/d_head)
+ * (the rotate-half form) and rope_theta = 0 means no rotation (then the result
+ * equals spectra_decode_attend's up to rounding).  The values are summed in the
+ * latent space and lifted once per head (the same result by linearity).
+ *   q   device fp32 [batch][n_q_heads][d_head] (before rotation)
+ *   out device fp32 [batch][n_q_heads][d_head]; a sequence of length 0 gives 0
+ *   workspace device, >= spectra_decode_reconstruct_workspace_bytes, 256-byte aligned.
+ * Needs d_head a multiple of 8 and <= 128, <= 128 kept coordinates per side and
+ * <= 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED).  A page id outside
+ * [0, n_pages) or a length outside [0, max_pages_per_seq * page_tokens) records
+ * SPECTRA_ERR_INVALID in the device error word (that part reads as zero). */
+SPECTRA_API spectra_status spectra_decode_attend_reconstruct(const spectra_codec* codec, const spectra_cache* cache,
+                                                             const float* q, double rope_theta, float* out,
+                                                             void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the codec's device error word.
  * Returns the recorded device-side status (SPECTRA_OK if none). */
 SPECTRA_API spectra_status spectra_device_status(const spectra_codec* codec, void* stream);

@@ -664,6 +664,49 @@ def decode_reference(pool: np.ndarray, page_bytes: int, layout: dict, g: int, P:
     return out
 
 
+def rope(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotary position embedding, rotate-half form (reading: the pages do not
+    model positions; this is the usual form for the models they name): for
+    i < d/2 the pair (x_i, x_{i+d/2}) of the row at position p is rotated by the
+    angle p * theta^(-2i/d).  ``x[..., n, d]``, ``positions[n]``; fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    inv = theta ** (-2.0 * np.arange(half) / d)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def decode_reference_rope(pool: np.ndarray, page_bytes: int, layout: dict, g: int, P: int,
+                          page_table: np.ndarray, lengths: np.ndarray, q: np.ndarray, W_up: list,
+                          n_q: int, n_kv: int, theta: float) -> np.ndarray:
+    """Reconstruct-then-attend ([SPECTRA] stage 3): k^, v^ rebuilt from the
+    dequantised cache, keys rotated at their positions 0..L-1 and the query at
+    position L-1 (theta = 0: no rotation), exact softmax attention."""
+    B, d_h = q.shape[0], q.shape[2]
+    gq = n_q // n_kv
+    out = np.zeros((B, n_q, d_h))
+    for b in range(B):
+        L = int(lengths[b])
+        if L == 0:
+            continue
+        for a in range(n_kv):
+            cK = read_side(pool, page_bytes, layout, g, P, page_table[b], L, a, 0)
+            cV = read_side(pool, page_bytes, layout, g, P, page_table[b], L, a, 1)
+            Kh = cK @ np.asarray(W_up[a][0], dtype=np.float64)
+            Vh = cV @ np.asarray(W_up[a][1], dtype=np.float64)
+            if theta > 0:
+                Kh = rope(Kh, np.arange(L), theta)
+            for h in range(a * gq, (a + 1) * gq):
+                qh = np.asarray(q[b, h], dtype=np.float64)[None, :]
+                if theta > 0:
+                    qh = rope(qh, np.array([L - 1]), theta)
+                out[b, h] = softmax_attention(qh[0], Kh, Vh)
+    return out
+
+
 # ----------------------------------------------------------------------------
 # W_O correction                                   [SPECTRA] stage 1, "Refinement"
 # ----------------------------------------------------------------------------

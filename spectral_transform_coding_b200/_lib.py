@@ -67,6 +67,8 @@ _SIGS = {
     "spectra_decode_attend_noalloc": [_vp, _P(CacheDesc), _vp, _vp, _vp],
     "spectra_device_status": [_vp, _vp],
     "spectra_reconstruct": [_vp, _P(CacheDesc), _i32, _i64, _i64, _vp, _vp, _vp],
+    "spectra_decode_reconstruct_workspace_bytes": [_vp, _i32, _i64, _P(ctypes.c_size_t)],
+    "spectra_decode_attend_reconstruct": [_vp, _P(CacheDesc), _vp, ctypes.c_double, _vp, _vp, _sz, _vp],
     "spectra_allocate_widths": [_vp, _i32, _i32, _i32, _i32, _vp, _vp],
     "spectra_allocate_widths_uniform": [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp],
     "spectra_energy_rank": [_vp, _i32, ctypes.c_double, _P(_i32)],

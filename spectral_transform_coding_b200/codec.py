@@ -131,6 +131,12 @@ class Codec:
               "decode_workspace_bytes")
         return n.value
 
+    def decode_reconstruct_workspace_bytes(self, batch: int, max_len: int) -> int:
+        n = ctypes.c_size_t(0)
+        check(lib.spectra_decode_reconstruct_workspace_bytes(self._h, int(batch), int(max_len), ctypes.byref(n)),
+              "decode_reconstruct_workspace_bytes")
+        return n.value
+
     def _workspace(self, nbytes, device):
         torch = _torch()
         return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
@@ -168,6 +174,21 @@ class Codec:
         d = cache.desc()
         check(lib.spectra_decode_attend(self._h, ctypes.byref(d), _ptr(q), _ptr(out), _ptr(ws), ws.numel(),
                                         _stream(stream)), "spectra_decode_attend")
+        return out
+
+    def decode_attend_reconstruct(self, cache: "LatentCache", q, rope_theta: float = 0.0, out=None,
+                                  workspace=None, stream=None):
+        """Decode attention over keys rebuilt from the cache, optionally with rotary
+        position embedding (keys at positions 0..len-1, the query at len-1)."""
+        torch = _torch()
+        if out is None:
+            out = torch.empty_like(q)
+        ws = workspace if workspace is not None else self._workspace(
+            self.decode_reconstruct_workspace_bytes(cache.batch, cache.capacity), q.device)
+        d = cache.desc()
+        check(lib.spectra_decode_attend_reconstruct(self._h, ctypes.byref(d), _ptr(q), float(rope_theta), _ptr(out),
+                                                    _ptr(ws), ws.numel(), _stream(stream)),
+              "spectra_decode_attend_reconstruct")
         return out
 
     def reconstruct(self, cache: "LatentCache", seq: int, t0: int, n: int, stream=None):

@@ -652,6 +652,36 @@ spectra_status spectra_decode_attend(const spectra_codec* c, const spectra_cache
   return SPECTRA_OK;
 }
 
+spectra_status spectra_decode_reconstruct_workspace_bytes(const spectra_codec* c, int32_t batch, int64_t max_len,
+                                                          size_t* bytes) {
+  if (!c || !bytes || batch <= 0 || max_len < 0) return fail(SPECTRA_ERR_INVALID, "bad arguments");
+  const int64_t pages = (max_len + c->h.P - 1) / c->h.P;
+  const RtPlan p = make_rt_plan(c->h, batch, (int)std::min<int64_t>(std::max<int64_t>(pages, 1), 1 << 30));
+  *bytes = p.ws_bytes;
+  return SPECTRA_OK;
+}
+
+spectra_status spectra_decode_attend_reconstruct(const spectra_codec* c, const spectra_cache* cache, const float* q,
+                                                 double rope_theta, float* out, void* workspace,
+                                                 size_t workspace_bytes, void* stream) {
+  if (!c || !q || !out || !workspace) return fail(SPECTRA_ERR_INVALID, "null pointer");
+  if (!(rope_theta == 0.0 || (rope_theta > 1.0 && std::isfinite(rope_theta))))
+    return fail(SPECTRA_ERR_INVALID, "rope_theta must be 0 (no rotation) or a finite base above 1");
+  std::string why;
+  if (!rt_supported(c->h, &why)) return fail(SPECTRA_ERR_UNSUPPORTED, why);
+  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(workspace, 256))
+    return fail(SPECTRA_ERR_INVALID, "misaligned buffer");
+  spectra_status s = check_cache(c, cache);
+  if (s != SPECTRA_OK) return s;
+  s = check_device(c);
+  if (s != SPECTRA_OK) return s;
+  const RtPlan plan = make_rt_plan(c->h, cache->batch, cache->max_pages_per_seq);
+  if (workspace_bytes < plan.ws_bytes) return fail(SPECTRA_ERR_INVALID, "workspace too small");
+  CUDA_TRY(launch_decode_reconstruct(c->h, c->d, *cache, q, rope_theta, out, workspace, plan,
+                                     static_cast<cudaStream_t>(stream)));
+  return SPECTRA_OK;
+}
+
 spectra_status spectra_reconstruct(const spectra_codec* c, const spectra_cache* cache, int32_t seq, int64_t t0,
                                    int64_t n, float* K_out, float* V_out, void* stream) {
   if (!c || !K_out || !V_out) return fail(SPECTRA_ERR_INVALID, "null pointer");

@@ -52,6 +52,21 @@ cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint
 cudaError_t launch_reconstruct(const CodecDev& h, const CodecDev* d, const spectra_cache& cache, int b, int64_t t0,
                                int64_t n, float* K_out, float* V_out, cudaStream_t st);
 
+// Reconstruct-then-attend decode (keys rebuilt per tile, optional rotary
+// position embedding, V summed in the latent space and lifted once per head).
+constexpr int kRtMaxDHead = 128;
+struct RtPlan {
+  int n_split;      // context splits per (KV head, sequence)
+  int part_stride;  // floats per partial record
+  int smem_bytes;   // dynamic shared memory of the split kernel
+  size_t ws_bytes;  // workspace: the partial records
+};
+RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq);
+bool rt_supported(const CodecDev& h, std::string* why);
+cudaError_t launch_decode_reconstruct(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,
+                                      const float* q, double theta, float* out, void* ws, const RtPlan& plan,
+                                      cudaStream_t st);
+
 // decode_kernels.cu
 // Raises `kern`'s dynamic shared-memory limit on the current device to at least
 // `bytes` (one record per kernel and device; the limit never shrinks).

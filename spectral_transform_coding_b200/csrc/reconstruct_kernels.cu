@@ -11,6 +11,10 @@
 // into shared memory, then multiplied by W_up (fp32 accumulation).
 #include <cuda_fp16.h>
 
+#include <algorithm>
+#include <cmath>
+#include <string>
+
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -120,7 +124,455 @@ __global__ void __launch_bounds__(128) reconstruct_kernel(const CodecDev* __rest
   }
 }
 
+// ---------------------------------------------------------------------------
+// Reconstruct-then-attend decode ("SPECTRA pipeline" stage 3 as the pages
+// integrate it: keys and values rebuilt from the latents, then standard
+// attention).  With rotary position embedding the query cannot be folded into
+// the latent space (the rotation depends on the key's position), so each tile
+// of keys is rebuilt in shared memory, rotated, and scored there:
+//
+//   k^_t = R(t) (c^_K,t W_up^K),  q' = R(L-1) q,  p = softmax(q' k^^T / sqrt(d_h))
+//   o = sum_t p_t v^_t = (sum_t p_t c^_V,t) W_up^V
+//
+// v^ is never materialised: by linearity the V lift runs once per head on the
+// probability-weighted latent sum, after the splits are merged.  R(p) turns the
+// pair (i, i + d_h/2) by p * theta^(-2i/d_h); theta = 0 means no rotation.
+//
+// One CTA per (KV head, sequence, context split), 256 threads, 64-token tiles:
+//   1. dequantise the tile's K latents (transposed) and V latents into smem;
+//   2. lift: each thread computes 4 tokens x (4 dims + their 4 rotation
+//      partners) of k^ with fp32 FMAs against W_up^K staged once per CTA, then
+//      rotates them;
+//   3. scores of the KV head's q heads, online softmax (exp2 domain), and the
+//      probability-weighted sum of the V latents in registers.
+// A combine kernel merges the splits and applies W_up^V.
+// ---------------------------------------------------------------------------
+constexpr int kRtTokens = 64;
+constexpr int kRtThreads = 256;
+constexpr int kRtMaxSplit = 64;
+constexpr int kRtAccSlots = kMaxGQ * kRtMaxDHead / kRtThreads;  // V accumulators per thread
+
+// Byte offsets of the split kernel's shared-memory regions.
+struct RtSmem {
+  int om, w, ct, cv, kh, qs, sc, ml, pg, total;
+  __host__ __device__ RtSmem(int d_h, int max_k, int max_v, int gq) {
+    int o = 0;
+    om = o;  // rotation frequencies in half-turns per position, double [d_h / 2]
+    o += kRtMaxDHead / 2 * 8;
+    w = o;  // W_up^K, [n_kept][d_h]
+    o += max_k * d_h * 4;
+    ct = o;  // K latents, transposed [n_kept][kRtTokens]
+    o += max_k * kRtTokens * 4;
+    cv = o;  // V latents [kRtTokens][max_v + 1]
+    o += (kRtTokens * (max_v + 1) * 4 + 15) / 16 * 16;
+    kh = o;  // rotated keys [kRtTokens][d_h + 1]
+    o += (kRtTokens * (d_h + 1) * 4 + 15) / 16 * 16;
+    qs = o;  // rotated, scaled queries [gq][d_h]
+    o += gq * d_h * 4;
+    sc = o;  // scores, then probabilities [gq][kRtTokens]
+    o += gq * kRtTokens * 4;
+    ml = o;  // running max, sum and correction per q head
+    o += 3 * kMaxGQ * 4;
+    o = (o + 15) / 16 * 16;
+    pg = o;  // byte offset of each tile token's page in the pool (-1: bad page id)
+    o += kRtTokens * 8;
+    total = o;
+  }
+};
+
+struct RtArgs {
+  const CodecDev* cd;
+  const uint8_t* pool;
+  const int32_t* page_table;
+  const int32_t* lengths;
+  int64_t n_pool_pages;
+  int max_pages;
+  int n_split;
+  int part_stride;  // floats per partial record: max, sum, then the V latent sum
+  double theta;     // rotary base; 0 = no rotation
+  float qscale;     // log2(e) / sqrt(d_h)
+  const float* q;
+  float* part;
+};
+
+// Turns (x, y) by `turns` * pi radians.  The angle, in half-turns, is reduced
+// to [-1, 1] in double (turns - 2 rint(turns / 2), exact up to the rounding of
+// `turns` itself), then sin(pi r) and cos(pi r) run in fp32.
+__device__ __forceinline__ void rope_rotate(float& x, float& y, double turns) {
+  const double k = rint(turns * 0.5);
+  const float r = (float)fma(-2.0, k, turns);
+  float sn, cs;
+  sincospif(r, &sn, &cs);
+  const float x2 = x * cs - y * sn, y2 = y * cs + x * sn;
+  x = x2;
+  y = y2;
+}
+
+// dst[k * stride] = code_k * s + z for the G codes of one token in one group of
+// width b (warp-uniform); G and the side are compile-time, so the fragment
+// positions fold to constants and the word loads of all G codes issue together.
+template <int G, int SIDE>
+__device__ __forceinline__ void dequant_token(const uint32_t* __restrict__ blk, int b, int tb, float s, float z,
+                                              float* dst, int stride) {
+  uint32_t code[G];
+  int gid[G], t4[G], slot[G];
+#pragma unroll
+  for (int k = 0; k < G; ++k) frag_pos(G, SIDE, tb, k, &gid[k], &t4[k], &slot[k]);
+  switch (b) {
+    case 4:
+#pragma unroll
+      for (int k = 0; k < G; ++k) code[k] = (__ldg(blk + 4 * gid[k] + t4[k]) >> (4 * slot[k])) & 0xFu;
+      break;
+    case 2:
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+        code[k] = (__ldg(blk + 2 * gid[k] + (t4[k] >> 1)) >> (4 * slot[k] + 2 * (t4[k] & 1))) & 0x3u;
+      break;
+    case 1:
+#pragma unroll
+      for (int k = 0; k < G; ++k) code[k] = (__ldg(blk + gid[k]) >> (4 * slot[k] + t4[k])) & 0x1u;
+      break;
+    case 3:
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+        code[k] = ((__ldg(blk + 2 * gid[k] + (t4[k] >> 1)) >> (4 * slot[k] + 2 * (t4[k] & 1))) & 0x3u) |
+                  (((__ldg(blk + 16 + gid[k]) >> (4 * slot[k] + t4[k])) & 0x1u) << 2);
+      break;
+    default:
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+        code[k] = (__ldg(blk + 2 * (4 * gid[k] + t4[k]) + ((slot[k] >> 1) & 1)) >>
+                   (8 * ((slot[k] & 1) + 2 * (slot[k] >> 2)))) & 0xFFu;
+      break;
+  }
+#pragma unroll
+  for (int k = 0; k < G; ++k) dst[k * stride] = fmaf((float)code[k], s, z);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const CodecDev* cd = A.cd;
+  const int a = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int d_h = cd->d_h, half = d_h / 2, gq = cd->gq, P = cd->P;
+  constexpr int TB = 256 / G;
+  const SideDev& sk = cd->head[a].side[0];
+  const SideDev& sv = cd->head[a].side[1];
+  const int nkK = sk.n_kept, nkV = sv.n_kept, cvs = cd->max_kept_v + 1;
+  const RtSmem L(d_h, cd->max_kept_k, cd->max_kept_v, gq);
+  double* om = reinterpret_cast<double*>(sm + L.om);
+  float* Ws = reinterpret_cast<float*>(sm + L.w);
+  float* cT = reinterpret_cast<float*>(sm + L.ct);
+  float* cV = reinterpret_cast<float*>(sm + L.cv);
+  float* kh = reinterpret_cast<float*>(sm + L.kh);
+  float* qs = reinterpret_cast<float*>(sm + L.qs);
+  float* sc = reinterpret_cast<float*>(sm + L.sc);
+  float* ml = reinterpret_cast<float*>(sm + L.ml);  // [0, 8) max, [8, 16) sum, [16, 24) correction
+  int64_t* pg = reinterpret_cast<int64_t*>(sm + L.pg);
+  const bool rot = A.theta > 0.0;
+
+  // W_up^K is stored transposed ([d_h][n_kept]); stage it as [n_kept][d_h]
+  const float* wk = cd->w_up + sk.wup_off;
+  for (int e = tid; e < nkK * d_h; e += kRtThreads) Ws[(e % nkK) * d_h + e / nkK] = wk[e];
+  if (rot)
+    for (int i = tid; i < half; i += kRtThreads) om[i] = pow(A.theta, -2.0 * i / d_h) / 3.141592653589793;
+  if (tid < kMaxGQ) {
+    ml[tid] = -INFINITY;
+    ml[kMaxGQ + tid] = 0.f;
+  }
+  int len = A.lengths[b];
+  if (len < 0 || (int64_t)len > (int64_t)A.max_pages * P) {
+    if (tid == 0) device_error(cd->err, SPECTRA_ERR_INVALID);
+    len = 0;
+  }
+  __syncthreads();
+  // queries of this KV head's q heads, turned to position len - 1 and scaled
+  for (int e = tid; e < gq * half; e += kRtThreads) {
+    const int h = e / half, i = e % half;
+    const float* qv = A.q + ((size_t)b * cd->n_q + (size_t)a * gq + h) * d_h;
+    float x = qv[i], y = qv[i + half];
+    if (rot && len > 0) rope_rotate(x, y, (double)(len - 1) * om[i]);
+    qs[h * d_h + i] = x * A.qscale;
+    qs[h * d_h + i + half] = y * A.qscale;
+  }
+
+  const int tiles = (len + kRtTokens - 1) / kRtTokens;
+  const int per = (tiles + A.n_split - 1) / A.n_split;
+  const int tok_begin = min(split * per, tiles) * kRtTokens;
+  const int tok_end = min(min((split + 1) * per, tiles) * kRtTokens, len);
+  const int ngK = sk.n_groups, n_items = kRtTokens * (ngK + sv.n_groups);
+  const int n_acc = gq * nkV;
+  float acc[kRtAccSlots];
+#pragma unroll
+  for (int k = 0; k < kRtAccSlots; ++k) acc[k] = 0.f;
+
+  for (int t0 = tok_begin; t0 < tok_end; t0 += kRtTokens) {
+    const int nt = min(kRtTokens, tok_end - t0);
+    // ---- 1. dequantised latents of the tile (rows past the end are zero) ----
+    if (tid < kRtTokens) {
+      int64_t off = -1;
+      if (tid < nt) {
+        const int pid = A.page_table[(size_t)b * A.max_pages + (t0 + tid) / P];
+        if (pid < 0 || (int64_t)pid >= A.n_pool_pages)
+          device_error(cd->err, SPECTRA_ERR_INVALID);
+        else
+          off = (int64_t)pid * cd->page_bytes;
+      }
+      pg[tid] = off;
+    }
+    __syncthreads();
+    for (int e = tid; e < n_items; e += kRtThreads) {
+      const int t = e % kRtTokens, jj = e / kRtTokens;
+      const int side = jj < ngK ? 0 : 1, j = side ? jj - ngK : jj;
+      const GroupDev gd = (side ? sv : sk).grp[j];
+      const int64_t off = pg[t];
+      float* dst = side == 0 ? cT + (j * G) * kRtTokens + t : cV + t * cvs + j * G;
+      const int stride = side == 0 ? kRtTokens : 1;
+      if (off < 0) {
+#pragma unroll
+        for (int k = 0; k < G; ++k) dst[k * stride] = 0.f;
+        continue;
+      }
+      const uint8_t* page = A.pool + off;
+      const int tau = (t0 + t) % P, u = tau >> 1;
+      const uint32_t* blk = reinterpret_cast<const uint32_t*>(page + gd.plane_off + (tau / TB) * (32 * gd.b));
+      const uint2 rec = __ldg(reinterpret_cast<const uint2*>(page + gd.sz_off + 8 * ((u & 7) * (P >> 4) + (u >> 3))));
+      const uint32_t sw = rec.x, zw = rec.y;  // {s[2u], s[2u+1]}, {z[2u], z[2u+1]}
+      const float sv_ = (tau & 1) ? half_hi(sw) : half_lo(sw), zv = (tau & 1) ? half_hi(zw) : half_lo(zw);
+      if (side == 0)
+        dequant_token<G, 0>(blk, gd.b, tau % TB, sv_, zv, dst, stride);
+      else
+        dequant_token<G, 1>(blk, gd.b, tau % TB, sv_, zv, dst, stride);
+    }
+    __syncthreads();
+    // ---- 2. k^ = c^_K W_up^K for 4 tokens x (4 dims + partners), rotated ----
+    for (int e = tid; e < (kRtTokens / 4) * (half / 4); e += kRtThreads) {
+      const int tq = e % (kRtTokens / 4), dq = e / (kRtTokens / 4);
+      float lo[4][4], hi[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jn = 0; jn < 4; ++jn) lo[i][jn] = hi[i][jn] = 0.f;
+      for (int c = 0; c < nkK; ++c) {
+        const float4 cv = *reinterpret_cast<const float4*>(cT + c * kRtTokens + 4 * tq);
+        const float4 wl = *reinterpret_cast<const float4*>(Ws + c * d_h + 4 * dq);
+        const float4 wh = *reinterpret_cast<const float4*>(Ws + c * d_h + half + 4 * dq);
+        const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, wa[4] = {wl.x, wl.y, wl.z, wl.w},
+                    wb[4] = {wh.x, wh.y, wh.z, wh.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jn = 0; jn < 4; ++jn) {
+            lo[i][jn] = fmaf(cc[i], wa[jn], lo[i][jn]);
+            hi[i][jn] = fmaf(cc[i], wb[jn], hi[i][jn]);
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * tq + i;
+#pragma unroll
+        for (int jn = 0; jn < 4; ++jn) {
+          const int d = 4 * dq + jn;
+          float x = lo[i][jn], y = hi[i][jn];
+          if (rot) rope_rotate(x, y, (double)(t0 + t) * om[d]);
+          kh[t * (d_h + 1) + d] = x;
+          kh[t * (d_h + 1) + half + d] = y;
+        }
+      }
+    }
+    __syncthreads();
+    // ---- 3. scores (log2 units), online softmax, V latent sums --------------
+    for (int e = tid; e < gq * kRtTokens; e += kRtThreads) {
+      const int h = e / kRtTokens, t = e % kRtTokens;
+      float v = -INFINITY;
+      if (t < nt) {
+        const float* qr = qs + h * d_h;
+        const float* kr = kh + t * (d_h + 1);
+        float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+        for (int d = 0; d < d_h; d += 4) {
+          v0 = fmaf(qr[d], kr[d], v0);
+          v1 = fmaf(qr[d + 1], kr[d + 1], v1);
+          v2 = fmaf(qr[d + 2], kr[d + 2], v2);
+          v3 = fmaf(qr[d + 3], kr[d + 3], v3);
+        }
+        v = (v0 + v1) + (v2 + v3);
+      }
+      sc[h * kRtTokens + t] = v;
+    }
+    __syncthreads();
+    if (warp < gq) {
+      float* row = sc + warp * kRtTokens;
+      float mx = -INFINITY;
+      for (int t = lane; t < kRtTokens; t += 32) mx = fmaxf(mx, row[t]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_old = ml[warp], m_new = fmaxf(m_old, mx);
+      float sum = 0.f;
+      for (int t = lane; t < kRtTokens; t += 32) {
+        const float p = exp2f(row[t] - m_new);
+        row[t] = p;
+        sum += p;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      __syncwarp();
+      if (lane == 0) {
+        const float corr = exp2f(m_old - m_new);
+        ml[warp] = m_new;
+        ml[kMaxGQ + warp] = ml[kMaxGQ + warp] * corr + sum;
+        ml[2 * kMaxGQ + warp] = corr;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kRtAccSlots; ++k) {
+      const int e = tid + k * kRtThreads;
+      if (e < n_acc) {
+        const int h = e / nkV, c = e % nkV;
+        const float* p = sc + h * kRtTokens;
+        const float* cc = cV + c;
+        float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+        int t = 0;
+        for (; t + 4 <= nt; t += 4) {
+          v0 = fmaf(p[t], cc[t * cvs], v0);
+          v1 = fmaf(p[t + 1], cc[(t + 1) * cvs], v1);
+          v2 = fmaf(p[t + 2], cc[(t + 2) * cvs], v2);
+          v3 = fmaf(p[t + 3], cc[(t + 3) * cvs], v3);
+        }
+        for (; t < nt; ++t) v0 = fmaf(p[t], cc[t * cvs], v0);
+        acc[k] = fmaf(acc[k], ml[2 * kMaxGQ + h], (v0 + v1) + (v2 + v3));
+      }
+    }
+    __syncthreads();  // the next tile overwrites the latents and probabilities
+  }
+  // ---- partial record per q head: max, sum, V latent sum ---------------------
+  const size_t rec0 = ((size_t)b * cd->n_q + (size_t)a * gq) * A.n_split + split;
+#pragma unroll
+  for (int k = 0; k < kRtAccSlots; ++k) {
+    const int e = tid + k * kRtThreads;
+    if (e < n_acc) {
+      const int h = e / nkV, c = e % nkV;
+      A.part[(rec0 + (size_t)h * A.n_split) * A.part_stride + 2 + c] = acc[k];
+    }
+  }
+  if (tid < gq) {
+    A.part[(rec0 + (size_t)tid * A.n_split) * A.part_stride] = ml[tid];
+    A.part[(rec0 + (size_t)tid * A.n_split) * A.part_stride + 1] = ml[kMaxGQ + tid];
+  }
+}
+
+// Merges the splits of one (q head, sequence) and lifts with W_up^V.
+__global__ void __launch_bounds__(128) rt_combine_kernel(const CodecDev* __restrict__ cd,
+                                                         const float* __restrict__ part, int n_split, int stride,
+                                                         float* __restrict__ out) {
+  __shared__ float wgt[kRtMaxSplit];
+  __shared__ float lat[kRtMaxDHead];
+  __shared__ float inv_l;
+  const int hq = blockIdx.x, b = blockIdx.y, a = hq / cd->gq, tid = threadIdx.x;
+  const SideDev& sv = cd->head[a].side[1];
+  const int nkV = sv.n_kept, d_h = cd->d_h;
+  const float* rec = part + ((size_t)b * cd->n_q + hq) * n_split * stride;
+  if (tid < 32) {
+    float M = -INFINITY;
+    for (int s = tid; s < n_split; s += 32) M = fmaxf(M, rec[(size_t)s * stride]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Lsum = 0.f;
+    for (int s = tid; s < n_split; s += 32) {
+      const float m = rec[(size_t)s * stride];
+      const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+      wgt[s] = w;
+      Lsum = fmaf(w, rec[(size_t)s * stride + 1], Lsum);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    if (tid == 0) inv_l = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  }
+  __syncthreads();
+  for (int c = tid; c < nkV; c += blockDim.x) {
+    float v = 0.f;
+    for (int s = 0; s < n_split; ++s) v = fmaf(wgt[s], rec[(size_t)s * stride + 2 + c], v);
+    lat[c] = v * inv_l;
+  }
+  __syncthreads();
+  const float* wv = cd->w_up + sv.wup_off;  // [n_kept][d_h]
+  for (int d = tid; d < d_h; d += blockDim.x) {
+    float o = 0.f;
+    for (int c = 0; c < nkV; ++c) o = fmaf(lat[c], wv[(size_t)c * d_h + d], o);
+    out[((size_t)b * cd->n_q + hq) * d_h + d] = o;
+  }
+}
+
+int rt_sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
 }  // namespace
+
+RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq) {
+  RtPlan p{};
+  const int64_t max_tiles = ((int64_t)max_pages_per_seq * h.P + kRtTokens - 1) / kRtTokens;
+  // one CTA per SM fits (about 170 KB of shared memory at d_h = 128): split the
+  // context so that the (KV head, sequence) pairs fill the SMs once
+  const int pairs = h.n_kv * batch;
+  int ns = rt_sm_count() / pairs;  // one wave: (KV head, sequence) pairs x splits <= SMs
+  ns = (int)std::max<int64_t>(1, std::min<int64_t>({(int64_t)ns, (int64_t)kRtMaxSplit, max_tiles}));
+  p.n_split = ns;
+  p.part_stride = (2 + h.max_kept_v + 3) / 4 * 4;
+  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq).total;
+  p.ws_bytes = ((size_t)batch * h.n_q * ns * p.part_stride * 4 + 255) / 256 * 256;
+  return p;
+}
+
+bool rt_supported(const CodecDev& h, std::string* why) {
+  if (h.d_h > kRtMaxDHead || h.d_h % 8 != 0) {
+    *why = "reconstruct-then-attend needs d_head a multiple of 8 and at most 128";
+    return false;
+  }
+  if (h.max_kept_k > kRtMaxDHead || h.max_kept_v > kRtMaxDHead) {
+    *why = "reconstruct-then-attend needs at most 128 kept coordinates per side";
+    return false;
+  }
+  if (h.gq > kMaxGQ) {
+    *why = "reconstruct-then-attend needs at most 8 q heads per KV head";
+    return false;
+  }
+  return true;
+}
+
+cudaError_t launch_decode_reconstruct(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,
+                                      const float* q, double theta, float* out, void* ws, const RtPlan& plan,
+                                      cudaStream_t st) {
+  RtArgs A{};
+  A.cd = d;
+  A.pool = static_cast<const uint8_t*>(cache.pool);
+  A.page_table = cache.page_table;
+  A.lengths = cache.lengths;
+  A.n_pool_pages = cache.n_pages;
+  A.max_pages = cache.max_pages_per_seq;
+  A.n_split = plan.n_split;
+  A.part_stride = plan.part_stride;
+  A.theta = theta;
+  A.qscale = (float)(1.4426950408889634 / std::sqrt((double)h.d_h));
+  A.q = q;
+  A.part = static_cast<float*>(ws);
+  auto kern = h.group == 16 ? rt_split_kernel<16> : rt_split_kernel<8>;
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), plan.smem_bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(h.n_kv, cache.batch, plan.n_split), kRtThreads, plan.smem_bytes, st>>>(A);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  rt_combine_kernel<<<dim3(h.n_q, cache.batch), 128, 0, st>>>(d, A.part, plan.n_split, plan.part_stride, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_reconstruct(const CodecDev& h, const CodecDev* d, const spectra_cache& cache, int b, int64_t t0,
                                int64_t n, float* K_out, float* V_out, cudaStream_t st) {

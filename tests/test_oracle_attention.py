@@ -113,3 +113,30 @@ def test_quantised_attention_close_to_exact(toy_cfg, toy_layer, toy_codec):
         ref = oracle.softmax_attention(q[0, hq], K, V)
         cos = out[0, hq] @ ref / np.linalg.norm(out[0, hq]) / np.linalg.norm(ref)
         assert cos > 0.8
+
+
+# --- rotary position embedding of the reconstruct-then-attend path -------------------
+
+def test_rope_is_identity_at_position_zero_and_preserves_norms():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, 16))
+    np.testing.assert_array_equal(oracle.rope(x, np.zeros(5), 10000.0), x)
+    y = oracle.rope(x, np.arange(5) * 37, 10000.0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    rng = np.random.default_rng(2)
+    q, k = rng.standard_normal((1, 32)), rng.standard_normal((1, 32))
+    s1 = oracle.rope(q, np.array([10]), 500.0) @ oracle.rope(k, np.array([3]), 500.0).T
+    s2 = oracle.rope(q, np.array([1007]), 500.0) @ oracle.rope(k, np.array([1000]), 500.0).T
+    np.testing.assert_allclose(s1, s2, rtol=1e-10)
+
+
+def test_rope_pair_rotation_by_hand():
+    """d = 4, theta = 100: pair (x0, x2) turns by p * 100^0 = p, pair (x1, x3) by
+    p * 100^(-1/2) = p / 10; at p = pi/2 the first pair maps (1, 0) -> (0, 1)."""
+    x = np.array([[1.0, 0.0, 0.0, 2.0]])
+    y = oracle.rope(x, np.array([np.pi / 2]), 100.0)
+    a2 = np.pi / 20
+    np.testing.assert_allclose(y[0], [0.0, -2 * np.sin(a2), 1.0, 2 * np.cos(a2)], atol=1e-15)
