@@ -333,7 +333,7 @@ SPECTRA_API spectra_status spectra_decode_reconstruct_workspace_bytes(const spec
  *   q   device fp32 [batch][n_q_heads][d_head] (before rotation)
  *   out device fp32 [batch][n_q_heads][d_head]; a sequence of length 0 gives 0
  *   workspace device, >= spectra_decode_reconstruct_workspace_bytes, 256-byte aligned.
- * Needs d_head a multiple of 8 and <= 128, <= 128 kept coordinates per side and
+ * Needs d_head a multiple of 16 and <= 128, <= 128 kept coordinates per side and
  * <= 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED).  A page id outside
  * [0, n_pages) or a length outside [0, max_pages_per_seq * page_tokens) records
  * SPECTRA_ERR_INVALID in the device error word (that part reads as zero). */

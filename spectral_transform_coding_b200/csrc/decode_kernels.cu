@@ -16,10 +16,11 @@
 // Three kernels per decode step, chained with programmatic dependent launch:
 //   fold    one CTA per (sequence, KV head): q_lat and its group sums, written
 //           as the split kernel's MMA B fragments;
-//   split   one CTA per (context split, KV head, sequence): streams its pages
-//           (bulk copies into per-warp shared-memory stages) while the fold
-//           runs, then an online softmax over 64-token chunks; one partial
-//           record (max, sum, latent accumulator) per q head;
+//   split   one CTA per (context split, KV head, sequence): prefetches its
+//           pages into L2 while the fold runs, then streams them (bulk copies
+//           into per-warp shared-memory stages) through an online softmax
+//           over 64-token chunks; one partial record (max, sum, latent
+//           accumulator) per q head;
 //   combine one CTA per (q head, sequence): merges the splits, applies W_up^V
 //           (bulk-copied into shared memory while the splits finish).
 #include <cuda_fp16.h>
@@ -458,18 +459,64 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   const int tpp = P / 16;  // tiles per page
   const HeadDev* hd = &cd->head[a];
   const int sec_off = hd->sec_off, sec_bytes = hd->sec_bytes;
-  const int len = A.lengths[b];
-  const int n_pages = (len + P - 1) / P;
-  // pages per split: a multiple of the warp count, so the warps of a CTA get
-  // equal shares (trailing splits may get fewer pages or none)
-  const int per = ((n_pages + A.n_split - 1) / A.n_split + kDecWarps - 1) / kDecWarps * kDecWarps;
-  const int p0 = min(split * per, n_pages), p1 = min(p0 + per, n_pages);
-  const int count = (p1 - p0 > warp) ? (p1 - p0 - warp + kDecWarps - 1) / kDecWarps : 0;
   const SideDev* sk = &hd->side[0];
   const SideDev* sv = &hd->side[1];
   const int nK = sk->n_groups, nV = sv->n_groups;
+  const int S = A.stages;
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // pages per split: a multiple of the warp count, so the warps of a CTA get
+  // equal shares (trailing splits may get fewer pages or none)
+  auto page_range = [&](int len_, int& p0_, int& count_) {
+    const int n_pages = (len_ + P - 1) / P;
+    const int per = ((n_pages + A.n_split - 1) / A.n_split + kDecWarps - 1) / kDecWarps * kDecWarps;
+    p0_ = min(split * per, n_pages);
+    const int p1_ = min(p0_ + per, n_pages);
+    count_ = (p1_ - p0_ > warp) ? (p1_ - p0_ - warp + kDecWarps - 1) / kDecWarps : 0;
+  };
 
-  // ---- 1. page ids of this warp, then its first bulk copies -----------------
+  // ---- 1. L2 warm-up of this warp's pages -----------------------------------
+  // Every kernel of the chain lets its successor start at its own start, so up
+  // to the dependency wait below the encode kernels of the same step may still
+  // be writing the lengths and the pages.  Here the length is only a hint for
+  // prefetches, which move bytes toward L2 and change nothing; the page table
+  // is written by no kernel.  Lengths and pages are read for real after the wait.
+  {
+    const int hint = A.lengths[b];
+    if (hint > 0 && (int64_t)hint <= (int64_t)A.max_pages * P) {
+      int hp0, hcount;
+      page_range(hint, hp0, hcount);
+      for (int i = lane; i < hcount; i += 32) {
+        const int pid = A.page_table[(size_t)b * A.max_pages + hp0 + warp + kDecWarps * i];
+        if (pid >= 0 && (int64_t)pid < A.n_pool_pages)
+          bulk_prefetch_l2(A.pool + (size_t)pid * (size_t)A.page_bytes + sec_off, (uint32_t)sec_bytes);
+      }
+    }
+  }
+
+  // group tables (built on the host with the page layout)
+  {
+    static_assert(sizeof(DecodeTables) % 16 == 0, "DecodeTables must copy as int4");
+    const int4* src = reinterpret_cast<const int4*>(&hd->dec);
+    int4* dst = reinterpret_cast<int4*>(&T);
+    for (int e = tid; e < (int)(sizeof(DecodeTables) / 16); e += blockDim.x) dst[e] = src[e];
+  }
+  for (int j = 0; j < kMaxG; ++j) vacc_s[j * 32 + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+  // ---- 2. wait; then the length, this warp's page ids, its first copies -----
+  // (the wait covers the fold grid, which waits before it exits, and so every
+  // earlier kernel of the stream)
+  pdl_wait();
+  int len = A.lengths[b];
+  if (len < 0 || (int64_t)len > (int64_t)A.max_pages * P) {  // lengths written outside the library
+    if (tid == 0) device_error(cd->err, SPECTRA_ERR_INVALID);
+    len = 0;
+  }
+  int p0, count;
+  page_range(len, p0, count);
   bool bad = false;
   for (int i = lane; i < count; i += 32) {
     const int pid = A.page_table[(size_t)b * A.max_pages + p0 + warp + kDecWarps * i];
@@ -478,12 +525,6 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   const bool warp_bad = __any_sync(0xffffffffu, bad);
   if (warp_bad && lane == 0) device_error(cd->err, SPECTRA_ERR_INVALID);
   const int my_count = warp_bad ? 0 : count;
-  const int S = A.stages;
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
   auto issue = [&](int i) {
     const int pg = p0 + warp + kDecWarps * i;
     const int pid = A.page_table[(size_t)b * A.max_pages + pg];
@@ -495,17 +536,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   if (lane == 0)
     for (int i = 0; i < min(S, my_count); ++i) issue(i);
 
-  // group tables (built on the host with the page layout)
-  {
-    static_assert(sizeof(DecodeTables) % 16 == 0, "DecodeTables must copy as int4");
-    const int4* src = reinterpret_cast<const int4*>(&hd->dec);
-    int4* dst = reinterpret_cast<int4*>(&T);
-    for (int e = tid; e < (int)(sizeof(DecodeTables) / 16); e += blockDim.x) dst[e] = src[e];
-  }
-  for (int j = 0; j < kMaxG; ++j) vacc_s[j * 32 + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
-
-  // ---- 2. the folded query (written by the fold grid) -----------------------
-  pdl_wait();
+  // ---- 3. the folded query (written by the fold grid) -----------------------
   {
     // rows j*NT + nt (j < kMaxG) and the bz rows kMaxG*2 + nt
     const uint2* src = A.frag + ((size_t)b * A.n_kv + a) * kFragWords;

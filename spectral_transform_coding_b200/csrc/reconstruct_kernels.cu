@@ -139,10 +139,15 @@ __global__ void __launch_bounds__(128) reconstruct_kernel(const CodecDev* __rest
 // pair (i, i + d_h/2) by p * theta^(-2i/d_h); theta = 0 means no rotation.
 //
 // One CTA per (KV head, sequence, context split), 256 threads, 64-token tiles:
-//   1. dequantise the tile's K latents (transposed) and V latents into smem;
-//   2. lift: each thread computes 4 tokens x (4 dims + their 4 rotation
-//      partners) of k^ with fp32 FMAs against W_up^K staged once per CTA, then
-//      rotates them;
+//   1. unpack the tile's K codes into shared memory as fp16 (exact: codes are
+//      integers below 256) with their per-group s and z, and dequantise the V
+//      latents (fp32);
+//   2. lift on the tensor cores (mma.sync): per group j,
+//        P_j = code_j W_j  (W_up^K rows of group j split into fp16 hi + lo,
+//                           so P_j keeps about 22 bits; fp32 accumulate)
+//        k^ += s_j P_j + z_j (sum of the rows of W_j)
+//      in 16-token x 8-dim tiles, a warp holding a dim and its rotation
+//      partner d + d_h/2 in the same registers; then the rotation;
 //   3. scores of the KV head's q heads, online softmax (exp2 domain), and the
 //      probability-weighted sum of the V latents in registers.
 // A combine kernel merges the splits and applies W_up^V.
@@ -152,17 +157,25 @@ constexpr int kRtThreads = 256;
 constexpr int kRtMaxSplit = 64;
 constexpr int kRtAccSlots = kMaxGQ * kRtMaxDHead / kRtThreads;  // V accumulators per thread
 
-// Byte offsets of the split kernel's shared-memory regions.
+// Byte offsets of the split kernel's shared-memory regions (max_k, max_v:
+// largest kept coordinates per side over the heads; G: group size).
 struct RtSmem {
-  int om, w, ct, cv, kh, qs, sc, ml, pg, total;
-  __host__ __device__ RtSmem(int d_h, int max_k, int max_v, int gq) {
+  int om, bf, ws, ck, sz, cv, kh, qs, sc, ml, pg, total;
+  int ck_stride, n_grp;  // halves per K code row; groups per side (max)
+  __host__ __device__ RtSmem(int d_h, int max_k, int max_v, int gq, int G) {
+    ck_stride = max_k + 8;
+    n_grp = max_k / G > 0 ? max_k / G : 1;
     int o = 0;
     om = o;  // rotation frequencies in half-turns per position, double [d_h / 2]
     o += kRtMaxDHead / 2 * 8;
-    w = o;  // W_up^K, [n_kept][d_h]
+    bf = o;  // W_up^K as MMA B fragments: fp16 hi and lo, [group][n-tile][hi, lo][G/8][32 lanes] words
     o += max_k * d_h * 4;
-    ct = o;  // K latents, transposed [n_kept][kRtTokens]
-    o += max_k * kRtTokens * 4;
+    ws = o;  // per group, the sum of its rows of W_up^K [group][d_h]
+    o += n_grp * d_h * 4;
+    ck = o;  // K codes, fp16 [kRtTokens][ck_stride]
+    o += kRtTokens * ck_stride * 2;
+    sz = o;  // K scale and zero, fp32 [2][kRtTokens][n_grp]
+    o += 2 * kRtTokens * n_grp * 4;
     cv = o;  // V latents [kRtTokens][max_v + 1]
     o += (kRtTokens * (max_v + 1) * 4 + 15) / 16 * 16;
     kh = o;  // rotated keys [kRtTokens][d_h + 1]
@@ -208,13 +221,11 @@ __device__ __forceinline__ void rope_rotate(float& x, float& y, double turns) {
   y = y2;
 }
 
-// dst[k * stride] = code_k * s + z for the G codes of one token in one group of
-// width b (warp-uniform); G and the side are compile-time, so the fragment
-// positions fold to constants and the word loads of all G codes issue together.
+// The G codes of one token in one group of width b (warp-uniform); G and the
+// side are compile-time, so the fragment positions fold to constants and the
+// word loads of all G codes issue together.
 template <int G, int SIDE>
-__device__ __forceinline__ void dequant_token(const uint32_t* __restrict__ blk, int b, int tb, float s, float z,
-                                              float* dst, int stride) {
-  uint32_t code[G];
+__device__ __forceinline__ void unpack_token(const uint32_t* __restrict__ blk, int b, int tb, uint32_t (&code)[G]) {
   int gid[G], t4[G], slot[G];
 #pragma unroll
   for (int k = 0; k < G; ++k) frag_pos(G, SIDE, tb, k, &gid[k], &t4[k], &slot[k]);
@@ -245,8 +256,6 @@ __device__ __forceinline__ void dequant_token(const uint32_t* __restrict__ blk, 
                    (8 * ((slot[k] & 1) + 2 * (slot[k] >> 2)))) & 0xFFu;
       break;
   }
-#pragma unroll
-  for (int k = 0; k < G; ++k) dst[k * stride] = fmaf((float)code[k], s, z);
 }
 
 template <int G>
@@ -260,10 +269,14 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   const SideDev& sk = cd->head[a].side[0];
   const SideDev& sv = cd->head[a].side[1];
   const int nkK = sk.n_kept, nkV = sv.n_kept, cvs = cd->max_kept_v + 1;
-  const RtSmem L(d_h, cd->max_kept_k, cd->max_kept_v, gq);
+  const RtSmem L(d_h, cd->max_kept_k, cd->max_kept_v, gq, G);
+  const int cks = L.ck_stride, ngs = L.n_grp, n_nt = d_h / 8, half_nt = n_nt / 2;
+  constexpr int KQ = G / 8;  // B fragment registers per lane (m16n8k16: 2, m16n8k8: 1)
   double* om = reinterpret_cast<double*>(sm + L.om);
-  float* Ws = reinterpret_cast<float*>(sm + L.w);
-  float* cT = reinterpret_cast<float*>(sm + L.ct);
+  uint32_t* bf = reinterpret_cast<uint32_t*>(sm + L.bf);
+  float* wsum = reinterpret_cast<float*>(sm + L.ws);
+  __half* ck = reinterpret_cast<__half*>(sm + L.ck);
+  float* szk = reinterpret_cast<float*>(sm + L.sz);  // [0]: s, [kRtTokens * ngs]: z
   float* cV = reinterpret_cast<float*>(sm + L.cv);
   float* kh = reinterpret_cast<float*>(sm + L.kh);
   float* qs = reinterpret_cast<float*>(sm + L.qs);
@@ -272,9 +285,27 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   int64_t* pg = reinterpret_cast<int64_t*>(sm + L.pg);
   const bool rot = A.theta > 0.0;
 
-  // W_up^K is stored transposed ([d_h][n_kept]); stage it as [n_kept][d_h]
+  // W_up^K (stored transposed, W[c][d] = wk[d * n_kept + c]) as B fragments of
+  // an m16n8k(G) MMA per (group j, n-tile of 8 dims): lane (gid, t4) register q
+  // holds rows c = jG + 2 t4 + 8 q + {0, 1} of column d = 8 n-tile + gid, as
+  // fp16 hi = rn(W) and lo = rn(W - hi); and the column sums of each group
   const float* wk = cd->w_up + sk.wup_off;
-  for (int e = tid; e < nkK * d_h; e += kRtThreads) Ws[(e % nkK) * d_h + e / nkK] = wk[e];
+  const int ngK = sk.n_groups;
+  for (int e = tid; e < ngK * n_nt * KQ * 32; e += kRtThreads) {
+    const int ln = e & 31, r = e >> 5, q = r % KQ, nt = (r / KQ) % n_nt, j = r / (KQ * n_nt);
+    const int d = 8 * nt + (ln >> 2), c = j * G + 2 * (ln & 3) + 8 * q;
+    const float w0 = wk[(size_t)d * nkK + c], w1 = wk[(size_t)d * nkK + c + 1];
+    const float h0 = __half2float(__float2half_rn(w0)), h1 = __half2float(__float2half_rn(w1));
+    uint32_t* dst = bf + ((j * n_nt + nt) * 2 * KQ + q) * 32 + ln;
+    dst[0] = pack_half2(w0, w1);
+    dst[KQ * 32] = pack_half2(w0 - h0, w1 - h1);
+  }
+  for (int e = tid; e < ngK * d_h; e += kRtThreads) {
+    const int j = e / d_h, d = e % d_h;
+    float acc = 0.f;
+    for (int k = 0; k < G; ++k) acc += wk[(size_t)d * nkK + j * G + k];
+    wsum[j * d_h + d] = acc;
+  }
   if (rot)
     for (int i = tid; i < half; i += kRtThreads) om[i] = pow(A.theta, -2.0 * i / d_h) / 3.141592653589793;
   if (tid < kMaxGQ) {
@@ -301,7 +332,7 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   const int per = (tiles + A.n_split - 1) / A.n_split;
   const int tok_begin = min(split * per, tiles) * kRtTokens;
   const int tok_end = min(min((split + 1) * per, tiles) * kRtTokens, len);
-  const int ngK = sk.n_groups, n_items = kRtTokens * (ngK + sv.n_groups);
+  const int n_items = kRtTokens * (ngK + sv.n_groups);
   const int n_acc = gq * nkV;
   float acc[kRtAccSlots];
 #pragma unroll
@@ -327,54 +358,85 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
       const int side = jj < ngK ? 0 : 1, j = side ? jj - ngK : jj;
       const GroupDev gd = (side ? sv : sk).grp[j];
       const int64_t off = pg[t];
-      float* dst = side == 0 ? cT + (j * G) * kRtTokens + t : cV + t * cvs + j * G;
-      const int stride = side == 0 ? kRtTokens : 1;
+      uint32_t code[G];
+      float sv_ = 0.f, zv = 0.f;
       if (off < 0) {
 #pragma unroll
-        for (int k = 0; k < G; ++k) dst[k * stride] = 0.f;
-        continue;
+        for (int k = 0; k < G; ++k) code[k] = 0u;
+      } else {
+        const uint8_t* page = A.pool + off;
+        const int tau = (t0 + t) % P, u = tau >> 1;
+        const uint32_t* blk = reinterpret_cast<const uint32_t*>(page + gd.plane_off + (tau / TB) * (32 * gd.b));
+        const uint2 rec =
+            __ldg(reinterpret_cast<const uint2*>(page + gd.sz_off + 8 * ((u & 7) * (P >> 4) + (u >> 3))));
+        sv_ = (tau & 1) ? half_hi(rec.x) : half_lo(rec.x);  // {s[2u], s[2u+1]}
+        zv = (tau & 1) ? half_hi(rec.y) : half_lo(rec.y);   // {z[2u], z[2u+1]}
+        if (side == 0)
+          unpack_token<G, 0>(blk, gd.b, tau % TB, code);
+        else
+          unpack_token<G, 1>(blk, gd.b, tau % TB, code);
       }
-      const uint8_t* page = A.pool + off;
-      const int tau = (t0 + t) % P, u = tau >> 1;
-      const uint32_t* blk = reinterpret_cast<const uint32_t*>(page + gd.plane_off + (tau / TB) * (32 * gd.b));
-      const uint2 rec = __ldg(reinterpret_cast<const uint2*>(page + gd.sz_off + 8 * ((u & 7) * (P >> 4) + (u >> 3))));
-      const uint32_t sw = rec.x, zw = rec.y;  // {s[2u], s[2u+1]}, {z[2u], z[2u+1]}
-      const float sv_ = (tau & 1) ? half_hi(sw) : half_lo(sw), zv = (tau & 1) ? half_hi(zw) : half_lo(zw);
-      if (side == 0)
-        dequant_token<G, 0>(blk, gd.b, tau % TB, sv_, zv, dst, stride);
-      else
-        dequant_token<G, 1>(blk, gd.b, tau % TB, sv_, zv, dst, stride);
+      if (side == 0) {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(ck + t * cks + j * G);
+#pragma unroll
+        for (int k = 0; k < G; k += 2) dst[k / 2] = pack_half2((float)code[k], (float)code[k + 1]);
+        szk[t * ngs + j] = sv_;
+        szk[(kRtTokens + t) * ngs + j] = zv;
+      } else {
+        float* dst = cV + t * cvs + j * G;
+#pragma unroll
+        for (int k = 0; k < G; ++k) dst[k] = fmaf((float)code[k], sv_, zv);
+      }
     }
     __syncthreads();
-    // ---- 2. k^ = c^_K W_up^K for 4 tokens x (4 dims + partners), rotated ----
-    for (int e = tid; e < (kRtTokens / 4) * (half / 4); e += kRtThreads) {
-      const int tq = e % (kRtTokens / 4), dq = e / (kRtTokens / 4);
-      float lo[4][4], hi[4][4];
+    // ---- 2. k^ = sum_j s_j (code_j W_j) + z_j (sum of W_j) on the tensor cores ----
+    {
+      const int gid = lane >> 2, t4 = lane & 3;
+      for (int pp = warp; pp < (kRtTokens / 16) * half_nt; pp += kRtThreads / 32) {
+        const int mt = pp % (kRtTokens / 16), np = pp / (kRtTokens / 16);
+        const int r0 = mt * 16 + gid, r1 = r0 + 8;
+        float acc[2][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+        for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-        for (int jn = 0; jn < 4; ++jn) lo[i][jn] = hi[i][jn] = 0.f;
-      for (int c = 0; c < nkK; ++c) {
-        const float4 cv = *reinterpret_cast<const float4*>(cT + c * kRtTokens + 4 * tq);
-        const float4 wl = *reinterpret_cast<const float4*>(Ws + c * d_h + 4 * dq);
-        const float4 wh = *reinterpret_cast<const float4*>(Ws + c * d_h + half + 4 * dq);
-        const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, wa[4] = {wl.x, wl.y, wl.z, wl.w},
-                    wb[4] = {wh.x, wh.y, wh.z, wh.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int jn = 0; jn < 4; ++jn) {
-            lo[i][jn] = fmaf(cc[i], wa[jn], lo[i][jn]);
-            hi[i][jn] = fmaf(cc[i], wb[jn], hi[i][jn]);
+          for (int r = 0; r < 4; ++r) acc[h2][r] = 0.f;
+        for (int j = 0; j < ngK; ++j) {
+          const __half* a0p = ck + r0 * cks + j * G + 2 * t4;
+          const __half* a1p = ck + r1 * cks + j * G + 2 * t4;
+          uint32_t af[4];
+          af[0] = *reinterpret_cast<const uint32_t*>(a0p);
+          af[1] = *reinterpret_cast<const uint32_t*>(a1p);
+          if (G == 16) {
+            af[2] = *reinterpret_cast<const uint32_t*>(a0p + 8);
+            af[3] = *reinterpret_cast<const uint32_t*>(a1p + 8);
           }
-      }
+          const float s0 = szk[r0 * ngs + j], s1 = szk[r1 * ngs + j];
+          const float z0 = szk[(kRtTokens + r0) * ngs + j], z1 = szk[(kRtTokens + r1) * ngs + j];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = 4 * tq + i;
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int nt = np + h2 * half_nt;
+            const uint32_t* bp = bf + (j * n_nt + nt) * 2 * KQ * 32 + lane;
+            float pr[4] = {0.f, 0.f, 0.f, 0.f};
+            if (G == 16) {
+              const uint32_t bh[2] = {bp[0], bp[32]}, bl[2] = {bp[64], bp[96]};
+              mma_m16n8k16(pr, af, bh);
+              mma_m16n8k16(pr, af, bl);
+            } else {
+              mma_m16n8k8(pr, af, bp[0]);
+              mma_m16n8k8(pr, af, bp[32]);
+            }
+            const float w0 = wsum[j * d_h + 8 * nt + 2 * t4], w1 = wsum[j * d_h + 8 * nt + 2 * t4 + 1];
+            acc[h2][0] = fmaf(s0, pr[0], fmaf(z0, w0, acc[h2][0]));
+            acc[h2][1] = fmaf(s0, pr[1], fmaf(z0, w1, acc[h2][1]));
+            acc[h2][2] = fmaf(s1, pr[2], fmaf(z1, w0, acc[h2][2]));
+            acc[h2][3] = fmaf(s1, pr[3], fmaf(z1, w1, acc[h2][3]));
+          }
+        }
+        // rows r0 / r1, dims d (n-tile np) and d + d_h/2 (n-tile np + half_nt)
 #pragma unroll
-        for (int jn = 0; jn < 4; ++jn) {
-          const int d = 4 * dq + jn;
-          float x = lo[i][jn], y = hi[i][jn];
+        for (int r = 0; r < 4; ++r) {
+          const int t = r < 2 ? r0 : r1, d = 8 * np + 2 * t4 + (r & 1);
+          float x = acc[0][r], y = acc[1][r];
           if (rot) rope_rotate(x, y, (double)(t0 + t) * om[d]);
           kh[t * (d_h + 1) + d] = x;
           kh[t * (d_h + 1) + half + d] = y;
@@ -527,14 +589,14 @@ RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq) {
   ns = (int)std::max<int64_t>(1, std::min<int64_t>({(int64_t)ns, (int64_t)kRtMaxSplit, max_tiles}));
   p.n_split = ns;
   p.part_stride = (2 + h.max_kept_v + 3) / 4 * 4;
-  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq).total;
+  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq, h.group).total;
   p.ws_bytes = ((size_t)batch * h.n_q * ns * p.part_stride * 4 + 255) / 256 * 256;
   return p;
 }
 
 bool rt_supported(const CodecDev& h, std::string* why) {
-  if (h.d_h > kRtMaxDHead || h.d_h % 8 != 0) {
-    *why = "reconstruct-then-attend needs d_head a multiple of 8 and at most 128";
+  if (h.d_h > kRtMaxDHead || h.d_h % 16 != 0) {
+    *why = "reconstruct-then-attend needs d_head a multiple of 16 and at most 128";
     return false;
   }
   if (h.max_kept_k > kRtMaxDHead || h.max_kept_v > kRtMaxDHead) {
