@@ -431,9 +431,11 @@ def run_gpu(args, rank, world):
         "clocks": clk,
     }
     if rt:
-        # the rebuild of the keys is fp32 FMA work on the CUDA cores: FLOPs per
-        # (token, KV head) = 2 n_kept_K d_h (lift) + 2 gq d_h (scores) + 2 gq n_kept_V
-        # (probability-weighted V latents), summed over the KV heads of a layer
+        # algorithmic FLOPs per (token, KV head) = 2 n_kept_K d_h (lift) + 2 gq d_h
+        # (scores) + 2 gq n_kept_V (probability-weighted V latents), summed over the
+        # KV heads of a layer; reported against the fp32 CUDA-core peak (the lift runs
+        # as fp16 hi/lo MMAs, but the per-tile unpacking, rotation, scores and sums,
+        # which bound the kernel, are CUDA-core work)
         widths = codecs[0].state()["widths"]
         gq = cfg.n_q_heads // cfg.n_kv_heads
         flop_tok = sum(2 * cfg.group * int((w[0] > 0).sum()) * cfg.d_head + 2 * gq * cfg.d_head
@@ -444,8 +446,8 @@ def run_gpu(args, rank, world):
         result["config"]["decode"] = f"reconstruct-then-attend, rotary base {args.rope_theta:g}"
         result["dtype"] = "u8 codes, fp16 scale/zero, fp32 lift and accumulate"
         result["roofline"] = {
-            "kernel": "rt_split_kernel (keys rebuilt per 64-token tile with fp32 FMAs, rotated, scored; V summed "
-                      "in the latent space), timed with its combine launch",
+            "kernel": "rt_split_kernel (keys rebuilt per 32-token tile on the tensor cores, rotated and scored "
+                      "with fp32 FMAs; V summed in the latent space), timed with its combine launch",
             "bound": "alu", "achieved": tflops, "peak": alu_peak, "unit": "TFLOP/s", "frac": tflops / alu_peak,
             "traffic": None,
             "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm)",

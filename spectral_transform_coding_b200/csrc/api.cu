@@ -656,7 +656,7 @@ spectra_status spectra_decode_reconstruct_workspace_bytes(const spectra_codec* c
                                                           size_t* bytes) {
   if (!c || !bytes || batch <= 0 || max_len < 0) return fail(SPECTRA_ERR_INVALID, "bad arguments");
   const int64_t pages = (max_len + c->h.P - 1) / c->h.P;
-  const RtPlan p = make_rt_plan(c->h, batch, (int)std::min<int64_t>(std::max<int64_t>(pages, 1), 1 << 30));
+  const RtPlan p = make_rt_plan(c->h, batch, (int)std::min<int64_t>(std::max<int64_t>(pages, 1), 1 << 30), true);
   *bytes = p.ws_bytes;
   return SPECTRA_OK;
 }

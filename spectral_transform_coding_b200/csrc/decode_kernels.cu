@@ -16,11 +16,11 @@
 // Three kernels per decode step, chained with programmatic dependent launch:
 //   fold    one CTA per (sequence, KV head): q_lat and its group sums, written
 //           as the split kernel's MMA B fragments;
-//   split   one CTA per (context split, KV head, sequence): prefetches its
-//           pages into L2 while the fold runs, then streams them (bulk copies
-//           into per-warp shared-memory stages) through an online softmax
-//           over 64-token chunks; one partial record (max, sum, latent
-//           accumulator) per q head;
+//   split   one CTA per (context split, KV head, sequence): streams its pages
+//           (bulk copies into per-warp shared-memory stages, the first ones
+//           issued while the fold runs) through an online softmax over
+//           64-token chunks; one partial record (max, sum, latent accumulator)
+//           per q head;
 //   combine one CTA per (q head, sequence): merges the splits, applies W_up^V
 //           (bulk-copied into shared memory while the splits finish).
 #include <cuda_fp16.h>
@@ -478,24 +478,40 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
     count_ = (p1_ - p0_ > warp) ? (p1_ - p0_ - warp + kDecWarps - 1) / kDecWarps : 0;
   };
 
-  // ---- 1. L2 warm-up of this warp's pages -----------------------------------
+  auto issue_page = [&](int pg, int i) {
+    const int pid = A.page_table[(size_t)b * A.max_pages + pg];
+    const uint8_t* src = A.pool + (size_t)pid * (size_t)A.page_bytes + sec_off;
+    uint64_t* bar = &bars[i % S];
+    mbar_arrive_expect_tx(bar, (uint32_t)sec_bytes);
+    bulk_copy_g2s(my_stages + (size_t)(i % S) * A.stage_bytes, src, (uint32_t)sec_bytes, bar);
+  };
+
+  // ---- 1. speculative first copies ------------------------------------------
   // Every kernel of the chain lets its successor start at its own start, so up
-  // to the dependency wait below the encode kernels of the same step may still
-  // be writing the lengths and the pages.  Here the length is only a hint for
-  // prefetches, which move bytes toward L2 and change nothing; the page table
-  // is written by no kernel.  Lengths and pages are read for real after the wait.
+  // to the dependency wait below an encode's commit kernel may still be
+  // advancing the length: the length read here is a hint.  The pages are
+  // final: each kernel that writes pages lets no successor start before its
+  // writes are complete (the commit kernel triggers only after its own wait on
+  // the fused encode; the quantise kernel does not trigger early), and the
+  // page table is written by no kernel.  The first copies go out for the
+  // hint's page range; after the wait they are kept if the final length gives
+  // this warp the same first pages, else drained and reissued.
+  int hp0 = 0, hcount = 0;
   {
     const int hint = A.lengths[b];
-    if (hint > 0 && (int64_t)hint <= (int64_t)A.max_pages * P) {
-      int hp0, hcount;
-      page_range(hint, hp0, hcount);
-      for (int i = lane; i < hcount; i += 32) {
-        const int pid = A.page_table[(size_t)b * A.max_pages + hp0 + warp + kDecWarps * i];
-        if (pid >= 0 && (int64_t)pid < A.n_pool_pages)
-          bulk_prefetch_l2(A.pool + (size_t)pid * (size_t)A.page_bytes + sec_off, (uint32_t)sec_bytes);
-      }
-    }
+    if (hint > 0 && (int64_t)hint <= (int64_t)A.max_pages * P) page_range(hint, hp0, hcount);
   }
+  int early = min(S, hcount);
+  {
+    bool hb = false;
+    if (lane < early) {
+      const int pid = A.page_table[(size_t)b * A.max_pages + hp0 + warp + kDecWarps * lane];
+      hb = pid < 0 || (int64_t)pid >= A.n_pool_pages;
+    }
+    if (__any_sync(0xffffffffu, hb)) early = 0;
+  }
+  if (lane == 0)
+    for (int i = 0; i < early; ++i) issue_page(hp0 + warp + kDecWarps * i, i);
 
   // group tables (built on the host with the page layout)
   {
@@ -524,17 +540,32 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   }
   const bool warp_bad = __any_sync(0xffffffffu, bad);
   if (warp_bad && lane == 0) device_error(cd->err, SPECTRA_ERR_INVALID);
-  const int my_count = warp_bad ? 0 : count;
-  auto issue = [&](int i) {
-    const int pg = p0 + warp + kDecWarps * i;
-    const int pid = A.page_table[(size_t)b * A.max_pages + pg];
-    const uint8_t* src = A.pool + (size_t)pid * (size_t)A.page_bytes + sec_off;
-    uint64_t* bar = &bars[i % S];
-    mbar_arrive_expect_tx(bar, (uint32_t)sec_bytes);
-    bulk_copy_g2s(my_stages + (size_t)(i % S) * A.stage_bytes, src, (uint32_t)sec_bytes, bar);
-  };
+  int my_count = warp_bad ? 0 : count;
+  // speculative copies: kept when they are this warp's first pages under the
+  // final length; else each is waited for (bounded) and its stage's first phase
+  // counted as used (off_mask), and the copies are reissued
+  uint32_t off_mask = 0u;
+  int issued = 0;
+  if (early > 0) {
+    if (p0 == hp0 && early <= my_count) {
+      issued = early;
+    } else {
+      bool drained = true;
+      if (lane == 0)
+        for (int i = 0; i < early; ++i) drained &= mbar_wait_bounded(&bars[i], 0u, kWaitLimitNs);
+      drained = __shfl_sync(0xffffffffu, drained, 0);
+      if (!drained) {
+        if (lane == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
+        my_count = 0;
+      }
+      off_mask = (1u << early) - 1u;
+    }
+  }
+  // parity of copy i's completion on its stage's barrier
+  auto parity = [&](int i) -> uint32_t { return (uint32_t)(((i / S) + ((off_mask >> (i % S)) & 1u)) & 1u); };
+  auto issue = [&](int i) { issue_page(p0 + warp + kDecWarps * i, i); };
   if (lane == 0)
-    for (int i = 0; i < min(S, my_count); ++i) issue(i);
+    for (int i = issued; i < min(S, my_count); ++i) issue(i);
 
   // ---- 3. the folded query (written by the fold grid) -----------------------
   {
@@ -581,7 +612,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   int i = 0;
   for (; i < my_count; ++i) {
     const int s = i % S;
-    const bool ok = mbar_wait_bounded(&bars[s], (uint32_t)((i / S) & 1), kWaitLimitNs);
+    const bool ok = mbar_wait_bounded(&bars[s], parity(i), kWaitLimitNs);
     if (!__all_sync(0xffffffffu, ok)) {
       timed_out = true;
       break;
@@ -761,7 +792,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
     if (lane == 0) {
       device_error(cd->err, SPECTRA_ERR_TIMEOUT);
       for (int k = i; k < min(i + S, my_count); ++k)  // let copies still in flight land
-        mbar_wait_bounded(&bars[k % S], (uint32_t)((k / S) & 1), kWaitLimitNs);
+        mbar_wait_bounded(&bars[k % S], parity(k), kWaitLimitNs);
     }
     __syncwarp();
   }

@@ -318,7 +318,9 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
   constexpr int TB = 256 / G;               // tokens per 256-bit block
   constexpr int LANES_PER_TOKENSET = TB;    // 16 or 32
   constexpr int GROUPS_PER_WARP = 32 / LANES_PER_TOKENSET;
-  pdl_launch_dependents();
+  // No early trigger: a decode launched next copies pages before its own
+  // dependency wait, so its kernels may start only once these writes are done
+  // (the implicit trigger at this grid's completion).
   pdl_wait();  // latents and the append plan come from the preceding kernels
   if (*ok_flag == 0) return;
   const int a = blockIdx.y >> 1, side = blockIdx.y & 1;
@@ -530,8 +532,11 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
 // Advances the lengths after a fused encode (same checks, so the same verdict).
 __global__ void __launch_bounds__(32) encode_commit_kernel(const int32_t* __restrict__ seq_ids, int T,
                                                            const spectra_cache cache, int P) {
-  pdl_launch_dependents();
   pdl_wait();  // the fused encode read the lengths before this point
+  // Triggered after the wait: the kernels after this one (a decode copies pages
+  // before its own dependency wait) start only once the fused encode's page
+  // writes are complete.
+  pdl_launch_dependents();
   const int t = threadIdx.x;
   int64_t pos = 0;
   const int err = t < T ? append_position(seq_ids, t, cache, P, &pos) : 0;

@@ -61,7 +61,8 @@ struct RtPlan {
   int smem_bytes;   // dynamic shared memory of the split kernel
   size_t ws_bytes;  // workspace: the partial records
 };
-RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq);
+// upper_bound: size for any call on any device (the workspace query)
+RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq, bool upper_bound = false);
 bool rt_supported(const CodecDev& h, std::string* why);
 cudaError_t launch_decode_reconstruct(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,
                                       const float* q, double theta, float* out, void* ws, const RtPlan& plan,

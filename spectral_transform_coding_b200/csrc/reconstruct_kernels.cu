@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(128) reconstruct_kernel(const CodecDev* __rest
 // probability-weighted latent sum, after the splits are merged.  R(p) turns the
 // pair (i, i + d_h/2) by p * theta^(-2i/d_h); theta = 0 means no rotation.
 //
-// One CTA per (KV head, sequence, context split), 256 threads, 64-token tiles:
+// One CTA per (KV head, sequence, context split), 256 threads, 32-token tiles:
 //   1. unpack the tile's K codes into shared memory as fp16 (exact: codes are
 //      integers below 256) with their per-group s and z, and dequantise the V
 //      latents (fp32);
@@ -147,12 +147,14 @@ __global__ void __launch_bounds__(128) reconstruct_kernel(const CodecDev* __rest
 //                           so P_j keeps about 22 bits; fp32 accumulate)
 //        k^ += s_j P_j + z_j (sum of the rows of W_j)
 //      in 16-token x 8-dim tiles, a warp holding a dim and its rotation
-//      partner d + d_h/2 in the same registers; then the rotation;
+//      partner d + d_h/2 in the same registers; then the rotation, the keys
+//      overwriting the consumed codes (two CTAs fit an SM at d_h = 128);
 //   3. scores of the KV head's q heads, online softmax (exp2 domain), and the
 //      probability-weighted sum of the V latents in registers.
 // A combine kernel merges the splits and applies W_up^V.
 // ---------------------------------------------------------------------------
-constexpr int kRtTokens = 64;
+constexpr int kRtTokens = 32;
+constexpr int kRtPairsPerWarp = 2;  // (16-token, 8-dim pair) MMA tiles per warp and tile: d_h <= 128
 constexpr int kRtThreads = 256;
 constexpr int kRtMaxSplit = 64;
 constexpr int kRtAccSlots = kMaxGQ * kRtMaxDHead / kRtThreads;  // V accumulators per thread
@@ -172,14 +174,17 @@ struct RtSmem {
     o += max_k * d_h * 4;
     ws = o;  // per group, the sum of its rows of W_up^K [group][d_h]
     o += n_grp * d_h * 4;
-    ck = o;  // K codes, fp16 [kRtTokens][ck_stride]
-    o += kRtTokens * ck_stride * 2;
-    sz = o;  // K scale and zero, fp32 [2][kRtTokens][n_grp]
-    o += 2 * kRtTokens * n_grp * 4;
+    // K codes, fp16 [kRtTokens][ck_stride], then K scale and zero, fp32
+    // [2][kRtTokens][n_grp]; once the lift has read them, the same bytes hold
+    // the rotated keys [kRtTokens][d_h + 1]
+    ck = o;
+    sz = ck + (kRtTokens * ck_stride * 2 + 15) / 16 * 16;
+    const int lift_in = sz - ck + 2 * kRtTokens * n_grp * 4;
+    const int keys = kRtTokens * (d_h + 1) * 4;
+    kh = ck;
+    o += ((lift_in > keys ? lift_in : keys) + 15) / 16 * 16;
     cv = o;  // V latents [kRtTokens][max_v + 1]
     o += (kRtTokens * (max_v + 1) * 4 + 15) / 16 * 16;
-    kh = o;  // rotated keys [kRtTokens][d_h + 1]
-    o += (kRtTokens * (d_h + 1) * 4 + 15) / 16 * 16;
     qs = o;  // rotated, scaled queries [gq][d_h]
     o += gq * d_h * 4;
     sc = o;  // scores, then probabilities [gq][kRtTokens]
@@ -278,7 +283,7 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   __half* ck = reinterpret_cast<__half*>(sm + L.ck);
   float* szk = reinterpret_cast<float*>(sm + L.sz);  // [0]: s, [kRtTokens * ngs]: z
   float* cV = reinterpret_cast<float*>(sm + L.cv);
-  float* kh = reinterpret_cast<float*>(sm + L.kh);
+  float* kh = reinterpret_cast<float*>(sm + L.kh);  // shares its bytes with ck and szk
   float* qs = reinterpret_cast<float*>(sm + L.qs);
   float* sc = reinterpret_cast<float*>(sm + L.sc);
   float* ml = reinterpret_cast<float*>(sm + L.ml);  // [0, 8) max, [8, 16) sum, [16, 24) correction
@@ -392,54 +397,70 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
     // ---- 2. k^ = sum_j s_j (code_j W_j) + z_j (sum of W_j) on the tensor cores ----
     {
       const int gid = lane >> 2, t4 = lane & 3;
-      for (int pp = warp; pp < (kRtTokens / 16) * half_nt; pp += kRtThreads / 32) {
-        const int mt = pp % (kRtTokens / 16), np = pp / (kRtTokens / 16);
-        const int r0 = mt * 16 + gid, r1 = r0 + 8;
-        float acc[2][4];
+      constexpr int kMT = kRtTokens / 16;
+      float acc[kRtPairsPerWarp][2][4];
+#pragma unroll
+      for (int w = 0; w < kRtPairsPerWarp; ++w)
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-          for (int r = 0; r < 4; ++r) acc[h2][r] = 0.f;
-        for (int j = 0; j < ngK; ++j) {
-          const __half* a0p = ck + r0 * cks + j * G + 2 * t4;
-          const __half* a1p = ck + r1 * cks + j * G + 2 * t4;
-          uint32_t af[4];
-          af[0] = *reinterpret_cast<const uint32_t*>(a0p);
-          af[1] = *reinterpret_cast<const uint32_t*>(a1p);
-          if (G == 16) {
-            af[2] = *reinterpret_cast<const uint32_t*>(a0p + 8);
-            af[3] = *reinterpret_cast<const uint32_t*>(a1p + 8);
-          }
-          const float s0 = szk[r0 * ngs + j], s1 = szk[r1 * ngs + j];
-          const float z0 = szk[(kRtTokens + r0) * ngs + j], z1 = szk[(kRtTokens + r1) * ngs + j];
+          for (int r = 0; r < 4; ++r) acc[w][h2][r] = 0.f;
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int nt = np + h2 * half_nt;
-            const uint32_t* bp = bf + (j * n_nt + nt) * 2 * KQ * 32 + lane;
-            float pr[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int w = 0; w < kRtPairsPerWarp; ++w) {
+        const int pp = warp + w * (kRtThreads / 32);
+        if (pp < kMT * half_nt) {  // warp-uniform
+          const int mt = pp % kMT, np = pp / kMT;
+          const int r0 = mt * 16 + gid, r1 = r0 + 8;
+          for (int j = 0; j < ngK; ++j) {
+            const __half* a0p = ck + r0 * cks + j * G + 2 * t4;
+            const __half* a1p = ck + r1 * cks + j * G + 2 * t4;
+            uint32_t af[4];
+            af[0] = *reinterpret_cast<const uint32_t*>(a0p);
+            af[1] = *reinterpret_cast<const uint32_t*>(a1p);
             if (G == 16) {
-              const uint32_t bh[2] = {bp[0], bp[32]}, bl[2] = {bp[64], bp[96]};
-              mma_m16n8k16(pr, af, bh);
-              mma_m16n8k16(pr, af, bl);
-            } else {
-              mma_m16n8k8(pr, af, bp[0]);
-              mma_m16n8k8(pr, af, bp[32]);
+              af[2] = *reinterpret_cast<const uint32_t*>(a0p + 8);
+              af[3] = *reinterpret_cast<const uint32_t*>(a1p + 8);
             }
-            const float w0 = wsum[j * d_h + 8 * nt + 2 * t4], w1 = wsum[j * d_h + 8 * nt + 2 * t4 + 1];
-            acc[h2][0] = fmaf(s0, pr[0], fmaf(z0, w0, acc[h2][0]));
-            acc[h2][1] = fmaf(s0, pr[1], fmaf(z0, w1, acc[h2][1]));
-            acc[h2][2] = fmaf(s1, pr[2], fmaf(z1, w0, acc[h2][2]));
-            acc[h2][3] = fmaf(s1, pr[3], fmaf(z1, w1, acc[h2][3]));
+            const float s0 = szk[r0 * ngs + j], s1 = szk[r1 * ngs + j];
+            const float z0 = szk[(kRtTokens + r0) * ngs + j], z1 = szk[(kRtTokens + r1) * ngs + j];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int ntl = np + h2 * half_nt;
+              const uint32_t* bp = bf + (j * n_nt + ntl) * 2 * KQ * 32 + lane;
+              float pr[4] = {0.f, 0.f, 0.f, 0.f};
+              if (G == 16) {
+                const uint32_t bh[2] = {bp[0], bp[32]}, bl[2] = {bp[64], bp[96]};
+                mma_m16n8k16(pr, af, bh);
+                mma_m16n8k16(pr, af, bl);
+              } else {
+                mma_m16n8k8(pr, af, bp[0]);
+                mma_m16n8k8(pr, af, bp[32]);
+              }
+              const float w0 = wsum[j * d_h + 8 * ntl + 2 * t4], w1 = wsum[j * d_h + 8 * ntl + 2 * t4 + 1];
+              acc[w][h2][0] = fmaf(s0, pr[0], fmaf(z0, w0, acc[w][h2][0]));
+              acc[w][h2][1] = fmaf(s0, pr[1], fmaf(z0, w1, acc[w][h2][1]));
+              acc[w][h2][2] = fmaf(s1, pr[2], fmaf(z1, w0, acc[w][h2][2]));
+              acc[w][h2][3] = fmaf(s1, pr[3], fmaf(z1, w1, acc[w][h2][3]));
+            }
           }
         }
-        // rows r0 / r1, dims d (n-tile np) and d + d_h/2 (n-tile np + half_nt)
+      }
+      __syncthreads();  // the codes are consumed: their bytes now take the keys
+      // rows r0 / r1, dims d (n-tile np) and d + d_h/2 (n-tile np + half_nt)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int t = r < 2 ? r0 : r1, d = 8 * np + 2 * t4 + (r & 1);
-          float x = acc[0][r], y = acc[1][r];
-          if (rot) rope_rotate(x, y, (double)(t0 + t) * om[d]);
-          kh[t * (d_h + 1) + d] = x;
-          kh[t * (d_h + 1) + half + d] = y;
+      for (int w = 0; w < kRtPairsPerWarp; ++w) {
+        const int pp = warp + w * (kRtThreads / 32);
+        if (pp < kMT * half_nt) {
+          const int mt = pp % kMT, np = pp / kMT;
+          const int r0 = mt * 16 + gid, r1 = r0 + 8;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int t = r < 2 ? r0 : r1, d = 8 * np + 2 * t4 + (r & 1);
+            float x = acc[w][0][r], y = acc[w][1][r];
+            if (rot) rope_rotate(x, y, (double)(t0 + t) * om[d]);
+            kh[t * (d_h + 1) + d] = x;
+            kh[t * (d_h + 1) + half + d] = y;
+          }
         }
       }
     }
@@ -577,19 +598,32 @@ int rt_sm_count() {
   return n;
 }
 
+// Resident split CTAs per SM at `smem` bytes of dynamic shared memory.
+int rt_ctas_per_sm(int group, int smem) {
+  const void* kern = group == 16 ? reinterpret_cast<const void*>(rt_split_kernel<16>)
+                                 : reinterpret_cast<const void*>(rt_split_kernel<8>);
+  int n = 0;
+  if (ensure_dynamic_smem(kern, smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kRtThreads, smem) != cudaSuccess || n <= 0)
+    n = 1;
+  return n;
+}
+
 }  // namespace
 
-RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq) {
+RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq, bool upper_bound) {
   RtPlan p{};
   const int64_t max_tiles = ((int64_t)max_pages_per_seq * h.P + kRtTokens - 1) / kRtTokens;
-  // one CTA per SM fits (about 170 KB of shared memory at d_h = 128): split the
-  // context so that the (KV head, sequence) pairs fill the SMs once
+  // split the context so that the (KV head, sequence) pairs fill the resident
+  // CTA slots once (two CTAs per SM fit at d_h = 128: about 106 KB each; more
+  // are not used, so that the bound below holds for any call)
+  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq, h.group).total;
   const int pairs = h.n_kv * batch;
-  int ns = rt_sm_count() / pairs;  // one wave: (KV head, sequence) pairs x splits <= SMs
+  const int per_sm = upper_bound ? 2 : std::min(2, rt_ctas_per_sm(h.group, p.smem_bytes));
+  int ns = rt_sm_count() * per_sm / pairs;
   ns = (int)std::max<int64_t>(1, std::min<int64_t>({(int64_t)ns, (int64_t)kRtMaxSplit, max_tiles}));
   p.n_split = ns;
   p.part_stride = (2 + h.max_kept_v + 3) / 4 * 4;
-  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq, h.group).total;
   p.ws_bytes = ((size_t)batch * h.n_q * ns * p.part_stride * 4 + 255) / 256 * 256;
   return p;
 }
