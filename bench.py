@@ -67,7 +67,14 @@ def _workload_name(cfg, layers):
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same workload)
 # ---------------------------------------------------------------------------
-TRAFFIC_PER_ALGO_BYTE = {"llama": 33_707_520 / (32_772 * 1024)}
+# DRAM bytes (read + write) per algorithmic byte of one launch of a kernel, from
+# one ncu capture of the current kernel on a 1-layer case of the workload; a
+# workload/kernel without a capture of its current code reports traffic null.
+#   latent split_kernel: none (its prologue changed after the last capture)
+#   rt_split_kernel, Llama-shaped, 32k context: 34,214,912 B read, 0 written,
+#     for 33,560,576 packed bytes
+TRAFFIC_PER_ALGO_BYTE = {}
+TRAFFIC_PER_PACKED_BYTE_RT = {"llama": 34_214_912 / 33_560_576}
 
 
 def _oracle_decode_case(cfg, n_tok=8192, rope_theta=None):
@@ -449,7 +456,8 @@ def run_gpu(args, rank, world):
             "kernel": "rt_split_kernel (keys rebuilt per 32-token tile on the tensor cores, rotated and scored "
                       "with fp32 FMAs; V summed in the latent space), timed with its combine launch",
             "bound": "alu", "achieved": tflops, "peak": alu_peak, "unit": "TFLOP/s", "frac": tflops / alu_peak,
-            "traffic": None,
+            "traffic": (TRAFFIC_PER_PACKED_BYTE_RT[args.workload] * dec_bytes
+                        if args.workload in TRAFFIC_PER_PACKED_BYTE_RT else None),
             "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm)",
             "avg_launch_us": dec_avg_ms * 1e3, "algorithmic_flops_per_launch": flops,
             "packed_bytes_per_launch": dec_bytes,
