@@ -140,3 +140,48 @@ def test_rope_pair_rotation_by_hand():
     y = oracle.rope(x, np.array([np.pi / 2]), 100.0)
     a2 = np.pi / 20
     np.testing.assert_allclose(y[0], [0.0, -2 * np.sin(a2), 1.0, 2 * np.cos(a2)], atol=1e-15)
+
+
+def test_rope_decode_without_rotation_equals_latent_route(toy_cfg, toy_codec):
+    """theta = 0: reconstruct-then-attend is the same function as the pinned
+    latent-space reference on the same pool."""
+    pool, lay, table, lengths, h, lat, widths = _toy_cache(toy_cfg, toy_codec, 150)
+    q = make_queries(toy_cfg, 1)
+    W_up = [[toy_codec["heads"][0]["K"]["W_up"], toy_codec["heads"][0]["V"]["W_up"]]]
+    a = oracle.decode_reference(pool, lay["page_bytes"], lay, toy_cfg.group, 64, table, lengths, q, W_up,
+                                toy_cfg.n_q_heads, 1)
+    b = oracle.decode_reference_rope(pool, lay["page_bytes"], lay, toy_cfg.group, 64, table, lengths, q, W_up,
+                                     toy_cfg.n_q_heads, 1, 0.0)
+    np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-13)
+
+
+def test_rope_decode_equals_rotation_matrices(toy_cfg, toy_codec):
+    """With rotation: the same attention written with explicit d x d rotation
+    matrices R(p) (pair (i, i + d/2) turned by p * theta^(-2i/d)), keys at
+    positions 0..n-1, the query at n-1."""
+    n, theta = 130, 50.0
+    pool, lay, table, lengths, h, lat, widths = _toy_cache(toy_cfg, toy_codec, n)
+    q = make_queries(toy_cfg, 1)
+    W_up = [[toy_codec["heads"][0]["K"]["W_up"], toy_codec["heads"][0]["V"]["W_up"]]]
+    out = oracle.decode_reference_rope(pool, lay["page_bytes"], lay, toy_cfg.group, 64, table, lengths, q, W_up,
+                                       toy_cfg.n_q_heads, 1, theta)
+    cK = oracle.read_side(pool, lay["page_bytes"], lay, toy_cfg.group, 64, table[0], n, 0, 0)
+    cV = oracle.read_side(pool, lay["page_bytes"], lay, toy_cfg.group, 64, table[0], n, 0, 1)
+    K, V = cK @ W_up[0][0], cV @ W_up[0][1]
+    d = K.shape[1]
+    hd = d // 2
+
+    def R(p):
+        m = np.zeros((d, d))
+        for i in range(hd):
+            a = p * theta ** (-2.0 * i / d)
+            m[i, i], m[i, i + hd] = math.cos(a), -math.sin(a)
+            m[i + hd, i], m[i + hd, i + hd] = math.sin(a), math.cos(a)
+        return m
+
+    Kr = np.stack([R(t) @ K[t] for t in range(n)])
+    for hq in range(toy_cfg.n_q_heads):
+        qr = R(n - 1) @ q[0, hq].astype(np.float64)
+        s = Kr @ qr / math.sqrt(d)
+        e = np.exp(s - s.max())
+        np.testing.assert_allclose(out[0, hq], (e / e.sum()) @ V, rtol=1e-11, atol=1e-12)
