@@ -146,11 +146,12 @@ def cpu_oracle_sample(cfg, target_s=12.0, rope_theta=None):
     return value, _blas_threads(), _sample_text(cfg, n_tok, what)
 
 
-def cpu_oracle_steps(cfg, steps, warm, budget_s=120.0):
+def cpu_oracle_steps(cfg, steps, warm, budget_s=120.0, rope_theta=None):
     """The oracle as the reference arm: ``warm`` untimed and ``steps`` timed steps,
     each the decode of one KV head over a context sample sized so that the whole
-    run takes about ``budget_s`` seconds."""
-    run, n_max = _oracle_decode_case(cfg)
+    run takes about ``budget_s`` seconds (rope_theta: reconstruct-then-attend with
+    that rotary base, else the latent decode's reference)."""
+    run, n_max = _oracle_decode_case(cfg, rope_theta=rope_theta)
     P = cfg.page_tokens
     t0 = time.perf_counter()
     run(n_max)
@@ -165,7 +166,10 @@ def cpu_oracle_steps(cfg, steps, warm, budget_s=120.0):
         run(n_tok)
     el = time.perf_counter() - t0
     value = steps * n_tok / el
-    return value, el / steps * 1e3, _blas_threads(), _sample_text(cfg, n_tok, f"{steps} timed steps in {el:.1f} s")
+    what = f"{steps} timed steps in {el:.1f} s"
+    if rope_theta is not None:
+        what += f", reconstruct-then-attend with rotary base {rope_theta:g}"
+    return value, el / steps * 1e3, _blas_threads(), _sample_text(cfg, n_tok, what)
 
 
 # ---------------------------------------------------------------------------
@@ -598,14 +602,18 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        value, ms, cores, sample = cpu_oracle_steps(cfg, args.steps, args.warmup)
+        rt = args.decode == "reconstruct"
+        value, ms, cores, sample = cpu_oracle_steps(cfg, args.steps, args.warmup,
+                                                    rope_theta=args.rope_theta if rt else None)
         L = args.layers or MODEL_LAYERS[args.workload]
         out = {
             "impl": "reference", "metric": "latent-KV decode attention: cache tokens/s/head", "value": value,
             "unit": "tokens/s/head", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": _workload_name(cfg, L)},
+            "data": "synthetic",
+            "config": dict({"workload": _workload_name(cfg, L)},
+                           **({"decode": f"reconstruct-then-attend, rotary base {args.rope_theta:g}"} if rt else {})),
             "cpu_baseline": {"value": value, "unit": "tokens/s/head", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s/head", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

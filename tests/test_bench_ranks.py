@@ -68,3 +68,15 @@ def test_reference_arm_runs_on_rank_zero_only():
     r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_times_the_rotating_oracle_in_reconstruct_mode():
+    """bench.py --impl reference --decode reconstruct times the oracle's
+    reconstruct-then-attend (with the rotary base) on a bounded sample."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    from workloads import get_config
+    value, ms, cores, sample = bench.cpu_oracle_steps(get_config("llama"), 1, 0, budget_s=1.0, rope_theta=500000.0)
+    assert value > 0 and ms > 0 and cores >= 1
+    assert "rotary base 500000" in sample
