@@ -498,7 +498,9 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   // this warp the same first pages, else drained and reissued.
   int hp0 = 0, hcount = 0;
   {
-    const int hint = A.lengths[b];
+    // L2-only loads here and after the wait: the first read must not leave an
+    // L1 line that the second one could hit
+    const int hint = __ldcg(A.lengths + b);
     if (hint > 0 && (int64_t)hint <= (int64_t)A.max_pages * P) page_range(hint, hp0, hcount);
   }
   int early = min(S, hcount);
@@ -526,7 +528,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) split_kernel(const DecodeArgs 
   // (the wait covers the fold grid, which waits before it exits, and so every
   // earlier kernel of the stream)
   pdl_wait();
-  int len = A.lengths[b];
+  int len = __ldcg(A.lengths + b);
   if (len < 0 || (int64_t)len > (int64_t)A.max_pages * P) {  // lengths written outside the library
     if (tid == 0) device_error(cd->err, SPECTRA_ERR_INVALID);
     len = 0;
