@@ -278,7 +278,12 @@ SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, con
  * masking beyond lengths[b].
  *   q   device fp32 [batch][n_q_heads][d_head]
  *   out device fp32 [batch][n_q_heads][d_head] (attention output before W_O)
- *   workspace device, >= spectra_decode_workspace_bytes, 256-byte aligned. */
+ *   workspace device, >= spectra_decode_workspace_bytes, 256-byte aligned.
+ * A length outside [0, max_pages_per_seq * page_tokens] (that sequence is then
+ * read as empty) or a page id outside [0, n_pages) (that warp's pages are
+ * skipped) records SPECTRA_ERR_INVALID in the device error word.  The cache may
+ * come straight from spectra_encode_append or spectra_quantize_append on the
+ * same stream, with no synchronisation in between. */
 SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, const spectra_cache* cache,
                                      const float* q, float* out, void* workspace,
                                      size_t workspace_bytes, void* stream);
@@ -334,8 +339,9 @@ SPECTRA_API spectra_status spectra_decode_reconstruct_workspace_bytes(const spec
  *   out device fp32 [batch][n_q_heads][d_head]; a sequence of length 0 gives 0
  *   workspace device, >= spectra_decode_reconstruct_workspace_bytes, 256-byte aligned.
  * Needs d_head a multiple of 16 and <= 128, <= 128 kept coordinates per side and
- * <= 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED).  A page id outside
- * [0, n_pages) or a length outside [0, max_pages_per_seq * page_tokens) records
+ * <= 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED).  rope_theta must be
+ * 0 or a finite value above 1 (else SPECTRA_ERR_INVALID).  A page id outside
+ * [0, n_pages) or a length outside [0, max_pages_per_seq * page_tokens] records
  * SPECTRA_ERR_INVALID in the device error word (that part reads as zero). */
 SPECTRA_API spectra_status spectra_decode_attend_reconstruct(const spectra_codec* codec, const spectra_cache* cache,
                                                              const float* q, double rope_theta, float* out,
