@@ -18,7 +18,7 @@ Sources (cited by page title and section):
   Thomas, Elements of Information Theory, ch. 10): D_i = min(theta, s_i^2),
   R_i = max(0, 1/2 log2(s_i^2/theta)).
 
-Readings of points the pages leave open (each listed in the design doc):
+Readings of points the pages leave open:
 
 * G is the mean E[h^T h]; the Gram's scale leaves the basis unchanged.
 * A latent coordinate's "variance" is its second moment s_i^2 (G is uncentred).

@@ -495,7 +495,7 @@ spectra_status spectra_wo_correction(const spectra_codec* c, int32_t dtype, cons
   };
   DevBuf buf;
   const size_t szQ = (size_t)n * nq * dh, szKV = (size_t)n * nkv * dh;
-  const size_t total = (szQ + 4 * szKV + 2 * (size_t)n * dh + 3 * (size_t)dh * dh) * 4 + 4096;
+  const size_t total = (szQ + 4 * szKV + 2 * (size_t)n * dh + (size_t)dh * dh) * 4 + 4096;
   CUDA_TRY(cudaMalloc(&buf.p, total));
   float* Q = static_cast<float*>(buf.p);
   float* K = Q + szQ;
@@ -505,7 +505,6 @@ spectra_status spectra_wo_correction(const spectra_codec* c, int32_t dtype, cons
   float* O = Vl + szKV;    // [n][dh]
   float* Ol = O + (size_t)n * dh;
   float* Pm = Ol + (size_t)n * dh;
-  float* AB = Pm + (size_t)dh * dh;
   CUDA_TRY(launch_gemm_nn_f32(H, bf, dm, W_Q, bf, nq * dh, Q, nq * dh, n, nq * dh, dm, st));
   CUDA_TRY(launch_gemm_nn_f32(H, bf, dm, W_K, bf, nkv * dh, K, nkv * dh, n, nkv * dh, dm, st));
   CUDA_TRY(launch_gemm_nn_f32(H, bf, dm, W_V, bf, nkv * dh, V, nkv * dh, n, nkv * dh, dm, st));
@@ -532,7 +531,7 @@ spectra_status spectra_wo_correction(const spectra_codec* c, int32_t dtype, cons
     }
     CUDA_TRY(cudaStreamSynchronize(st));  // host buffers are reused for the next head
   }
-  std::vector<float> Ah((size_t)dh * dh), Bh((size_t)dh * dh), Ms((size_t)dh * dh);
+  std::vector<float> Lh((size_t)n * dh), Oh((size_t)n * dh), Ms((size_t)dh * dh);
   for (int h = 0; h < nq; ++h) {
     const int a = h / gq, kv = keptV[a];
     std::fill(Ms.begin(), Ms.end(), 0.f);
@@ -542,17 +541,24 @@ spectra_status spectra_wo_correction(const spectra_codec* c, int32_t dtype, cons
                                        nkv * dh, nkv * dh, dh, st));
       CUDA_TRY(launch_causal_attention(Qh, Kt + (size_t)a * dh, Vl + (size_t)a * dh, Ol, n, dh, kv, nq * dh,
                                        nkv * dh, nkv * dh, kv, st));
-      CUDA_TRY(launch_gemm_tn_f32(Ol, false, kv, Ol, false, kv, AB, kv, kv, kv, n, st));
-      CUDA_TRY(launch_gemm_tn_f32(Ol, false, kv, O, false, dh, AB + (size_t)dh * dh, dh, kv, dh, n, st));
-      CUDA_TRY(cudaMemcpyAsync(Ah.data(), AB, (size_t)kv * kv * 4, cudaMemcpyDeviceToHost, st));
-      CUDA_TRY(cudaMemcpyAsync(Bh.data(), AB + (size_t)dh * dh, (size_t)kv * dh * 4, cudaMemcpyDeviceToHost, st));
+      CUDA_TRY(cudaMemcpyAsync(Lh.data(), Ol, (size_t)n * kv * 4, cudaMemcpyDeviceToHost, st));
+      CUDA_TRY(cudaMemcpyAsync(Oh.data(), O, (size_t)n * dh * 4, cudaMemcpyDeviceToHost, st));
       CUDA_TRY(cudaStreamSynchronize(st));
-      std::vector<double> A2((size_t)kv * kv), B2((size_t)kv * dh);
+      // normal equations formed in fp64 from the fp32 attention outputs: the
+      // solve then loses about cond(L) (not cond(L)^2) digits of the fp32 inputs
+      std::vector<double> A2((size_t)kv * kv, 0.0), B2((size_t)kv * dh, 0.0);
+      for (int t = 0; t < n; ++t) {
+        const float* lr = Lh.data() + (size_t)t * kv;
+        const float* orow = Oh.data() + (size_t)t * dh;
+        for (int i = 0; i < kv; ++i) {
+          const double li = lr[i];
+          for (int j = 0; j < kv; ++j) A2[(size_t)i * kv + j] += li * lr[j];
+          for (int j = 0; j < dh; ++j) B2[(size_t)i * dh + j] += li * orow[j];
+        }
+      }
       double tr = 0.0;
-      for (int i = 0; i < kv; ++i) tr += Ah[(size_t)i * kv + i];
+      for (int i = 0; i < kv; ++i) tr += A2[(size_t)i * kv + i];
       const double eps = 1e-8 * tr / kv;
-      for (size_t i = 0; i < A2.size(); ++i) A2[i] = Ah[i];
-      for (size_t i = 0; i < B2.size(); ++i) B2[i] = Bh[i];
       for (int i = 0; i < kv; ++i) A2[(size_t)i * kv + i] += eps;
       if (!solve_dense(A2, B2, kv, dh)) return fail(SPECTRA_ERR_NUMERIC, "singular W_O correction system");
       // M = U M'  (dh x dh)

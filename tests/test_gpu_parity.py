@@ -289,7 +289,25 @@ def test_wo_correction_matches_oracle():
     ref = oracle.wo_correction(layer["H_calib"], layer["W_Q"], layer["W_K"], layer["W_V"], layer["W_O"],
                                ref_codec, 2, 1, 16)
     err = np.abs(W_Op - ref["W_O"]).max() / np.abs(ref["W_O"]).max()
-    assert err < 2e-2, err
+    # Bar: the library's attention outputs L (truncated, latent) and O (exact)
+    # are fp32 (rounding u = 2^-24 per operation, d_model- and n-term sums); the
+    # normal equations are then formed and solved in fp64, so the map inherits
+    # the inputs' relative error amplified by about cond(L).  The bar allows 16
+    # fp32 roundings of L and O per element times cond(L), and never less than
+    # 1e-4.
+    H64 = layer["H_calib"].astype(np.float64)
+    conds = []
+    for h in range(2):
+        q = H64 @ layer["W_Q"][:, h * 16:(h + 1) * 16]
+        tr = []
+        for side, W in (("K", layer["W_K"]), ("V", layer["W_V"])):
+            hs = ref_codec["heads"][0][side]
+            Vr = hs["V"][:, hs["keep"]]
+            tr.append((H64 @ W[:, :16]) @ Vr @ (Vr.T if side == "K" else np.eye(Vr.shape[1])))
+        conds.append(np.linalg.cond(oracle.causal_attention(q, tr[0], tr[1])))
+    bar = max(1e-4, 16 * 2.0 ** -24 * max(conds))
+    print(f"W_O correction: err {err:.3e}, cond(L) {max(conds):.3e}, bar {bar:.3e}")
+    assert err <= bar, (err, bar)
 
 
 # --- fused encode of decode steps (T <= 16) ---------------------------------------
