@@ -275,15 +275,24 @@ SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, con
  * the cache, in the latent space: q_lat = q W_up^K^T, scores against the
  * dequantised latent keys of all lengths[b] tokens, exact (online) softmax,
  * sum_t p_t c_V,t, then W_up^V once per head.  Split-K over the context; no
- * masking beyond lengths[b].
+ * masking beyond lengths[b].  One kernel launch; the split-K partition and the
+ * merge order depend only on the lengths, so the result is deterministic.
  *   q   device fp32 [batch][n_q_heads][d_head]
  *   out device fp32 [batch][n_q_heads][d_head] (attention output before W_O)
- *   workspace device, >= spectra_decode_workspace_bytes, 256-byte aligned.
+ *   workspace device, >= spectra_decode_workspace_bytes, 256-byte aligned.  It
+ *       holds the split-K records and per-(sequence, KV head) arrival counters
+ *       that must be zero when a call starts: zero the workspace once before
+ *       its first use; every call leaves the counters at zero again.  Calls
+ *       that share a workspace must not overlap on the GPU.
+ * q must not be written by a kernel of this library still running in the
+ * same stream (q is read before the dependency on earlier launches resolves).
  * A length outside [0, max_pages_per_seq * page_tokens] (that sequence is then
- * read as empty) or a page id outside [0, n_pages) (that warp's pages are
- * skipped) records SPECTRA_ERR_INVALID in the device error word.  The cache may
- * come straight from spectra_encode_append or spectra_quantize_append on the
- * same stream, with no synchronisation in between. */
+ * read as empty) or a page id outside [0, n_pages) (that context split's pages
+ * are skipped) records SPECTRA_ERR_INVALID in the device error word.  The cache
+ * may come straight from spectra_encode_append or spectra_quantize_append on
+ * the same stream, with no synchronisation in between.  Needs d_head a
+ * multiple of 16 and at most 256, at most 8 kept groups per head and side and
+ * at most 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED). */
 SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, const spectra_cache* cache,
                                      const float* q, float* out, void* workspace,
                                      size_t workspace_bytes, void* stream);
@@ -294,13 +303,15 @@ SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, con
  * belongs to another framework, code running where an allocation would stall
  * or be refused).  No counterpart on the SPECTRA pages: an interface of this
  * library only.  Arguments as for spectra_decode_attend minus the workspace.
- * The scratch (folded queries, split-K partials) lives in one static 4 MiB
+ * The scratch (split-K records and arrival counters) lives in one static 4 MiB
  * device array per GPU, kept until the process exits.  The first call on a
  * device looks up that array's device address (cudaGetSymbolAddress), so make
  * the first call on each device before any stream capture.  Every call shares
- * the array and leaves its contents behind; nothing in it needs to start at
- * zero.  Calls whose kernels can overlap on the GPU (other streams, other
- * codecs at the same time) race on the array: serialise them.  A batch/context
+ * the array and leaves its contents behind: the counters, which must start at
+ * zero, are zero when the library loads and every completed call leaves them
+ * at zero; the records are rewritten by each call before they are read.
+ * Calls whose kernels can overlap on the GPU (other streams, other codecs at
+ * the same time) race on the array: serialise them.  A batch/context
  * whose scratch would exceed 4 MiB fails with SPECTRA_ERR_CAPACITY.  Calls no
  * cudaMalloc, cudaFree or allocating library routine. */
 SPECTRA_API spectra_status spectra_decode_attend_noalloc(const spectra_codec* codec,

@@ -17,6 +17,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -48,7 +49,7 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) 
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
     hdr_time = _newest_header()
-    objs = []
+    objs, cmds = [], []
     for src in srcs:
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         objs.append(obj)
@@ -59,7 +60,13 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) 
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
+    # translation units compile in parallel (the decode kernel's variants are
+    # split over several units for this)
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for r in pool.map(lambda c: subprocess.run(c), cmds):
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
         cmd = [nvcc, *ARCH, "-shared", "-o", LIB, *objs, "-Xcompiler", "-fPIC"]
         if verbose:

@@ -96,6 +96,10 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
         c->decode_ok = false;
         c->decode_why = "decode supports at most 8 kept groups per head and side";
       }
+  if (cfg.d_head % 16 != 0 || cfg.d_head > 256) {
+    c->decode_ok = false;
+    c->decode_why = "decode needs d_head a multiple of 16 and at most 256";
+  }
   if (c->h.max_sec_bytes > 27 * 1024) {
     c->decode_ok = false;
     c->decode_why = "head section of a page exceeds 27 KB; use fewer page_tokens";
@@ -109,9 +113,9 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
   const size_t off_wt = off_err + 256;
   const size_t wt_bytes = (size_t)c->h.n_eff_pad * dm * 2;
   const size_t off_wu = off_wt + (wt_bytes + 255) / 256 * 256;
-  size_t kept_total = 0;
+  size_t kept_total = 0;  // floats of W_up: per-side blocks, then the K sides again as rows
   for (int a = 0; a < cfg.n_kv_heads; ++a)
-    for (int s = 0; s < 2; ++s) kept_total += c->h.head[a].side[s].n_kept;
+    kept_total += 2 * (size_t)c->h.head[a].side[0].n_kept + c->h.head[a].side[1].n_kept;
   const size_t wu_bytes = std::max<size_t>(kept_total * dh * 4, 4);
   const size_t total = off_wu + wu_bytes;
   CUDA_TRY(cudaMalloc(&c->dmem, total));
@@ -140,6 +144,7 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
           for (int d = 0; d < dh; ++d) {
             const size_t at = s == 0 ? (size_t)d * sd.n_kept + row : (size_t)row * dh + d;
             wu[sd.wup_off + at] = from[d];
+            if (s == 0) wu[c->h.head[a].wupk_rows_off + (size_t)row * dh + d] = from[d];
           }
         }
       }

@@ -87,7 +87,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 
 // ---- legacy warp-level tensor core MMA (fp16 in, fp32 accumulate) -----------
 __device__ __forceinline__ void mma_m16n8k16(float d[4], const uint32_t a[4], const uint32_t b[2]) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -95,7 +95,7 @@ __device__ __forceinline__ void mma_m16n8k16(float d[4], const uint32_t a[4], co
 }
 
 __device__ __forceinline__ void mma_m16n8k8(float d[4], const uint32_t a[2], uint32_t b) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(b));

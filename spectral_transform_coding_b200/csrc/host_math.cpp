@@ -318,30 +318,30 @@ int build_layout(const spectra_config& cfg, const int32_t* widths, CodecDev* cd)
     }
     hd.sec_bytes = (int32_t)(off - hd.sec_off);
     max_sec = std::max(max_sec, hd.sec_bytes);
-    // decode walk order: width classes 4, 2, 1, 3, 8
     static const int kClassOrder[5] = {4, 2, 1, 3, 8};
     for (int s = 0; s < 2; ++s) {
       const SideDev& sd = hd.side[s];
-      DecodeTables& T = hd.dec;
       int n = 0;
       for (int ci = 0; ci < 5; ++ci) {
-        T.cls[s][ci] = n;
-        for (int j = 0; j < sd.n_groups && j < kDecMaxGroups; ++j) {
+        hd.dec.cls[s][ci] = n;
+        for (int j = 0; j < sd.n_groups && n < kDecMaxGroups; ++j) {
           const GroupDev& gd = sd.grp[j];
           if (gd.b != kClassOrder[ci]) continue;
-          T.ord[s][n][0] = gd.plane_off - hd.sec_off;
-          T.ord[s][n][1] = gd.sz_off - hd.sec_off;
-          T.ord[s][n][2] = j;
-          T.ord[s][n][3] = gd.b;
+          hd.dec.ord[s][n][0] = gd.plane_off - hd.sec_off;
+          hd.dec.ord[s][n][1] = gd.sz_off - hd.sec_off;
+          hd.dec.ord[s][n][2] = j;
+          hd.dec.ord[s][n][3] = gd.b;
           ++n;
         }
       }
-      for (int ci = 5; ci < 8; ++ci) T.cls[s][ci] = n;
-      for (int j = 0; j < kDecMaxGroups; ++j) {
-        T.rec[s][j] = j < sd.n_groups ? sd.grp[j].sz_off - hd.sec_off : -1;
-        T.wid[s][j] = j < sd.n_groups ? sd.grp[j].b : 0;
-      }
+      for (int ci = 5; ci < 8; ++ci) hd.dec.cls[s][ci] = n;
     }
+  }
+  // a second copy of each K side's W_up, as rows [n_kept][d_head], after all the
+  // per-side blocks (the decode's query fold reads it row by row)
+  for (int a = 0; a < cfg.n_kv_heads; ++a) {
+    cd->head[a].wupk_rows_off = wup;
+    wup += cd->head[a].side[0].n_kept * cfg.d_head;
   }
   if (off > (int64_t)1 << 30) return 2;
   cd->d_model = cfg.d_model;

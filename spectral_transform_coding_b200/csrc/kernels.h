@@ -73,12 +73,17 @@ cudaError_t launch_decode_reconstruct(const CodecDev& h, const CodecDev* d, cons
 // `bytes` (one record per kernel and device; the limit never shrinks).
 cudaError_t ensure_dynamic_smem(const void* kern, int bytes);
 struct DecodePlan {
-  int n_split;       // context splits per (sequence, KV head), before clamping to the cache's pages
-  int stages;        // bulk-copy stages per warp
+  int n_split;       // context splits per (sequence, KV head)
+  int cl;            // CTAs per thread-block cluster (divides n_split)
+  int slice_k;       // K coordinates folded per cluster rank
+  int slice_v;       // V coordinates lifted per cluster rank
+  int wv_staged;     // the rank's W_up^V rows are bulk-copied into shared memory
+  int stages;        // page stages of the CTA's ring
   int stage_bytes;   // bytes per stage (largest head section, rounded to 16)
-  int smem_bytes;    // dynamic shared memory of the split kernel
-  size_t frag_off, part_off, ws_bytes;  // workspace carve-up: folded-query fragments, partial records
-  int part_stride;   // floats per partial record (multiple of 4)
+  int off_stages;    // shared-memory offset of the ring
+  int smem_bytes;    // dynamic shared memory per CTA
+  int rec_stride;    // floats per cluster record of one q head
+  size_t cnt_off, rec_off, ws_bytes;  // workspace: arrival counters (zero between calls), cluster records
 };
 DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq);
 cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,

@@ -32,24 +32,22 @@ struct SideDev {
   GroupDev grp[kMaxGroups];
 };
 
-// Kept groups of a head as the decode kernel walks them, per side (0 K, 1 V):
-// ordered by width class (4, 2, 1, 3, 8), each entry {block offset, record
-// offset (both from the head section start), group index, width}; class bounds
-// cls[side][0..5]; record offsets and widths by group index (-1 / 0 if absent).
-constexpr int kDecMaxGroups = 8;  // kept groups per side the decode kernels handle
-struct DecodeTables {
+// Kept groups of a head side in the order the decode kernel walks them: width
+// classes 4, 2, 1, 3, 8; entry {block offset, record offset (both from the head
+// section start), group index, width}; class bounds cls[0..5] (the rest pad).
+constexpr int kDecMaxGroups = 8;  // kept groups per side the decode kernel handles
+struct DecodeOrder {
   int32_t ord[2][kDecMaxGroups][4];
   int32_t cls[2][8];
-  int32_t rec[2][kDecMaxGroups];
-  int32_t wid[2][kDecMaxGroups];
 };
 
 struct HeadDev {
   SideDev side[2];
-  int32_t sec_off;    // byte offset of the head section in a page
-  int32_t sec_bytes;  // bytes of the head section (K + V)
-  int32_t pad[2];
-  DecodeTables dec;   // filled when both sides have <= kDecMaxGroups kept groups
+  int32_t sec_off;        // byte offset of the head section in a page
+  int32_t sec_bytes;      // bytes of the head section (K + V)
+  int32_t wupk_rows_off;  // offset (floats) of the K side's W_up rows [n_kept][d_head] (the query fold)
+  int32_t pad;
+  DecodeOrder dec;        // filled when both sides have <= kDecMaxGroups kept groups
 };
 
 // Device-resident description of a codec; kernels read it from global memory.

@@ -5,11 +5,11 @@ A step is the encode of the new tokens, then decode attention.  In the chained
 run no host synchronisation or other kernel separates the launches, so the
 kernels' early starts under programmatic dependent launch are in play:
 - a decode's first page copies are issued before its dependency wait;
-- the length it reads there may still be advancing.
+- the length it reads there may still be advancing (a hint).
 Lengths start just below page boundaries, so some steps cross into a new
-page.  That is the case in which the speculative copies must be drained and
-reissued.  The decode is deterministic (fixed split-K partition and merge
-order), so the two runs must agree bit for bit."""
+page: then the length the decode reads before its wait may lag the final one.
+The decode is deterministic (its split-K partition and merge order depend only
+on the final length), so the two runs must agree bit for bit."""
 import numpy as np
 import pytest
 
@@ -67,3 +67,32 @@ def test_chained_steps_equal_synchronised_steps(name, T):
     assert torch.equal(a[2], b[2]) and list(a[2].numpy()) == [L + n_steps * T for L in start]
     assert torch.equal(a[1], b[1]), "packed pages differ between chained and synchronised steps"
     assert torch.equal(a[0], b[0]), "decode outputs differ between chained and synchronised steps"
+
+
+@pytest.mark.parametrize("lag", [1, 65, 1 << 20, -200])
+def test_length_hint_does_not_change_the_result(lag, monkeypatch):
+    """The decode reads the length before its dependency wait as a hint and copies
+    the pages that are full under it early.  The page partition and summation
+    order depend only on the final length, so offsetting the hint (the library's
+    SPECTRA_DECODE_HINT_LAG test hook) must give the same bits: a positive lag
+    moves page copies after the wait, a negative one makes the kernel copy pages
+    beyond the length that it must drain unused."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup("llama4x", seed=6)
+    codec, P = s["codec"], s["P"]
+    lengths = [333, 64, 1, 2049]
+    B, maxp = len(lengths), 40
+    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=maxp, device=dev())
+    seqs = np.concatenate([np.full(L, b, np.int32) for b, L in enumerate(lengths)])
+    lat = synthetic_latents(seqs.size, codec.n_eff, seed=8, decay=0.5, scale=2.0)
+    codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+    rng = np.random.default_rng(9)
+    q = torch.from_numpy((rng.standard_normal((B, s["n_q"], s["d_h"])) * 0.6).astype(np.float32)).to(dev())
+    ref = codec.decode_attend(cache, q)
+    codec.device_status()
+    monkeypatch.setenv("SPECTRA_DECODE_HINT_LAG", str(lag))
+    for _ in range(2):
+        got = codec.decode_attend(cache, q)
+        codec.device_status()
+        assert torch.equal(got, ref)
