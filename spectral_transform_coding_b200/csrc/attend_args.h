@@ -15,7 +15,6 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxG = 8;          // kept groups per side handled by the decode kernel
 constexpr int kMaxKept = 128;     // kept coordinates per side
 constexpr int kMaxStages = 32;    // page stages per CTA
-constexpr int kMaxCluster = 8;
 constexpr int kMaxSplit = 128;    // context splits per (sequence, KV head)
 constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // bounded waits
 constexpr float kPScaleLog2 = 8.f;   // p = 2^(s - m + 8): fp16 keeps small weights normal
@@ -35,11 +34,11 @@ constexpr int kOffCls = kOffOrd + 256;
 constexpr int kOffBq = kOffCls + 128;                // uint2 [(kMaxG*2 + 2) * 32] fragments
 constexpr int kBqWords = (kMaxG * 2 + 2) * 32;
 constexpr int kOffQlat = kOffBq + kBqWords * 8;      // float [kMaxGQ][kMaxKept]
-constexpr int kOffX = kOffQlat + kMaxGQ * kMaxKept * 4;  // q (prologue) / CTA partial (merge)
+constexpr int kOffX = kOffQlat + kMaxGQ * kMaxKept * 4;  // q (prologue) / merged latent sums (last CTA)
 constexpr int kXBytes = kMaxGQ * kMaxDHead * 4;
-constexpr int kOffW = kOffX + kXBytes;               // float [2][kMaxGQ][kMaxCluster + 2]: merge weights
-constexpr int kOffFixedEnd = kOffW + 2 * kMaxGQ * (kMaxCluster + 2) * 4;  // W_up^V slice, then the stages
-constexpr int kCpStride = 2 + kMaxKept;              // floats per q head in a CTA partial
+constexpr int kOffW = kOffX + kXBytes;               // float [kMaxGQ][kWarps + 2]: merge weights, sums
+constexpr int kOffFixedEnd = kOffW + kMaxGQ * (kWarps + 2) * 4;  // then the stage ring
+constexpr int kCpStride = 2 + kMaxKept;              // floats per q head in a warp's partial
 
 enum { kFlagPre = 0, kFlagStop = 1, kFlagLast = 2 };
 
@@ -50,20 +49,17 @@ struct AttendArgs {
   const int32_t* lengths;
   const float* q;
   float* out;
-  float* rec;       // cluster records [B][n_kv][n_clusters][gq][rec_stride]
+  float* rec;       // split records [B][n_kv][n_split][gq][rec_stride]: m, l, -, -, latent sums
   int32_t* cnt;     // [B][n_kv] arrival counters, zero between calls
   int64_t n_pool_pages;
   int64_t page_bytes;
   int max_pages;
   int n_split;
-  int cl;           // CTAs per cluster (divides n_split)
   int stages;
   int stage_bytes;
   int off_stages;
   int rec_stride;
-  int slice_k;      // K coordinates folded per cluster rank
-  int slice_v;      // V coordinates lifted per cluster rank
-  int wv_staged;    // the W_up^V slice is bulk-copied into shared memory
+  int wv_staged;    // the last CTA bulk-copies the head's W_up^V into its stage ring
   int n_q;
   int n_kv;
   int d_h;

@@ -84,11 +84,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
 
 // Split x into fp16 hi (part 0) or the fp16 of the remainder (part 1).
 __device__ __forceinline__ float split_half(float x, int part) {
@@ -316,10 +311,6 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
   const int split = blockIdx.x, a = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, t4 = lane & 3;
-  const int CL = A.cl;
-  const int rank = CL > 1 ? (int)cluster_rank() : 0;
-  const int n_clusters = A.n_split / CL;
-  const int cluster_id = split / CL;
   pdl_launch_dependents();
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
@@ -330,7 +321,6 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
   uint2* bq_s = reinterpret_cast<uint2*>(smem + kOffBq);
   float* qlat_s = reinterpret_cast<float*>(smem + kOffQlat);  // [kMaxGQ][kMaxKept]
   float* x_s = reinterpret_cast<float*>(smem + kOffX);
-  float* wv_s = reinterpret_cast<float*>(smem + kOffFixedEnd);
   uint8_t* stages = smem + A.off_stages;
   const uint32_t stages_u32 = smem_u32(stages);
 
@@ -345,8 +335,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
   const int ns = A.n_split;
   const int64_t cap = (int64_t)A.max_pages * P;
   const int32_t* ptab = A.page_table + (size_t)b * A.max_pages;
-  const int kv0 = min(nkV, rank * A.slice_v), kv1 = min(nkV, kv0 + A.slice_v);
-  const int k0 = min(nkK, rank * A.slice_k), k1 = min(nkK, k0 + A.slice_k);
+  const int k0 = 0, k1 = nkK;  // the fold covers every kept K coordinate
 
   // ---- 1. the independent global loads first, all in flight together -----------
   // (warp 0: the length hint and this CTA's first page ids; warp 1: the group
@@ -426,11 +415,6 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
       issued[lane] = 1;
     }
     if (lane == 0) flags[kFlagPre] = n_pre;
-    if (lane == 31 && A.wv_staged && kv1 > kv0) {
-      const uint32_t bytes = (uint32_t)(kv1 - kv0) * d_h * 4;
-      mbar_arrive_expect_tx(&bars[kMaxStages], bytes);
-      bulk_copy_g2s(wv_s, A.cd->w_up + hm[7] + (size_t)kv0 * d_h, bytes, &bars[kMaxStages]);
-    }
   }
   __syncthreads();
 
@@ -472,29 +456,6 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
           v += __shfl_xor_sync(0xffffffffu, v, 1);
           v += __shfl_xor_sync(0xffffffffu, v, 2);
           if (qd == 0 && k < k1) qlat_s[h * kMaxKept + k] = v * A.q_scale;
-        }
-      }
-    }
-  }
-  // gather the other ranks' slices (distributed shared memory): warp h < gq
-  // copies head h, all remote loads of a pass in flight together
-  if (CL > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    if (warp < gq) {
-      for (int kb = 0; kb < A.slice_k; kb += 32) {
-        float v[kMaxCluster];
-#pragma unroll
-        for (int r = 0; r < kMaxCluster; ++r) {
-          const int k = r * A.slice_k + kb + lane;
-          v[r] = 0.f;
-          if (r < CL && r != rank && kb + lane < A.slice_k && k < nkK)
-            v[r] = cluster.map_shared_rank(qlat_s, r)[warp * kMaxKept + k];
-        }
-#pragma unroll
-        for (int r = 0; r < kMaxCluster; ++r) {
-          const int k = r * A.slice_k + kb + lane;
-          if (r < CL && r != rank && kb + lane < A.slice_k && k < nkK) qlat_s[warp * kMaxKept + k] = v[r];
         }
       }
     }
@@ -853,12 +814,11 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
   }
   __syncthreads();
 
-  // ---- 9. merge the warps into this CTA's partial (m, l, latent sums) ---------------
+  // ---- 9. merge the warps into this CTA's record (m, l, latent sums) ----------------
   // latent sum of (head h, coordinate j*G + k) = 2^24 * f * va + the z term of
   // group j; f = 1/16 for rows k >= 8 of a G = 16 group of width <= 4
   constexpr int kWs = kCpStride;
   float* wsm = reinterpret_cast<float*>(stages);            // [warp][gq][kWs]
-  float* cpart = x_s;                                       // [gq][kCpStride]
   if (gid == 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -893,9 +853,12 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     }
   }
   __syncthreads();
+  const size_t unit = (size_t)b * A.n_kv + a;
+  float* recs = A.rec + unit * ns * gq * A.rec_stride;  // [split][gq][rec_stride]
   {
-    // weights of the warps per head: wts[h][w], then M, L
+    // weights of the warps per head: wts[h][w]; the record's m and l
     float* wts = reinterpret_cast<float*>(smem + kOffW);  // [gq][kWarps + 2]
+    float* rec = recs + (size_t)split * gq * A.rec_stride;
     if (tid < gq) {
       float M = -CUDART_INF_F;
       for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wsm[(w * gq + tid) * kWs]);
@@ -906,8 +869,8 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
         wts[tid * (kWarps + 2) + w] = wt;
         Ls = fmaf(wt, wsm[(w * gq + tid) * kWs + 1], Ls);
       }
-      cpart[tid * kCpStride + 0] = M;
-      cpart[tid * kCpStride + 1] = Ls;
+      rec[tid * A.rec_stride + 0] = M;
+      rec[tid * A.rec_stride + 1] = Ls;
     }
     __syncthreads();
     if (tid < nkV) {
@@ -916,168 +879,106 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
         float v = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) v = fmaf(wt[w], wsm[(w * gq + h) * kWs + 2 + tid], v);
-        cpart[h * kCpStride + 2 + tid] = v;
+        rec[h * A.rec_stride + 4 + tid] = v;
       }
     }
   }
-
-  // ---- 10. merge the cluster; lift this rank's value slice with W_up^V ---------------
-  // (remote loads are issued for all ranks before they are combined, so each
-  // phase costs one distributed-shared-memory round trip)
-  cg::cluster_group cluster = cg::this_cluster();
-  if (CL > 1) cluster.sync();
-  else __syncthreads();
-  auto peer = [&](float* p, int r) -> const float* { return CL > 1 ? cluster.map_shared_rank(p, r) : p; };
-  float* mw = reinterpret_cast<float*>(smem + kOffW) + kMaxGQ * (kMaxCluster + 2);  // [gq][kMaxCluster + 2]
-  float* accs = reinterpret_cast<float*>(smem + kOffBq);    // [gq][slice]: merged latent sums of the slice
-  const int nsv = kv1 - kv0;
-  if (tid < gq) {
-    float mr[kMaxCluster], lr[kMaxCluster];
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      mr[r] = -CUDART_INF_F;
-      lr[r] = 0.f;
-      if (r < CL) {
-        const float* cp = peer(cpart, r);
-        mr[r] = cp[tid * kCpStride];
-        lr[r] = cp[tid * kCpStride + 1];
-      }
-    }
-    float M = -CUDART_INF_F;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) M = fmaxf(M, mr[r]);
-    float Ls = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      const float wt = (mr[r] == -CUDART_INF_F) ? 0.f : ex2_approx(mr[r] - M);
-      mw[tid * (kMaxCluster + 2) + r] = wt;
-      Ls = fmaf(wt, lr[r], Ls);
-    }
-    mw[tid * (kMaxCluster + 2) + kMaxCluster] = M;
-    mw[tid * (kMaxCluster + 2) + kMaxCluster + 1] = Ls;
-  }
+  // ---- 10. the last CTA of this (sequence, KV head) merges the records and lifts ------
+  __threadfence();
   __syncthreads();
-  if (warp < gq) {  // warp h: head h's latent sums of this rank's value slice
-    const int h = warp;
-    for (int cb = 0; cb < nsv; cb += 32) {
-      const int c = kv0 + cb + lane;
-      float x[kMaxCluster];
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) x[r] = (r < CL && cb + lane < nsv) ? peer(cpart, r)[h * kCpStride + 2 + c] : 0.f;
-      float v = 0.f;
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) v = fmaf(mw[h * (kMaxCluster + 2) + r], x[r], v);
-      if (cb + lane < nsv) accs[h * A.slice_v + cb + lane] = v;
-    }
-  }
-  bool wv_ok = true;
-  if (A.wv_staged && nsv > 0) wv_ok = mbar_wait_bounded(&bars[kMaxStages], 0u, kWaitLimitNs);
-  if (!wv_ok && tid == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
-  __syncthreads();
-  float* orp = reinterpret_cast<float*>(stages);  // [gq][d_h]: this rank's lifted slice
-  if (warp < gq) {  // warp h: head h, lanes over 4 consecutive output dimensions
-    const int h = warp;
-    const float* wv = A.wv_staged ? wv_s : cd->w_up + hm[7] + (size_t)kv0 * d_h;
-    for (int d4 = lane; d4 < d_h / 4; d4 += 32) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (wv_ok) {
-        for (int c = 0; c < nsv; ++c) {
-          const float x = accs[h * A.slice_v + c];
-          const float4 w = reinterpret_cast<const float4*>(wv + (size_t)c * d_h)[d4];
-          v.x = fmaf(x, w.x, v.x);
-          v.y = fmaf(x, w.y, v.y);
-          v.z = fmaf(x, w.z, v.z);
-          v.w = fmaf(x, w.w, v.w);
-        }
-      }
-      reinterpret_cast<float4*>(orp + h * d_h)[d4] = v;
-    }
-  }
-  if (CL > 1) cluster.sync();
-  else __syncthreads();
-  // this rank's slice of the output dimension: the cluster's sum
-  const int ds = (d_h + CL - 1) / CL;
-  const int d0 = min(d_h, rank * ds), d1 = min(d_h, d0 + ds);
-  float* recb = A.rec + (((size_t)b * A.n_kv + a) * n_clusters + cluster_id) * gq * A.rec_stride;
-  if (warp < gq) {
-    const int h = warp;
-    const float Ls = mw[h * (kMaxCluster + 2) + kMaxCluster + 1];
-    for (int d = d0 + lane; d < d1; d += 32) {
-      float x[kMaxCluster];
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) x[r] = r < CL ? peer(orp, r)[h * d_h + d] : 0.f;
-      float v = 0.f;
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) v += x[r];
-      if (n_clusters == 1) A.out[((size_t)b * A.n_q + (size_t)a * gq + h) * d_h + d] = Ls > 0.f ? v / Ls : 0.f;
-      else recb[h * A.rec_stride + 4 + d] = v;
-    }
-  }
-  if (n_clusters > 1 && rank == 0 && tid < gq) {
-    recb[tid * A.rec_stride + 0] = mw[tid * (kMaxCluster + 2) + kMaxCluster];
-    recb[tid * A.rec_stride + 1] = mw[tid * (kMaxCluster + 2) + kMaxCluster + 1];
-  }
-  if (n_clusters > 1) __threadfence();
-  // no CTA leaves while a peer may still read its shared memory
-  if (CL > 1) cluster.sync();
-  else __syncthreads();
-
-  // ---- 11. the last cluster of this (sequence, KV head) merges the records ------------
-  if (n_clusters == 1 || rank != 0) return;
   if (tid == 0) {
-    const int t = atomicAdd(A.cnt + (size_t)b * A.n_kv + a, 1);
-    const int last = t == n_clusters - 1;
-    if (last) atomicExch(A.cnt + (size_t)b * A.n_kv + a, 0);  // ready for the next call
+    const int t = atomicAdd(A.cnt + unit, 1);
+    const int last = t == ns - 1;
+    if (last) atomicExch(A.cnt + unit, 0);  // ready for the next call
     flags[kFlagLast] = last;
   }
   __syncthreads();
   if (!flags[kFlagLast]) return;
   __threadfence();
-  const float* recs = A.rec + ((size_t)b * A.n_kv + a) * n_clusters * gq * A.rec_stride;
-  const size_t cstride = (size_t)gq * A.rec_stride;  // floats between clusters' records
-  if (warp < gq) {
-    // warp h: head h; lane: 4 consecutive output dimensions; the records of up
-    // to 16 clusters are loaded in one batch
+  // W_up^V of this head into the (idle) stage ring while the records merge
+  const uint32_t wv_bytes = (uint32_t)nkV * d_h * 4;
+  const bool wv_staged = A.wv_staged != 0;
+  float* wv_s = reinterpret_cast<float*>(stages);
+  if (tid == 0 && wv_staged && wv_bytes > 0) {
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&bars[kMaxStages], wv_bytes);
+    bulk_copy_g2s(wv_s, cd->w_up + hm[7], wv_bytes, &bars[kMaxStages]);
+  }
+  float* wts = reinterpret_cast<float*>(smem + kOffQlat);   // [gq][kMaxSplit] weights (q_lat is dead)
+  float* acc = reinterpret_cast<float*>(smem + kOffX);      // [gq][kMaxKept] merged latent sums
+  float* lsum = reinterpret_cast<float*>(smem + kOffW);     // [gq] sum of weights x l
+  const size_t hs = (size_t)gq * A.rec_stride;              // floats between splits' records
+  if (warp < gq) {  // warp h: the maximum and the weights of the splits for head h
     const int h = warp;
-    for (int d4 = lane; d4 < d_h / 4; d4 += 32) {
-      float M = -CUDART_INF_F, den = 0.f;
-      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c0 = 0; c0 < n_clusters; c0 += 16) {
-        float m[16], l[16];
-        float4 o[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const bool ok = c0 + u < n_clusters;
-          const float* r = recs + (c0 + u) * cstride + h * A.rec_stride;
-          m[u] = ok ? __ldcg(r) : -CUDART_INF_F;
-          l[u] = ok ? __ldcg(r + 1) : 0.f;
-          o[u] = ok ? __ldcg(reinterpret_cast<const float4*>(r + 4) + d4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float Mn = M;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) Mn = fmaxf(Mn, m[u]);
-        // rescale what earlier batches summed to the new maximum
-        const float sc = (M == -CUDART_INF_F) ? 0.f : ex2_approx(M - Mn);
-        den *= sc;
-        num.x *= sc;
-        num.y *= sc;
-        num.z *= sc;
-        num.w *= sc;
-        M = Mn;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float wt = (m[u] == -CUDART_INF_F) ? 0.f : ex2_approx(m[u] - M);
-          den = fmaf(wt, l[u], den);
-          num.x = fmaf(wt, o[u].x, num.x);
-          num.y = fmaf(wt, o[u].y, num.y);
-          num.z = fmaf(wt, o[u].z, num.z);
-          num.w = fmaf(wt, o[u].w, num.w);
-        }
-      }
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-      reinterpret_cast<float4*>(A.out + ((size_t)b * A.n_q + (size_t)a * gq + h) * d_h)[d4] =
-          make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+    float M = -CUDART_INF_F;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      const int sp = s0 + lane;
+      const float m = sp < ns ? __ldcg(recs + sp * hs + h * A.rec_stride) : -CUDART_INF_F;
+      M = fmaxf(M, m);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Ls = 0.f;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      const int sp = s0 + lane;
+      if (sp < ns) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(recs + sp * hs + h * A.rec_stride));
+        const float wt = (ml.x == -CUDART_INF_F) ? 0.f : ex2_approx(ml.x - M);
+        wts[h * kMaxSplit + sp] = wt;
+        Ls = fmaf(wt, ml.y, Ls);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (lane == 0) lsum[h] = Ls;
+  }
+  __syncthreads();
+  // thread (h, 4 consecutive coordinates): the splits' records, 16 loads in flight
+  for (int e = tid; e < gq * (kMaxKept / 4); e += kThreads) {
+    const int h = e / (kMaxKept / 4), c4 = e - h * (kMaxKept / 4);
+    if (4 * c4 >= nkV) continue;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float* base = recs + h * A.rec_stride + 4;
+    for (int s0 = 0; s0 < ns; s0 += 16) {
+      float4 x[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        x[u] = s0 + u < ns ? __ldcg(reinterpret_cast<const float4*>(base + (s0 + u) * hs) + c4)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float wt = s0 + u < ns ? wts[h * kMaxSplit + s0 + u] : 0.f;
+        v.x = fmaf(wt, x[u].x, v.x);
+        v.y = fmaf(wt, x[u].y, v.y);
+        v.z = fmaf(wt, x[u].z, v.z);
+        v.w = fmaf(wt, x[u].w, v.w);
+      }
+    }
+    reinterpret_cast<float4*>(acc + h * kMaxKept)[c4] = v;
+  }
+  bool wv_ok = true;
+  if (wv_staged && wv_bytes > 0) wv_ok = mbar_wait_bounded(&bars[kMaxStages], 0u, kWaitLimitNs);
+  if (!wv_ok && tid == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
+  __syncthreads();
+  // out = (merged latent sums / L) W_up^V: thread (h, 4 consecutive dims)
+  const float* wv = wv_staged ? wv_s : cd->w_up + hm[7];
+  for (int e = tid; e < gq * (d_h / 4); e += kThreads) {
+    const int h = e / (d_h / 4), d4 = e - h * (d_h / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (wv_ok) {
+      for (int c = 0; c < nkV; ++c) {
+        const float x = acc[h * kMaxKept + c];
+        const float4 w = reinterpret_cast<const float4*>(wv + (size_t)c * d_h)[d4];
+        v.x = fmaf(x, w.x, v.x);
+        v.y = fmaf(x, w.y, v.y);
+        v.z = fmaf(x, w.z, v.z);
+        v.w = fmaf(x, w.w, v.w);
+      }
+    }
+    const float Ls = lsum[h];
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    reinterpret_cast<float4*>(A.out + ((size_t)b * A.n_q + (size_t)a * gq + h) * d_h)[d4] =
+        make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
   }
 }
 

@@ -51,7 +51,7 @@ using attend::AttendKernel;
 using attend::kThreads;
 using attend::kWarps;
 using attend::kMaxStages;
-using attend::kMaxCluster;
+using attend::kMaxKept;
 using attend::kMaxSplit;
 using attend::kOffFixedEnd;
 using attend::kCpStride;
@@ -106,70 +106,42 @@ AttendKernel attend_kernel_for(const CodecDev& h) {
   return attend::attend_kernel_ptr(h.group, h.gq > 4 ? 2 : 1, chunk_tiles(h.P), value_group_bound(h));
 }
 
-// Clusters of `cl` CTAs with `smem` bytes each that the device holds at once
-// (clusters must fit in one GPC, so this is below slots / cl in general).
-int max_active_clusters(AttendKernel kern, int cl, int smem) {
+// CTAs with `smem` bytes of dynamic shared memory that one SM holds.
+int ctas_per_sm(AttendKernel kern, int smem) {
   static std::mutex mu;
-  static std::map<std::tuple<const void*, int, int, int>, int> memo;
+  static std::map<std::tuple<const void*, int, int>, int> memo;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), cl, smem, dev);
+  const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), smem, dev);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = memo.find(key);
     if (it != memo.end()) return it->second;
   }
   int n = 0;
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl, 1, 1);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess)
+    n = 0;
   (void)cudaGetLastError();
-  if (n <= 0) n = std::max(1, 2 * sm_count() / cl);  // no device answer: the ideal packing
+  if (n <= 0) n = 2;  // no device answer: what the shared-memory budget is sized for
   std::lock_guard<std::mutex> lock(mu);
   memo[key] = n;
   return n;
 }
 
-DecodePlan plan_for_cluster(const CodecDev& h, int cl) {
-  DecodePlan p{};
-  p.cl = cl;
-  p.stage_bytes = std::max(16, ((h.max_sec_bytes + 15) / 16) * 16);
-  p.slice_k = std::max(1, (h.max_kept_k + cl - 1) / cl);
-  p.slice_v = std::max(1, (h.max_kept_v + cl - 1) / cl);
-  const int wv_bytes = ((p.slice_v * h.d_h * 4 + 127) / 128) * 128;
-  p.wv_staged = wv_bytes <= 32 * 1024 ? 1 : 0;
-  const int fixed = kOffFixedEnd + (p.wv_staged ? wv_bytes : 0);
-  p.off_stages = ((fixed + 127) / 128) * 128;
-  const int budget = 112 * 1024 - p.off_stages;
-  p.stages = std::max(1, std::min(kMaxStages, budget / p.stage_bytes));
-  const int merge_bytes = std::max(kWarps * kMaxGQ * kCpStride * 4, kMaxGQ * h.d_h * 4);
-  p.smem_bytes = p.off_stages + std::max(p.stages * p.stage_bytes, merge_bytes);
-  p.rec_stride = 4 + h.d_h;  // {M, L, -, -} then d_head floats (16-byte aligned rows)
-  return p;
-}
-
 }  // namespace
 
-// Plan of one decode step (memoised per shape, batch and device).  Context
-// splits come in clusters of up to 8 CTAs, which share the query fold and the
-// value lift; the split count minimises an estimated step time: a nominal
-// 16 us of streaming spread over the CTA slots that one wave of clusters fills
-// (the device reports how many clusters fit at once), 2 us of fixed work
-// (fold, merges) per wave, and a penalty for clusters of fewer than 4 CTAs.
-// The count does not depend on the context length, so a workspace sized once
-// fits every call.  Shared memory: fixed tables, the W_up^V slice when it
-// fits, and a ring of page stages of up to ~100 KB (two CTAs per SM).
+// Plan of one decode step (memoised per shape, batch and device).
+// Shared memory: fixed tables and a ring of page stages, ~112 KB per CTA so
+// that two CTAs fit an SM; the last CTA of a (sequence, KV head) reuses its
+// ring for W_up^V when the head's rows fit.
+// Splits per (sequence, KV head): few units (batch-1 decode) mean little
+// streaming work per CTA, so a launch takes one CTA slot per SM and the other
+// slot lets the next launch's CTAs become resident, fold and prefetch while
+// this one runs; many units fill both slots.  The count minimises an estimated
+// step time, a nominal 16 us of streaming over the slots one wave fills plus
+// 2 us of fixed work (fold, merges) per wave; it does not depend on the
+// context length, so a workspace sized once fits every call.
 DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq) {
   (void)max_pages_per_seq;
   static std::mutex mu;
@@ -183,33 +155,38 @@ DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq)
     auto it = memo.find(key);
     if (it != memo.end()) return it->second;
   }
+  DecodePlan p{};
+  p.cl = 1;
+  p.stage_bytes = std::max(16, ((h.max_sec_bytes + 15) / 16) * 16);
+  p.off_stages = ((kOffFixedEnd + 127) / 128) * 128;
+  const int budget = 112 * 1024 - p.off_stages;
+  p.stages = std::max(1, std::min(kMaxStages, budget / p.stage_bytes));
+  const int merge_bytes = kWarps * kMaxGQ * kCpStride * 4;
+  const int wv_bytes = h.max_kept_v * h.d_h * 4;
+  int ring = std::max(p.stages * p.stage_bytes, merge_bytes);
+  p.wv_staged = wv_bytes <= std::max(ring, budget) ? 1 : 0;
+  if (p.wv_staged) ring = std::max(ring, wv_bytes);
+  p.smem_bytes = p.off_stages + ring;
+  p.rec_stride = 4 + kMaxKept;  // {m, l, -, -} then the latent sums (16-byte aligned rows)
+  p.slice_k = h.max_kept_k;
+  p.slice_v = h.max_kept_v;
   const AttendKernel kern = attend_kernel_for(h);
   const int units = std::max(1, batch * h.n_kv);
-  // Few (sequence, KV head) units (batch-1 decode) means little streaming work
-  // per CTA, so a layer takes one CTA slot per SM: the other slot lets the next
-  // launch's CTAs become resident, fold and prefetch while this one runs.  Many
-  // units fill both slots.
   const bool one_per_sm = units * 2 < sm_count();
-  const int slots = (one_per_sm ? 1 : 2) * sm_count();
-  DecodePlan best{};
+  const int slots = (one_per_sm ? 1 : std::max(1, ctas_per_sm(kern, p.smem_bytes))) * sm_count();
+  int best_ns = 1;
   double best_t = 1e30;
-  for (int cl = 1; cl <= kMaxCluster; ++cl) {
-    const DecodePlan p = plan_for_cluster(h, cl);
-    const int cap_dev = max_active_clusters(kern, cl, p.smem_bytes);
-    const int cap = one_per_sm ? std::max(1, std::min(cap_dev / 2, slots / cl)) : cap_dev;
-    for (int ns = cl; ns <= kMaxSplit; ns += cl) {
-      const long clusters = (long)units * (ns / cl);
-      const long waves = (clusters + cap - 1) / cap;
-      const double eff = (double)units * ns / (double)(waves * slots);
-      const double t = 16.0 / eff + 2.0 * waves + (cl < std::min(4, ns) ? 1.0 : 0.0);
-      if (t < best_t - 1e-9) {
-        best_t = t;
-        best = p;
-        best.n_split = ns;
-      }
+  for (int ns = 1; ns <= kMaxSplit; ++ns) {
+    const long ctas = (long)units * ns;
+    const long waves = (ctas + slots - 1) / slots;
+    const double eff = (double)ctas / (double)(waves * slots);
+    const double t = 16.0 / eff + 2.0 * waves;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best_ns = ns;
     }
   }
-  DecodePlan& p = best;
+  p.n_split = best_ns;
   size_t off = 0;
   auto carve = [&](size_t bytes) {
     const size_t o = off;
@@ -217,7 +194,7 @@ DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq)
     return o;
   };
   p.cnt_off = carve((size_t)batch * h.n_kv * 4);
-  p.rec_off = carve((size_t)batch * h.n_kv * (p.n_split / p.cl) * h.gq * p.rec_stride * 4);
+  p.rec_off = carve((size_t)batch * h.n_kv * p.n_split * h.gq * p.rec_stride * 4);
   p.ws_bytes = off;
   std::lock_guard<std::mutex> lock(mu);
   memo[key] = p;
@@ -240,13 +217,10 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
   args.page_bytes = h.page_bytes;
   args.max_pages = cache.max_pages_per_seq;
   args.n_split = plan.n_split;
-  args.cl = plan.cl;
   args.stages = plan.stages;
   args.stage_bytes = plan.stage_bytes;
   args.off_stages = plan.off_stages;
   args.rec_stride = plan.rec_stride;
-  args.slice_k = plan.slice_k;
-  args.slice_v = plan.slice_v;
   args.wv_staged = plan.wv_staged;
   args.n_q = h.n_q;
   args.n_kv = h.n_kv;
@@ -287,21 +261,17 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = plan.smem_bytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = plan.cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_ok ? 2 : 1;
+  cfg.numAttrs = pdl_ok ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, kern, args);
   if (e != cudaSuccess && pdl_ok) {
     // without programmatic serialisation: plain stream order
     (void)cudaGetLastError();
     pdl_ok = false;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 0;
     e = cudaLaunchKernelEx(&cfg, kern, args);
   }
   return e;

@@ -74,16 +74,16 @@ cudaError_t launch_decode_reconstruct(const CodecDev& h, const CodecDev* d, cons
 cudaError_t ensure_dynamic_smem(const void* kern, int bytes);
 struct DecodePlan {
   int n_split;       // context splits per (sequence, KV head)
-  int cl;            // CTAs per thread-block cluster (divides n_split)
-  int slice_k;       // K coordinates folded per cluster rank
-  int slice_v;       // V coordinates lifted per cluster rank
-  int wv_staged;     // the rank's W_up^V rows are bulk-copied into shared memory
+  int cl;            // CTAs per thread-block cluster (1: no clusters)
+  int slice_k;       // K coordinates folded per CTA
+  int slice_v;       // V coordinates lifted by the last CTA
+  int wv_staged;     // the last CTA bulk-copies W_up^V into its stage ring
   int stages;        // page stages of the CTA's ring
   int stage_bytes;   // bytes per stage (largest head section, rounded to 16)
   int off_stages;    // shared-memory offset of the ring
   int smem_bytes;    // dynamic shared memory per CTA
   int rec_stride;    // floats per cluster record of one q head
-  size_t cnt_off, rec_off, ws_bytes;  // workspace: arrival counters (zero between calls), cluster records
+  size_t cnt_off, rec_off, ws_bytes;  // workspace: arrival counters (zero between calls), split records
 };
 DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq);
 cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_cache& cache,

@@ -1,0 +1,135 @@
+"""GPU parity at the shapes the benchmark runs (Llama-3.1-8B- and Qwen2.5-7B-
+shaped layers), through the C ABI.
+
+- The decode-step fused encode at d_model 4096 and 3584, so that its loop over
+  d_model slices runs more than once.
+- The tcgen05 projection at K = d_model = 4096 with 1024 and 2048 latent
+  columns and a row count that is not a multiple of the 128-row tile.
+- The latent decode at 32,768 + 5 tokens with 8 KV heads (Llama 4x) and at
+  131,072 + 3 tokens with 7 q heads per KV head (Qwen 8x), checked on sampled
+  (sequence, q head) pairs against the oracle's decode over its own copy of
+  the pool, which must equal the library's byte for byte.
+
+Bars as in the other parity tests: latents 1e-3 (per token and head-side, L2),
+packed pages bit-exact, attention 2e-3 (max over the sampled pairs of
+||diff||_inf / ||ref||_inf)."""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_helpers import (attention_rel_err, codec_from, dev, kept_wup, make_cfg, oracle_widths, random_factors,
+                         synthetic_latents, torch_mod)
+from workloads import bf16_round
+
+pytestmark = pytest.mark.gpu
+
+LLAMA4X = [4, 2, 2, 2, 2, 2, 1, 1]          # widths of a Llama-shaped head side at 4x
+QWEN8X_K = [4, 2, 1, 1, 0, 0, 0, 0]         # Qwen-shaped head at 8x
+QWEN8X_V = [4, 3, 3, 0, 0, 0, 0, 0]
+
+
+def _codec(d_model, n_q, n_kv, wk, wv, seed, P=64):
+    widths = np.array([[wk, wv]] * n_kv, np.int32)
+    widths, W_down, W_up = random_factors(d_model, n_kv, 128, 128, 16, widths, seed=seed)
+    cfg = make_cfg(d_model, n_q, n_kv, 128, 128, 16, 512, True, P)
+    return codec_from(cfg, widths, W_down, W_up), widths, W_down, W_up
+
+
+def _check_latents(lat, ref, widths):
+    c0 = 0
+    for a in range(widths.shape[0]):
+        for side in range(2):
+            nk = int(sum(16 for b in widths[a, side] if b > 0))
+            d = lat[:, c0:c0 + nk] - ref[:, c0:c0 + nk]
+            rel = np.linalg.norm(d, axis=1) / np.maximum(np.linalg.norm(ref[:, c0:c0 + nk], axis=1), 1e-30)
+            assert rel.max() <= 1e-3, (a, side, rel.max())
+            c0 += nk
+
+
+@pytest.mark.parametrize("d_model,n_q,n_kv,wk,wv", [(4096, 32, 8, LLAMA4X, LLAMA4X),
+                                                    (3584, 28, 4, QWEN8X_K, QWEN8X_V)])
+@pytest.mark.parametrize("T", [1, 16])
+def test_fused_encode_full_width(d_model, n_q, n_kv, wk, wv, T):
+    """The fused decode-step encode over a full-width layer: latents within 1e-3
+    of the oracle's H W_down, pages equal to what the (bit-exact) quantiser
+    writes for the same latents, lengths advanced."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    codec, widths, W_down, _ = _codec(d_model, n_q, n_kv, wk, wv, seed=11)
+    B = 2
+    seqs = np.sort(np.arange(T, dtype=np.int32) % B)
+    rng = np.random.default_rng(12 + T)
+    H = bf16_round(rng.standard_normal((T, d_model)).astype(np.float32))
+    table = np.arange(B * 2, dtype=np.int32).reshape(B, 2)
+    c1 = st.LatentCache(codec, batch=B, max_pages_per_seq=2, device=dev(), page_table=torch.from_numpy(table))
+    c2 = st.LatentCache(codec, batch=B, max_pages_per_seq=2, device=dev(), page_table=torch.from_numpy(table))
+    start = np.array([5, 60], np.int32)  # mid-block; sequence 1 crosses into its second page
+    c1.lengths.copy_(torch.from_numpy(start))
+    c2.lengths.copy_(torch.from_numpy(start))
+    lat = torch.empty((T, codec.n_eff), dtype=torch.float32, device=dev())
+    codec.encode_append(c1, torch.from_numpy(H).to(dev()).to(torch.bfloat16), torch.from_numpy(seqs).to(dev()),
+                        latents_out=lat)
+    codec.device_status()
+    _check_latents(lat.cpu().numpy(), H.astype(np.float64) @ W_down.astype(np.float64), widths)
+    codec.quantize_append(c2, lat, torch.from_numpy(seqs).to(dev()))
+    codec.device_status()
+    assert np.array_equal(c1.pool.cpu().numpy(), c2.pool.cpu().numpy())
+    np.testing.assert_array_equal(c1.lengths.cpu().numpy(), start + np.bincount(seqs, minlength=B))
+
+
+@pytest.mark.parametrize("n_kv", [4, 8])
+def test_projection_tcgen05_full_width(n_kv):
+    """H W_down on the tcgen05 GEMM at K = 4096 (64 k-blocks) with N_eff = 128 n_kv
+    latent columns (1024 or 2048) and 1000 rows (a ragged last M tile); checked
+    on a sample of rows against the fp64 product of the same bf16 values."""
+    torch = torch_mod()
+    codec, widths, W_down, _ = _codec(4096, 4 * n_kv, n_kv, [2] * 8, [2] * 8, seed=13)
+    assert codec.n_eff == 256 * n_kv
+    rng = np.random.default_rng(14)
+    H = bf16_round(rng.standard_normal((1000, 4096)).astype(np.float32))
+    lat = codec.project(torch.from_numpy(H).to(dev()).to(torch.bfloat16)).cpu().numpy()
+    rows = np.r_[0:8, 120:136, rng.choice(1000, 40, replace=False), 992:1000]
+    _check_latents(lat[rows], H[rows].astype(np.float64) @ W_down.astype(np.float64), widths)
+
+
+def _long_decode(n_q, n_kv, wk, wv, length, pairs, seed):
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    codec, widths, _, W_up = _codec(512, n_q, n_kv, wk, wv, seed=seed)
+    P = 64
+    maxp = (length + P - 1) // P + 1
+    rng = np.random.default_rng(seed + 1)
+    table = rng.permutation(maxp).astype(np.int32)[None, :]
+    cache = st.LatentCache(codec, batch=1, max_pages_per_seq=maxp, device=dev(), page_table=torch.from_numpy(table))
+    lay = oracle.page_layout(oracle_widths(widths), 16, P)
+    pool = np.zeros(cache.pool.numel(), np.uint8)
+    lengths = np.zeros(1, np.int64)
+    chunk = 8192
+    for t0 in range(0, length, chunk):
+        n = min(chunk, length - t0)
+        lat = synthetic_latents(n, codec.n_eff, seed=seed + 2 + t0 // chunk, decay=0.5, scale=2.0)
+        seqs = np.zeros(n, np.int32)
+        codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+        lengths = oracle.append_tokens(pool, codec.page_bytes, lay, oracle_widths(widths), 16, P, table, lengths,
+                                       seqs, lat, n_kv)
+    codec.device_status()
+    assert int(cache.lengths.cpu()[0]) == length
+    assert np.array_equal(cache.pool.cpu().numpy(), pool), "packed cache differs from the oracle's"
+    q = (rng.standard_normal((1, n_q, 128)) * 0.6).astype(np.float32)
+    out = codec.decode_attend(cache, torch.from_numpy(q).to(dev())).cpu().numpy()
+    codec.device_status()
+    ref = oracle.decode_reference(pool, codec.page_bytes, lay, 16, P, table, np.array([length]), q,
+                                  kept_wup(W_up, widths, 16), n_q, n_kv, pairs=pairs)
+    got = np.stack([out[b, h] for b, h in pairs])
+    want = np.stack([ref[b, h] for b, h in pairs])
+    return attention_rel_err(got, want)
+
+
+def test_decode_llama_32k_context_8_kv_heads():
+    err = _long_decode(32, 8, LLAMA4X, LLAMA4X, 32768 + 5, [(0, 0), (0, 13), (0, 31)], seed=21)
+    assert err <= 2e-3, err
+
+
+def test_decode_qwen_128k_context_gqa7():
+    err = _long_decode(28, 4, QWEN8X_K, QWEN8X_V, 131072 + 3, [(0, 0), (0, 20), (0, 27)], seed=31)
+    assert err <= 2e-3, err
