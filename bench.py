@@ -299,7 +299,7 @@ def run_gpu(args, rank, world):
     Q = (torch.randn((L, B, cfg.n_q_heads, cfg.d_head), generator=gen, device=dev) * 0.5).contiguous()
     OUT = torch.empty_like(Q)
     seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
-    ews = [torch.empty(codecs[l].encode_workspace_bytes(B), dtype=torch.uint8, device=dev) for l in range(L)]
+    ews = [torch.zeros(codecs[l].encode_workspace_bytes(B), dtype=torch.uint8, device=dev) for l in range(L)]
     rt = args.decode == "reconstruct"
     ws_bytes = (codecs[0].decode_reconstruct_workspace_bytes if rt else codecs[0].decode_workspace_bytes)
     dws = [torch.zeros(ws_bytes(B, cap_tokens), dtype=torch.uint8, device=dev) for l in range(L)]
@@ -514,7 +514,7 @@ def run_prefill(args):
         H = acts(T, 12345)
         cache = st.LatentCache(codec, batch=1, max_pages_per_seq=(T + P - 1) // P + 1, device=dev, zero=False)
         seq = torch.zeros(T, dtype=torch.int32, device=dev)
-        ws = torch.empty(codec.encode_workspace_bytes(T), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(codec.encode_workspace_bytes(T), dtype=torch.uint8, device=dev)
         lat = torch.empty((T, codec.n_eff), dtype=torch.float32, device=dev)
         stream = torch.cuda.Stream(device=dev)
         q = (torch.randn((1, cfg.n_q_heads, cfg.d_head), generator=gen, device=dev) * 0.5).contiguous()

@@ -260,12 +260,16 @@ SPECTRA_API spectra_status spectra_quantize_append(const spectra_codec* codec, c
 /* spectra_encode_append -- spectra_project followed by spectra_quantize_append.
  *   H device bf16 [T][d_model]; seq_ids as above; latents_out device fp32
  *   [T][n_eff] or NULL (when given, the latents are kept there);
- *   workspace device, >= spectra_encode_workspace_bytes(T), 256-byte aligned.
+ *   workspace device, >= spectra_encode_workspace_bytes(T), 256-byte aligned;
+ *   its first 256 bytes hold an arrival counter that must be zero when a call
+ *   starts: zero the workspace once before its first use; every call leaves
+ *   the counter at zero.  Calls that share a workspace must not overlap.
  * For T <= 16 (decode steps) the projection, quantisation and packing run fused
- * in one kernel per kept group (latents summed in a different order than
- * spectra_project's, so they may differ from it in the last bits; the codes are
- * those spectra_quantize_append gives for these latents), followed by a kernel
- * that advances the lengths; the same checks apply and a failure writes nothing. */
+ * in one kernel with one CTA per kept group (latents summed in a different
+ * order than spectra_project's, so they may differ from it in the last bits;
+ * the codes are those spectra_quantize_append gives for these latents); the
+ * CTA that finishes last advances the lengths.  The same checks apply and a
+ * failure writes nothing. */
 SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, const spectra_cache* cache,
                                      const void* H, const int32_t* seq_ids, int64_t T,
                                      float* latents_out, void* workspace, size_t workspace_bytes,

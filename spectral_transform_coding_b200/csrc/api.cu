@@ -157,11 +157,13 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
   return SPECTRA_OK;
 }
 
+// Encode workspace: [arrival counter of the fused path, 256 B][positions][flag][latents].
+constexpr size_t kEncCounterBytes = 256;
 size_t encode_ws_bytes(const spectra_codec* c, int64_t T) {
   const size_t pos = ((size_t)std::max<int64_t>(T, 1) * 4 + 255) / 256 * 256;
   const size_t flag = 256;
   const size_t lat = ((size_t)std::max<int64_t>(T, 1) * c->h.n_eff * 4 + 255) / 256 * 256;
-  return pos + flag + lat;
+  return kEncCounterBytes + pos + flag + lat;
 }
 
 spectra_status check_cache(const spectra_codec* c, const spectra_cache* cache) {
@@ -189,7 +191,7 @@ spectra_status do_project(const spectra_codec* c, const void* H, int64_t T, floa
 
 spectra_status do_quantize_append(const spectra_codec* c, const spectra_cache* cache, const float* C,
                                   const int32_t* seq_ids, int64_t T, void* ws, cudaStream_t st) {
-  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint8_t* w = static_cast<uint8_t*>(ws) + kEncCounterBytes;
   int32_t* pos = reinterpret_cast<int32_t*>(w);
   int32_t* flag = reinterpret_cast<int32_t*>(w + ((size_t)T * 4 + 255) / 256 * 256);
   CUDA_TRY(launch_append_plan(seq_ids, (int)T, *cache, c->cfg.page_tokens, pos, flag, c->err, st));
@@ -612,7 +614,8 @@ spectra_status spectra_quantize_append(const spectra_codec* c, const spectra_cac
   if (!c || !latents || !seq_ids || !workspace) return fail(SPECTRA_ERR_INVALID, "null pointer");
   if (T <= 0 || T > (1 << 24)) return fail(SPECTRA_ERR_INVALID, "T out of range");
   if (!aligned(latents, 16) || !aligned(workspace, 256)) return fail(SPECTRA_ERR_INVALID, "misaligned buffer");
-  if (workspace_bytes < ((size_t)T * 4 + 255) / 256 * 256 + 256) return fail(SPECTRA_ERR_INVALID, "workspace too small");
+  if (workspace_bytes < kEncCounterBytes + ((size_t)T * 4 + 255) / 256 * 256 + 256)
+    return fail(SPECTRA_ERR_INVALID, "workspace too small");
   spectra_status s = check_cache(c, cache);
   if (s != SPECTRA_OK) return s;
   s = check_device(c);
@@ -636,11 +639,11 @@ spectra_status spectra_encode_append(const spectra_codec* c, const spectra_cache
   if (T <= kFusedMaxT) {
     // decode steps: projection, quantisation and packing fused per kept group
     CUDA_TRY(launch_encode_fused(c->h, c->d, static_cast<const uint16_t*>(H), seq_ids, (int)T, *cache,
-                                 latents_out, st));
+                                 latents_out, static_cast<int32_t*>(workspace), st));
     return SPECTRA_OK;
   }
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  const size_t lat_off = ((size_t)T * 4 + 255) / 256 * 256 + 256;
+  const size_t lat_off = kEncCounterBytes + ((size_t)T * 4 + 255) / 256 * 256 + 256;
   float* C = latents_out ? latents_out : reinterpret_cast<float*>(w + lat_off);
   s = do_project(c, H, T, C, st);
   if (s != SPECTRA_OK) return s;

@@ -412,12 +412,14 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
                                                            const uint16_t* __restrict__ H, int T,
                                                            const int32_t* __restrict__ seq_ids,
                                                            const spectra_cache cache,
-                                                           float* __restrict__ latents_out) {
+                                                           float* __restrict__ latents_out,
+                                                           int32_t* __restrict__ arrivals) {
   constexpr int CPW = G / 8;       // columns per warp (8 warps cover the group)
   constexpr int BATCH = KC / 256;  // 16-byte chunks per column and lane per slice
   __shared__ __align__(16) uint16_t h_s[ROWS * KC];
   __shared__ float x_s[ROWS][G];
   __shared__ int worst;
+  __shared__ int is_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
   // this CTA's group: kept groups numbered head-major, K side then V side
@@ -501,11 +503,8 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
   __syncthreads();
   if (code_err) atomicMax(&worst, code_err);
   __syncthreads();
-  if (worst) {
-    if (blockIdx.x == 0 && tid == 0) device_error(cd->err, worst);
-    return;
-  }
-  if (tid < T) {
+  if (worst && blockIdx.x == 0 && tid == 0) device_error(cd->err, worst);
+  if (!worst && tid < T) {
     float x[G];
 #pragma unroll
     for (int k = 0; k < G; ++k) x[k] = x_s[tid][k];
@@ -527,22 +526,39 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
     put_codes<G, false>(blkw, sd_i, tau % TB, b, code);
     put_record(page + gd.sz_off, P, tau, s_h, z_h);
   }
+  // The CTA that arrives last advances the lengths: every CTA read them (to
+  // place its tokens) before it arrived, and every page write precedes the
+  // arrival of its CTA.  The counter is left at zero for the next call.
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int t = atomicAdd(arrivals, 1);
+    is_last = t == (int)gridDim.x - 1;
+    if (is_last) atomicExch(arrivals, 0);
+  }
+  __syncthreads();
+  if (is_last && !worst && tid < T && (tid == T - 1 || seq_ids[tid + 1] != seq_ids[tid]))
+    cache.lengths[seq_ids[tid]] = (int32_t)(pos + 1);
 }
 
-// Advances the lengths after a fused encode (same checks, so the same verdict).
-__global__ void __launch_bounds__(32) encode_commit_kernel(const int32_t* __restrict__ seq_ids, int T,
-                                                           const spectra_cache cache, int P) {
-  pdl_wait();  // the fused encode read the lengths before this point
-  // Triggered after the wait: the kernels after this one (a decode copies pages
-  // before its own dependency wait) start only once the fused encode's page
-  // writes are complete.
-  pdl_launch_dependents();
+// Advances the lengths of an append that writes no codes (a codec that keeps
+// no group at all), with the checks of the fused encode.
+__global__ void __launch_bounds__(32) length_advance_kernel(const int32_t* __restrict__ seq_ids, int T,
+                                                            const spectra_cache cache, int P, int32_t* err) {
+  pdl_wait();
   const int t = threadIdx.x;
   int64_t pos = 0;
-  const int err = t < T ? append_position(seq_ids, t, cache, P, &pos) : 0;
-  if (__any_sync(0xffffffffu, err != 0)) return;
+  const int e = t < T ? append_position(seq_ids, t, cache, P, &pos) : 0;
+  const int bad = __reduce_max_sync(0xffffffffu, e);
+  if (bad) {
+    if (t == 0) device_error(err, bad);
+    return;
+  }
   if (t < T && (t == T - 1 || seq_ids[t + 1] != seq_ids[t])) cache.lengths[seq_ids[t]] = (int32_t)(pos + 1);
 }
+
+cudaError_t launch_length_advance(const int32_t* seq_ids, int T, const spectra_cache& cache, int P, cudaStream_t st,
+                                  int32_t* err = nullptr);
 
 // ---------------------------------------------------------------------------
 // launchers
@@ -584,26 +600,27 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
                           (int)cache.max_pages_per_seq);
 }
 
+cudaError_t launch_length_advance(const int32_t* seq_ids, int T, const spectra_cache& cache, int P, cudaStream_t st,
+                                  int32_t* err) {
+  return launch_dependent(length_advance_kernel, dim3(1), dim3(32), 0, st, seq_ids, T, cache, P, err);
+}
+
 cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
-                                int T, const spectra_cache& cache, float* latents_out, cudaStream_t st) {
+                                int T, const spectra_cache& cache, float* latents_out, int32_t* arrivals,
+                                cudaStream_t st) {
   int n_groups = 0;
   for (int a = 0; a < h.n_kv; ++a) n_groups += h.head[a].side[0].n_groups + h.head[a].side[1].n_groups;
-  cudaError_t e = cudaSuccess;
-  if (n_groups > 0) {
-    const dim3 grid(n_groups), block(256);
-    if (h.group == 16)
-      e = T <= 1 ? launch_dependent(encode_fused_kernel<16, 1, 2048>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                                    latents_out)
-                 : launch_dependent(encode_fused_kernel<16, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T,
-                                    seq_ids, cache, latents_out);
-    else
-      e = T <= 1 ? launch_dependent(encode_fused_kernel<8, 1, 4096>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                                    latents_out)
-                 : launch_dependent(encode_fused_kernel<8, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T, seq_ids,
-                                    cache, latents_out);
-    if (e != cudaSuccess) return e;
-  }
-  return launch_dependent(encode_commit_kernel, dim3(1), dim3(32), 0, st, seq_ids, T, cache, h.P);
+  if (n_groups == 0) return launch_length_advance(seq_ids, T, cache, h.P, st, h.err);
+  const dim3 grid(n_groups), block(256);
+  if (h.group == 16)
+    return T <= 1 ? launch_dependent(encode_fused_kernel<16, 1, 2048>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                                     latents_out, arrivals)
+                  : launch_dependent(encode_fused_kernel<16, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T, seq_ids,
+                                     cache, latents_out, arrivals);
+  return T <= 1 ? launch_dependent(encode_fused_kernel<8, 1, 4096>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                                   latents_out, arrivals)
+                : launch_dependent(encode_fused_kernel<8, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T, seq_ids,
+                                   cache, latents_out, arrivals);
 }
 
 }  // namespace spectra

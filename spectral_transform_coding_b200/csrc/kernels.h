@@ -42,10 +42,12 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
                                    int T, const spectra_cache& cache, cudaStream_t st);
 
 // Fused encode for decode steps: projection, quantisation and packing in one
-// kernel per kept group, then a commit kernel that advances the lengths.
+// kernel per kept group; the CTA that arrives last (counter `arrivals`, zero
+// between calls) advances the lengths.
 constexpr int kFusedMaxT = 16;
 cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
-                                int T, const spectra_cache& cache, float* latents_out, cudaStream_t st);
+                                int T, const spectra_cache& cache, float* latents_out, int32_t* arrivals,
+                                cudaStream_t st);
 
 // reconstruct_kernels.cu: k^ = (code s + z) W_up^K, v^ likewise, for tokens
 // [t0, t0 + n) of sequence b; out of range or bad page ids -> device error INVALID

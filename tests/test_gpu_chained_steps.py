@@ -29,7 +29,7 @@ def _run(codec, P, start, H, Q, seq_ids, maxp, sync, seed):
     lat = synthetic_latents(seqs.size, codec.n_eff, seed=seed, decay=0.5, scale=2.0)
     codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
     torch.cuda.synchronize()
-    ews = torch.empty(codec.encode_workspace_bytes(H.shape[1]), dtype=torch.uint8, device=dev())
+    ews = torch.zeros(codec.encode_workspace_bytes(H.shape[1]), dtype=torch.uint8, device=dev())
     dws = torch.zeros(codec.decode_workspace_bytes(B, cache.capacity), dtype=torch.uint8, device=dev())
     out = torch.zeros_like(Q)
     stream = torch.cuda.Stream(device=dev())
