@@ -1,17 +1,22 @@
 """Decode-step benchmark of libspectra on B200.
 
 One step = one decode step through a stack of attention layers shaped like the
-named model: per layer, spectra_encode_append of the new token (projection +
-quantise + pack + append) followed by spectra_decode_attend over the whole
-latent cache.  Caches and codec factors of all layers (> L2) are resident in HBM.
+named workload: per layer, spectra_encode_append of each sequence's new token
+(projection + quantise + pack + append, one fused kernel) followed by
+spectra_decode_attend over the whole latent cache (one kernel).  Caches and codec
+factors of all layers (> L2) are resident in HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama|qwen|stress]
-                    [--impl ours|reference] [--decode latent|reconstruct] [--rope-theta T]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stress|qwen|llama]
+                    [--extra qwen,llama,prefill] [--check] [--impl ours|reference]
+                    [--decode latent|reconstruct] [--rope-theta T]
 
-Prints one JSON line (rank 0).  Metric: cache tokens/s/head = sum over layers of
-batch * context * n_kv_heads per second of step time.  ``roofline`` reports the
-decode-attention launch sequence against the measured HBM copy bandwidth over
-the packed bytes it must read.
+Prints one JSON line (rank 0).  Its top-level figures are the --workload's
+(default: the 12x heavy-tail stress layer, batch 16 at 32k context); the --extra
+workloads' records (default: Qwen-shaped 8x at 128k, Llama-shaped 4x at 32k, and
+the 65,536-token prefill encode) are nested under "workloads".  Metric: cache
+tokens/s/head = sum over layers of batch * context * n_kv_heads per second of
+step time.  ``roofline`` reports the decode kernel against the measured HBM copy
+bandwidth over the packed bytes it must read.
 """
 from __future__ import annotations
 
@@ -230,31 +235,12 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def run_gpu(args, rank, world):
-    import numpy as np
+def _activation_source(cfg, dev, gen):
+    """Seeded activations h = z sqrt(lambda) Q^T in the workload's basis (Gaussian,
+    or multivariate Student-t when the workload says so), generated on the GPU."""
     import torch
 
-    import spectral_transform_coding_b200 as st
-    from spectral_transform_coding_b200.codec import make_config
-    from workloads import get_config
     from workloads.synthetic import _basis
-
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    cfg = get_config(args.workload)
-    L = args.layers or MODEL_LAYERS[args.workload]
-    B = cfg.batch
-    ctx = cfg.cache_len
-    steps, warm = args.steps, args.warmup
-    P = cfg.page_tokens
-    cap_tokens = ctx + warm + steps + max(3, steps // 4) + 8
-    max_pages = (cap_tokens + P - 1) // P
-    c = make_config(cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head, cfg.rank, cfg.group,
-                    cfg.budget_bits, cfg.count_overhead, P)
-    gen = torch.Generator(device=dev)
-
-    # activations h = z sqrt(lambda) Q^T with the workload's basis, generated on the GPU
     basis = _basis(cfg.d_model, cfg.seed)
     lam = torch.arange(1, cfg.d_model + 1, device=dev, dtype=torch.float32) ** (-cfg.spectrum_exp)
     q1 = torch.from_numpy(basis[1]).to(dev, torch.float32)
@@ -272,15 +258,59 @@ def run_gpu(args, rank, world):
             w = torch.distributions.Chi2(torch.tensor(cfg.nu, device=dev)).sample((n,))
             h = h * torch.sqrt(cfg.nu / w)[:, None]
         return h.to(torch.bfloat16)
+    return acts
+
+
+def _calibrated_codec(cfg, acts, gen, dev, layer):
+    import torch
+
+    import spectral_transform_coding_b200 as st
+    from spectral_transform_coding_b200.codec import make_config
+    c = make_config(cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head, cfg.rank, cfg.group,
+                    cfg.budget_bits, cfg.count_overhead, cfg.page_tokens)
+    kvw = cfg.n_kv_heads * cfg.d_head
+    gen.manual_seed(1000 * cfg.seed + layer)
+    W_K = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+    W_V = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+    return st.Codec.calibrate(c, acts(cfg.calib_tokens, 7000 + layer), W_K, W_V)
+
+
+def _launches_per_layer(B, rt):
+    """Library kernels one layer of a decode step launches: the encode of B new
+    tokens is one fused kernel for B <= 16 (projection, quantise, pack, append,
+    length advance), else projection + append plan + quantise/pack; the latent
+    decode is one kernel (query fold, split-K flash-decode, merge and W_up^V lift),
+    reconstruct-then-attend is its split kernel and a combine kernel."""
+    return (1 if B <= 16 else 3) + (2 if rt else 1)
+
+
+def run_decode(args, name, world, local):
+    """Decode steps through a stack of ``layers`` calibrated layers of workload
+    ``name``; returns the JSON record of that workload."""
+    import numpy as np
+    import torch
+
+    import spectral_transform_coding_b200 as st
+    from workloads import get_config
+
+    dev = torch.device("cuda", local)
+    cfg = get_config(name)
+    L = args.layers or MODEL_LAYERS[name]
+    B = cfg.batch
+    ctx = cfg.cache_len
+    steps, warm = args.steps, args.warmup
+    P = cfg.page_tokens
+    ksteps_e2e = max(3, steps // 4)
+    # every decode step appends one token per sequence: warm-up, timed, eager
+    # end-to-end and graph end-to-end steps
+    cap_tokens = ctx + warm + steps + 2 * ksteps_e2e + 8
+    max_pages = (cap_tokens + P - 1) // P
+    gen = torch.Generator(device=dev)
+    acts = _activation_source(cfg, dev, gen)
 
     codecs, caches = [], []
-    kvw = cfg.n_kv_heads * cfg.d_head
     for l in range(L):
-        gen.manual_seed(1000 * cfg.seed + l)
-        W_K = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
-        W_V = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
-        codec = st.Codec.calibrate(c, acts(cfg.calib_tokens, 7000 + l), W_K, W_V)
-        del W_K, W_V
+        codec = _calibrated_codec(cfg, acts, gen, dev, l)
         cache = st.LatentCache(codec, batch=B, max_pages_per_seq=max_pages, device=dev, zero=False)
         chunk = 8192
         for b in range(B):
@@ -320,12 +350,13 @@ def run_gpu(args, rank, world):
             encode_layer(l)
             decode_layer(l)
 
-    # host (pinned) buffers for the end-to-end arm
+    # host (pinned) buffers of the end-to-end arms: the step's new hidden states
+    # and queries go up, its attention outputs come back
     H_host = H_new.cpu().pin_memory()
     Q_host = Q.cpu().pin_memory()
     OUT_host = torch.empty(OUT.shape, dtype=OUT.dtype).pin_memory()
 
-    def step_e2e():
+    def step_copies():
         H_new.copy_(H_host, non_blocking=True)
         Q.copy_(Q_host, non_blocking=True)
         step()
@@ -346,7 +377,7 @@ def run_gpu(args, rank, world):
         for l in range(L):
             decode_layer(l)
     with torch.cuda.graph(g_e2e, stream=stream):
-        step_e2e()
+        step_copies()
     torch.cuda.synchronize()
     for codec in codecs:
         codec.device_status()
@@ -356,55 +387,56 @@ def run_gpu(args, rank, world):
             import torch.distributed as dist
             dist.barrier()
 
-    def timed(graph, n):
+    def timed(body, n):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             a.record(stream)
             for _ in range(n):
-                graph.replay()
+                body()
             b.record(stream)
         torch.cuda.synchronize()
         barrier()
         return a.elapsed_time(b)
 
+    def eager_e2e():
+        # one step as a user runs it: eager calls through the C ABI for every
+        # layer, inputs copied up from host memory, outputs read back on the host
+        step_copies()
+        stream.synchronize()
+
     # ---- device-resident timed region: K decode steps ----
     with ClockSampler(local) as clocks:
-        total_ms = timed(g_step, steps)
+        total_ms = timed(g_step.replay, steps)
     clk = clocks.summary()
     len_after = int(caches[0].lengths.float().mean().item())
     # ---- decode-attention launches alone (same kernels, same resident caches) ----
-    dec_ms = timed(g_dec, steps) / (steps * L)
-    # ---- end-to-end: host buffers, copies inside the timed region ----
-    ksteps_e2e = max(3, steps // 4)
-    e2e_ms = timed(g_e2e, ksteps_e2e) / ksteps_e2e
+    dec_ms = timed(g_dec.replay, steps) / (steps * L)
+    # ---- end to end: eager per-step calls with host buffers; graph replay of the same ----
+    e2e_ms = timed(eager_e2e, ksteps_e2e) / ksteps_e2e
+    e2e_graph_ms = timed(g_e2e.replay, ksteps_e2e) / ksteps_e2e
     for codec in codecs:
         codec.device_status(stream)
     ms_per_step = total_ms / steps
     if world > 1:
-        ms_per_step, e2e_ms, dec_ms = max_over_ranks([ms_per_step, e2e_ms, dec_ms], dev)
+        ms_per_step, e2e_ms, e2e_graph_ms, dec_ms = max_over_ranks([ms_per_step, e2e_ms, e2e_graph_ms, dec_ms], dev)
     mean_ctx = (len0 + len_after) / 2.0
     tok_per_step = L * B * mean_ctx * cfg.n_kv_heads
     value = replicas_throughput(tok_per_step, ms_per_step, world)
     e2e_value = replicas_throughput(tok_per_step, e2e_ms, world)
+    e2e_graph_value = replicas_throughput(tok_per_step, e2e_graph_ms, world)
 
-    # roofline: packed bytes the decode reads per layer.  traffic: DRAM bytes
-    # (read + write) of one split_kernel launch per algorithmic byte, from one ncu
-    # capture of the 1-layer Llama-shaped case at 32k context (33,707,520 B for
-    # 32,772 tokens x 1,024 B); only workloads with a capture of the current kernel
-    # have one, else traffic is null.
+    # roofline of the decode kernel: the packed bytes one launch must read (every
+    # token of every sequence of the layer, all KV heads) over its average launch
+    # time, launches timed back to back over resident caches of all layers
     bytes_per_tok_all_heads = codecs[0].page_bytes / P
     dec_bytes = B * len_after * bytes_per_tok_all_heads
-    dec_avg_ms = dec_ms
     peaks = _peaks()
-    achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
-    # encode: fused projection/quantise/pack + commit for steps of <= 16 tokens,
-    # else projection + append plan + quantise/pack; decode: fold, split, combine
-    # (reconstruct-then-attend: split, combine)
-    launches_per_layer = (2 if B <= 16 else 3) + (2 if rt else 3)
-    h2d = H_new.numel() * 2 + Q.numel() * 4
-    d2h = OUT.numel() * 4
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    h2d = H_new.numel() * H_new.element_size() + Q.numel() * Q.element_size()
+    d2h = OUT.numel() * OUT.element_size()
+    check = _self_check(codecs[0], caches[0], Q[0], OUT[0], stream) if args.check else None
 
     result = {
         "metric": "latent-KV decode attention: cache tokens/s/head",
@@ -427,20 +459,28 @@ def run_gpu(args, rank, world):
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
-            "kernel": "split_kernel (latent flash-decode over the packed pages), timed with its fold and combine "
-                      "launches chained by programmatic dependent launch",
+            "kernel": "attend_kernel (query fold, split-K latent flash-decode over the packed pages, "
+                      "last-CTA merge and W_up^V lift in one launch)",
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"],
-            "traffic": (TRAFFIC_PER_ALGO_BYTE[args.workload] * dec_bytes
-                        if args.workload in TRAFFIC_PER_ALGO_BYTE else None),
-            "peak_src": peaks["src"], "avg_launch_us": dec_avg_ms * 1e3,
+            "traffic": (TRAFFIC_PER_ALGO_BYTE[name] * dec_bytes if name in TRAFFIC_PER_ALGO_BYTE else None),
+            "peak_src": peaks["src"], "avg_launch_us": dec_ms * 1e3,
             "algorithmic_bytes_per_launch": dec_bytes,
+            "timing": "decode launches of all layers replayed back to back (CUDA graph, PDL chained), "
+                      "CUDA events on the launching stream",
         },
         "e2e": {"value": e2e_value, "unit": "tokens/s/head", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_layer * L * steps,
+                "d2h_bytes_per_step": d2h,
+                "how": "eager per-step calls through the C ABI (encode_append + decode_attend per layer), "
+                       "inputs copied from pinned host memory, outputs copied back and the host synchronised "
+                       "on them every step"},
+        "e2e_graph": {"value": e2e_graph_value, "unit": "tokens/s/head", "ms_per_step": e2e_graph_ms,
+                      "how": "the same step with its copies captured once in a CUDA graph and replayed"},
+        "gpu_launches": _launches_per_layer(B, rt) * L * steps,
         "clocks": clk,
     }
+    if check is not None:
+        result["check"] = check
     if rt:
         # algorithmic FLOPs per (token, KV head) = 2 n_kept_K d_h (lift) + 2 gq d_h
         # (scores) + 2 gq n_kept_V (probability-weighted V latents), summed over the
@@ -453,77 +493,79 @@ def run_gpu(args, rank, world):
                        + 2 * gq * cfg.group * int((w[1] > 0).sum()) for w in widths)
         flops = B * len_after * flop_tok
         alu_peak = 148 * 128 * 2 * 1965e6 / 1e12
-        tflops = flops / (dec_avg_ms / 1e3) / 1e12
+        tflops = flops / (dec_ms / 1e3) / 1e12
         result["config"]["decode"] = f"reconstruct-then-attend, rotary base {args.rope_theta:g}"
         result["dtype"] = "u8 codes, fp16 scale/zero, fp32 lift and accumulate"
         result["roofline"] = {
             "kernel": "rt_split_kernel (keys rebuilt per 32-token tile on the tensor cores, rotated and scored "
                       "with fp32 FMAs; V summed in the latent space), timed with its combine launch",
             "bound": "alu", "achieved": tflops, "peak": alu_peak, "unit": "TFLOP/s", "frac": tflops / alu_peak,
-            "traffic": (TRAFFIC_PER_PACKED_BYTE_RT[args.workload] * dec_bytes
-                        if args.workload in TRAFFIC_PER_PACKED_BYTE_RT else None),
+            "traffic": (TRAFFIC_PER_PACKED_BYTE_RT[name] * dec_bytes if name in TRAFFIC_PER_PACKED_BYTE_RT
+                        else None),
             "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm)",
-            "avg_launch_us": dec_avg_ms * 1e3, "algorithmic_flops_per_launch": flops,
+            "avg_launch_us": dec_ms * 1e3, "algorithmic_flops_per_launch": flops,
             "packed_bytes_per_launch": dec_bytes,
+            "hbm_gbs": achieved, "hbm_frac": achieved / peaks["hbm_gbs"],
         }
+    del g_step, g_dec, g_e2e, codecs, caches
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return result
 
 
-def run_prefill(args):
-    """Prefill encode (one 65,536-token bf16 chunk for all KV heads, 4x and 8x
-    budgets), then one decode step: encode tokens/s, the tensor-core projection's
-    TFLOP/s and the quantise/pack kernel's GB/s.  One JSON line per budget."""
+def _self_check(codec, cache, q, out, stream):
+    """Opt-in self-consistency check after timing: the latent decode of layer 0
+    against reconstruct-then-attend without rotation over the same pages (a second
+    kernel that rebuilds keys and values from the codes and attends over them; the
+    two agree to rounding).  The element-wise checks against the CPU oracle at
+    these shapes live in the GPU test suite."""
+    import torch
+    torch.cuda.synchronize()
+    a = codec.decode_attend(cache, q)
+    b = codec.decode_attend_reconstruct(cache, q, rope_theta=0.0)
+    codec.device_status()
+    a64, b64 = a.double(), b.double()
+    err = ((a64 - b64).abs().amax(dim=-1) / b64.abs().amax(dim=-1).clamp_min(1e-30)).max().item()
+    return {"what": "layer 0: latent decode vs reconstruct-then-attend (no rotation), all sequences and q heads",
+            "max_rel_err": err, "bar": 2e-3, "ok": bool(err <= 2e-3)}
+
+
+def run_prefill(args, local):
+    """Prefill encode of one 65,536-token bf16 chunk for all KV heads of the
+    Llama-shaped layer at 4x and 8x, then one decode step over it.  Per budget:
+    encode tokens/s and TFLOP/s (projection GEMM with the quantiser in its
+    epilogue), for comparison the projection alone and the separate quantise/pack
+    kernel on its fp32 latents, and the decode after it."""
     import torch
 
     import spectral_transform_coding_b200 as st
-    from spectral_transform_coding_b200.codec import make_config
     from workloads import get_config
-    from workloads.synthetic import _basis
 
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
+    dev = torch.device("cuda", local)
     peaks = _peaks()
     out = []
     for name in ("prefill", "prefill8"):
         cfg = get_config(name)
         T, P = args.prefill_tokens or cfg.prefill_tokens, cfg.page_tokens
         gen = torch.Generator(device=dev)
-        basis = _basis(cfg.d_model, cfg.seed)
-        lam = torch.arange(1, cfg.d_model + 1, device=dev, dtype=torch.float32) ** (-cfg.spectrum_exp)
-        q1 = torch.from_numpy(basis[1]).to(dev, torch.float32)
-        q2 = torch.from_numpy(basis[2]).to(dev, torch.float32) if basis[0] == "kron" else None
-
-        def acts(n, seed):
-            gen.manual_seed(seed)
-            y = torch.randn((n, cfg.d_model), generator=gen, device=dev) * lam.sqrt()
-            if q2 is None:
-                h = y @ q1.T
-            else:
-                a_, b_ = q1.shape[0], q2.shape[0]
-                h = torch.einsum("ia,nab,jb->nij", q1, y.view(n, a_, b_), q2).reshape(n, a_ * b_)
-            return h.to(torch.bfloat16)
-
-        c = make_config(cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head, cfg.rank, cfg.group,
-                        cfg.budget_bits, cfg.count_overhead, P)
-        kvw = cfg.n_kv_heads * cfg.d_head
-        gen.manual_seed(1000 * cfg.seed)
-        W_K = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
-        W_V = (torch.randn((cfg.d_model, kvw), generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
-        codec = st.Codec.calibrate(c, acts(cfg.calib_tokens, 7000), W_K, W_V)
-        del W_K, W_V
+        acts = _activation_source(cfg, dev, gen)
+        codec = _calibrated_codec(cfg, acts, gen, dev, 0)
         H = acts(T, 12345)
         cache = st.LatentCache(codec, batch=1, max_pages_per_seq=(T + P - 1) // P + 1, device=dev, zero=False)
         seq = torch.zeros(T, dtype=torch.int32, device=dev)
         ws = torch.zeros(codec.encode_workspace_bytes(T), dtype=torch.uint8, device=dev)
         lat = torch.empty((T, codec.n_eff), dtype=torch.float32, device=dev)
         stream = torch.cuda.Stream(device=dev)
+        gen.manual_seed(77)
         q = (torch.randn((1, cfg.n_q_heads, cfg.d_head), generator=gen, device=dev) * 0.5).contiguous()
         o = torch.empty_like(q)
         dws = torch.zeros(codec.decode_workspace_bytes(1, cache.capacity), dtype=torch.uint8, device=dev)
 
         def timed(fn, reps):
+            # each repetition encodes the chunk into an emptied cache; the chunk and
+            # its latents (0.5 + 0.5 GB at 4x) exceed L2
             tot = 0.0
-            for r in range(reps + 2):
+            for r in range(reps + 3):
                 cache.lengths.zero_()
                 torch.cuda.synchronize()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -532,14 +574,16 @@ def run_prefill(args):
                     fn()
                     e1.record(stream)
                 torch.cuda.synchronize()
-                if r >= 2:
+                if r >= 3:
                     tot += e0.elapsed_time(e1)
             return tot / reps
 
         reps = max(3, min(args.steps, 10))
-        t_enc = timed(lambda: codec.encode_append(cache, H, seq, workspace=ws, stream=stream), reps)
-        t_proj = timed(lambda: codec.project(H, out=lat, stream=stream), reps)
-        t_quant = timed(lambda: codec.quantize_append(cache, lat, seq, workspace=ws, stream=stream), reps)
+        with ClockSampler(local) as clocks:
+            t_enc = timed(lambda: codec.encode_append(cache, H, seq, workspace=ws, stream=stream), reps)
+            t_proj = timed(lambda: codec.project(H, out=lat, stream=stream), reps)
+            t_quant = timed(lambda: codec.quantize_append(cache, lat, seq, workspace=ws, stream=stream), reps)
+        clk = clocks.summary()
         cache.lengths.zero_()
         codec.encode_append(cache, H, seq, workspace=ws, stream=stream)  # leave the cache full for decode
         torch.cuda.synchronize()
@@ -555,72 +599,93 @@ def run_prefill(args):
         t_dec = e0.elapsed_time(e1) / 10
         codec.device_status(stream)
         flops = 2.0 * cfg.d_model * codec.n_eff * T
-        qbytes = T * (4.0 * codec.n_eff + codec.page_bytes / P)
-        tfl = flops / (t_proj / 1e3) / 1e12
-        gbs = qbytes / (t_quant / 1e3) / 1e9
+        packed = T * codec.page_bytes / P
+        qbytes = T * 4.0 * codec.n_eff + packed
+        bf16 = peaks["bf16_tflops"]
         out.append({
             "metric": "prefill encode-append tokens/s", "value": T / (t_enc / 1e3), "unit": "tokens/s",
             "workload": f"{name}: {T} tokens x (d_model {cfg.d_model}, {cfg.n_kv_heads} kv heads, "
                         f"{cfg.budget_bits} bits/side), one chunk, then one decode step",
-            "encode_ms": t_enc, "n_eff": codec.n_eff,
-            "projection": {"ms": t_proj, "tflops": tfl, "peak": peaks["bf16_tflops"],
-                           "frac": tfl / peaks["bf16_tflops"], "kernel": "gemm_tcgen05_kernel (bf16, fp32 out)"},
-            "quantize_pack": {"ms": t_quant, "gbs": gbs, "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
-                              "bytes": qbytes},
-            "decode_after_us": t_dec * 1e3, "peak_src": peaks["src"],
+            "n_eff": codec.n_eff, "packed_bytes": packed,
+            "encode": {"ms": t_enc, "tflops": flops / (t_enc / 1e3) / 1e12, "peak": bf16,
+                       "frac": flops / (t_enc / 1e3) / 1e12 / bf16, "latent_bytes_written": 0,
+                       "kernels": "append_plan_kernel, then encode_gemm_kernel (tcgen05 projection with "
+                                  "quantise/pack/append in its epilogue)"},
+            "projection_only": {"ms": t_proj, "tflops": flops / (t_proj / 1e3) / 1e12, "peak": bf16,
+                                "frac": flops / (t_proj / 1e3) / 1e12 / bf16,
+                                "kernel": "gemm_tcgen05_kernel (bf16 in, fp32 latents out)"},
+            "unfused_quantize_pack": {"ms": t_quant, "gbs": qbytes / (t_quant / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                                      "frac": qbytes / (t_quant / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes": qbytes,
+                                      "kernels": "append_plan_kernel + quantize_append_kernel on fp32 latents"},
+            "decode_after_us": t_dec * 1e3, "peak_src": peaks["src"], "clocks": clk,
         })
-    for r in out:
-        print(json.dumps(r), flush=True)
-    return 0
+        del codec, cache, H, lat, ws, dws
+        torch.cuda.empty_cache()
+    return out
+
+
+def _reference_line(args, name):
+    """The CPU oracle as the reference arm on ``name``'s configuration."""
+    from workloads import get_config
+    cfg = get_config(name)
+    rt = args.decode == "reconstruct"
+    value, ms, cores, sample = cpu_oracle_steps(cfg, args.steps, args.warmup,
+                                                rope_theta=args.rope_theta if rt else None)
+    L = args.layers or MODEL_LAYERS[name]
+    return {
+        "impl": "reference", "metric": "latent-KV decode attention: cache tokens/s/head", "value": value,
+        "unit": "tokens/s/head", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": dict({"workload": _workload_name(cfg, L)},
+                       **({"decode": f"reconstruct-then-attend, rotary base {args.rope_theta:g}"} if rt else {})),
+        "cpu_baseline": {"value": value, "unit": "tokens/s/head", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s/head", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="llama", choices=sorted(MODEL_LAYERS) + ["prefill"])
-    ap.add_argument("--layers", type=int, default=0)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="stress", choices=sorted(MODEL_LAYERS),
+                    help="the workload of the line's top-level figures")
+    ap.add_argument("--extra", default="qwen,llama,prefill",
+                    help="comma-separated workloads measured after it and nested in the same line "
+                         "(decode workloads and/or 'prefill'; empty for none)")
+    ap.add_argument("--layers", type=int, default=0, help="layers per decode workload (default: the model's)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--check", action="store_true",
+                    help="after timing, check layer 0's decode against reconstruct-then-attend")
     ap.add_argument("--decode", default="latent", choices=["latent", "reconstruct"],
                     help="decode attention: in the latent space (default) or over keys rebuilt per tile")
     ap.add_argument("--rope-theta", type=float, default=500000.0,
                     help="reconstruct decode: rotary base (0 = no rotation)")
     ap.add_argument("--prefill-tokens", type=int, default=0,
-                    help="prefill mode: tokens in the chunk (default: the workload's 65,536)")
+                    help="prefill: tokens in the chunk (default: the workload's 65,536)")
     args = ap.parse_args()
+    if args.impl == "ours" and args.warmup < 3:
+        ap.error("--warmup must be at least 3")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    from workloads import get_config
-    if args.workload == "prefill":
-        if args.impl == "reference" or rank != 0:
-            return 0
-        return run_prefill(args)
-    cfg = get_config(args.workload)
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    extras = [e for e in args.extra.split(",") if e]
+    for e in extras:
+        if e != "prefill" and e not in MODEL_LAYERS:
+            ap.error(f"unknown workload {e!r}")
 
     if args.impl == "reference":
-        if rank != 0:
-            return 0
-        rt = args.decode == "reconstruct"
-        value, ms, cores, sample = cpu_oracle_steps(cfg, args.steps, args.warmup,
-                                                    rope_theta=args.rope_theta if rt else None)
-        L = args.layers or MODEL_LAYERS[args.workload]
-        out = {
-            "impl": "reference", "metric": "latent-KV decode attention: cache tokens/s/head", "value": value,
-            "unit": "tokens/s/head", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": dict({"workload": _workload_name(cfg, L)},
-                           **({"decode": f"reconstruct-then-attend, rotary base {args.rope_theta:g}"} if rt else {})),
-            "cpu_baseline": {"value": value, "unit": "tokens/s/head", "cores": cores, "kind": "oracle",
-                             "sample": sample},
-            "e2e": {"value": value, "unit": "tokens/s/head", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        }
-        print(json.dumps(out), flush=True)
+        if rank == 0:
+            print(json.dumps(_reference_line(args, args.workload)), flush=True)
         return 0
 
+    from workloads import get_config
+    import torch
+    torch.cuda.set_device(local)
     if world > 1:
         import datetime
 
@@ -628,12 +693,23 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(cfg, rope_theta=args.rope_theta if args.decode == "reconstruct" else None)
-    res = run_gpu(args, rank, world)
+        cpu = cpu_oracle_sample(get_config(args.workload),
+                                rope_theta=args.rope_theta if args.decode == "reconstruct" else None)
+    res = run_decode(args, args.workload, world, local)
+    nested = {}
+    for e in extras:
+        if e == "prefill":
+            nested["prefill"] = run_prefill(args, local)
+        elif e != args.workload:
+            r = run_decode(args, e, world, local)
+            nested[e] = {k: r[k] for k in ("value", "unit", "ms_per_step", "config", "roofline", "e2e",
+                                           "e2e_graph", "gpu_launches", "clocks", "check") if k in r}
     if rank == 0:
         if cpu is not None:
             res["cpu_baseline"] = {"value": cpu[0], "unit": "tokens/s/head", "cores": cpu[1], "kind": "oracle",
                                    "sample": cpu[2]}
+        if nested:
+            res["workloads"] = nested
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist

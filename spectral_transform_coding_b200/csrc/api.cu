@@ -117,13 +117,16 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
   for (int a = 0; a < cfg.n_kv_heads; ++a)
     kept_total += 2 * (size_t)c->h.head[a].side[0].n_kept + c->h.head[a].side[1].n_kept;
   const size_t wu_bytes = std::max<size_t>(kept_total * dh * 4, 4);
-  const size_t total = off_wu + wu_bytes;
+  const size_t off_cg = off_wu + (wu_bytes + 255) / 256 * 256;
+  const size_t n_cg = std::max<size_t>((size_t)n_eff / cfg.group, 1);
+  const size_t total = off_cg + n_cg * 16;
   CUDA_TRY(cudaMalloc(&c->dmem, total));
   uint8_t* base = static_cast<uint8_t*>(c->dmem);
   c->err = reinterpret_cast<int32_t*>(base + off_err);
   c->h.err = c->err;
   c->h.wt_down = reinterpret_cast<const uint16_t*>(base + off_wt);
   c->h.w_up = reinterpret_cast<const float*>(base + off_wu);
+  c->h.col_groups = reinterpret_cast<const int32_t*>(base + off_cg);
   c->d = reinterpret_cast<CodecDev*>(base);
 
   std::vector<uint16_t> wt((size_t)c->h.n_eff_pad * dm, 0);
@@ -149,16 +152,32 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
         }
       }
     }
+  // groups of G latent columns (head-major, K then V, kept groups ascending):
+  // {width, code block offset, scale/zero offset, side} for the GEMM epilogue
+  std::vector<int32_t> cg(n_cg * 4, 0);
+  for (int a = 0; a < cfg.n_kv_heads; ++a)
+    for (int s = 0; s < 2; ++s) {
+      const SideDev& sd = c->h.head[a].side[s];
+      for (int j = 0; j < sd.n_groups; ++j) {
+        const size_t g = (size_t)(sd.c_col0 + sd.grp[j].col) / cfg.group;
+        cg[4 * g] = sd.grp[j].b;
+        cg[4 * g + 1] = sd.grp[j].plane_off;
+        cg[4 * g + 2] = sd.grp[j].sz_off;
+        cg[4 * g + 3] = s;
+      }
+    }
   CUDA_TRY(cudaMemset(c->dmem, 0, off_wt));
   CUDA_TRY(cudaMemcpy(base, &c->h, sizeof(CodecDev), cudaMemcpyHostToDevice));
   CUDA_TRY(cudaMemcpy(base + off_wt, wt.data(), wt.size() * 2, cudaMemcpyHostToDevice));
   CUDA_TRY(cudaMemcpy(base + off_wu, wu.data(), wu.size() * 4, cudaMemcpyHostToDevice));
+  CUDA_TRY(cudaMemcpy(base + off_cg, cg.data(), cg.size() * 4, cudaMemcpyHostToDevice));
   *out = c.release();
   return SPECTRA_OK;
 }
 
 // Encode workspace: [arrival counter of the fused path, 256 B][positions][flag][latents].
 constexpr size_t kEncCounterBytes = 256;
+constexpr int64_t kGemmMinT = 64;  // rows from which the projection runs on the tcgen05 GEMM
 size_t encode_ws_bytes(const spectra_codec* c, int64_t T) {
   const size_t pos = ((size_t)std::max<int64_t>(T, 1) * 4 + 255) / 256 * 256;
   const size_t flag = 256;
@@ -179,7 +198,7 @@ spectra_status check_cache(const spectra_codec* c, const spectra_cache* cache) {
 spectra_status do_project(const spectra_codec* c, const void* H, int64_t T, float* C, cudaStream_t st) {
   // T >= 64 rows: tcgen05 tensor-core GEMM; fewer rows: the projection is a
   // weight-streaming GEMV bounded by HBM, done on CUDA cores.
-  if (T >= 64) {
+  if (T >= kGemmMinT) {
     CUDA_TRY(launch_project_tcgen05(c->h, c->h.wt_down, static_cast<const uint16_t*>(H), (int)T, C,
                                     c->h.n_eff, st));
   } else {
@@ -640,6 +659,17 @@ spectra_status spectra_encode_append(const spectra_codec* c, const spectra_cache
     // decode steps: projection, quantisation and packing fused per kept group
     CUDA_TRY(launch_encode_fused(c->h, c->d, static_cast<const uint16_t*>(H), seq_ids, (int)T, *cache,
                                  latents_out, static_cast<int32_t*>(workspace), st));
+    return SPECTRA_OK;
+  }
+  if (!latents_out && T >= kGemmMinT) {
+    // prefill: the append plan, then the projection GEMM with quantise/pack in
+    // its epilogue (no fp32 latents in memory)
+    uint8_t* w = static_cast<uint8_t*>(workspace) + kEncCounterBytes;
+    int32_t* pos = reinterpret_cast<int32_t*>(w);
+    int32_t* flag = reinterpret_cast<int32_t*>(w + ((size_t)T * 4 + 255) / 256 * 256);
+    CUDA_TRY(launch_append_plan(seq_ids, (int)T, *cache, c->cfg.page_tokens, pos, flag, c->err, st));
+    CUDA_TRY(launch_encode_gemm(c->h, c->d, static_cast<const uint16_t*>(H), (int)T, seq_ids, pos, flag, *cache,
+                                st));
     return SPECTRA_OK;
   }
   uint8_t* w = static_cast<uint8_t*>(workspace);

@@ -905,27 +905,49 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     bulk_copy_g2s(wv_s, cd->w_up + hm[7], wv_bytes, &bars[kMaxStages]);
   }
   float* wts = reinterpret_cast<float*>(smem + kOffQlat);   // [gq][kMaxSplit] weights (q_lat is dead)
-  float* acc = reinterpret_cast<float*>(smem + kOffX);      // [gq][kMaxKept] merged latent sums
+  float* part = reinterpret_cast<float*>(smem + kOffX);     // [ch][gq][4 n4] partial merges
   float* lsum = reinterpret_cast<float*>(smem + kOffW);     // [gq] sum of weights x l
   const size_t hs = (size_t)gq * A.rec_stride;              // floats between splits' records
+  // thread (chunk k, head h, 4 consecutive coordinates c4) sums splits k, k + ch,
+  // ... of the records; the chunks are added in order afterwards (a fixed order)
+  const int n4 = (nkV + 3) / 4;
+  const int pairs = gq * n4;
+  int ch = pairs > 0 ? kThreads / pairs : 1;
+  ch = ch < ns ? ch : ns;
+  const int ch_cap = pairs > 0 ? (kXBytes / 16) / pairs : 1;
+  ch = ch < ch_cap ? ch : ch_cap;
+  ch = ch > 1 ? ch : 1;
+  const int pr = pairs > 0 ? tid % pairs : 0, k = pairs > 0 ? tid / pairs : ch;
+  const bool act = k < ch;
+  const int hh = pairs > 0 ? pr / n4 : 0, c4 = pairs > 0 ? pr - hh * n4 : 0;
+  const int nsp = act ? (ns - k + ch - 1) / ch : 0;  // splits of this thread
+  const float4* xb = reinterpret_cast<const float4*>(recs + (size_t)hh * A.rec_stride + 4) + c4;
+  // the first 16 of this thread's records are loaded while the weights are formed
+  float4 x[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u)
+    x[u] = u < nsp ? __ldcg(xb + (size_t)(k + u * ch) * (hs / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
   if (warp < gq) {  // warp h: the maximum and the weights of the splits for head h
     const int h = warp;
+    float2 ml[kMaxSplit / 32];
     float M = -CUDART_INF_F;
-    for (int s0 = 0; s0 < ns; s0 += 32) {
-      const int sp = s0 + lane;
-      const float m = sp < ns ? __ldcg(recs + sp * hs + h * A.rec_stride) : -CUDART_INF_F;
-      M = fmaxf(M, m);
+#pragma unroll
+    for (int r = 0; r < kMaxSplit / 32; ++r) {
+      const int sp = lane + 32 * r;
+      ml[r] = sp < ns ? __ldcg(reinterpret_cast<const float2*>(recs + sp * hs + h * A.rec_stride))
+                      : make_float2(-CUDART_INF_F, 0.f);
+      M = fmaxf(M, ml[r].x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Ls = 0.f;
-    for (int s0 = 0; s0 < ns; s0 += 32) {
-      const int sp = s0 + lane;
+#pragma unroll
+    for (int r = 0; r < kMaxSplit / 32; ++r) {
+      const int sp = lane + 32 * r;
       if (sp < ns) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(recs + sp * hs + h * A.rec_stride));
-        const float wt = (ml.x == -CUDART_INF_F) ? 0.f : ex2_approx(ml.x - M);
+        const float wt = (ml[r].x == -CUDART_INF_F) ? 0.f : ex2_approx(ml[r].x - M);
         wts[h * kMaxSplit + sp] = wt;
-        Ls = fmaf(wt, ml.y, Ls);
+        Ls = fmaf(wt, ml[r].y, Ls);
       }
     }
 #pragma unroll
@@ -933,33 +955,46 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     if (lane == 0) lsum[h] = Ls;
   }
   __syncthreads();
-  // thread (h, 4 consecutive coordinates): the splits' records, 16 loads in flight
-  for (int e = tid; e < gq * (kMaxKept / 4); e += kThreads) {
-    const int h = e / (kMaxKept / 4), c4 = e - h * (kMaxKept / 4);
-    if (4 * c4 >= nkV) continue;
+  if (act) {
+    const float* wt = wts + hh * kMaxSplit + k;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float* base = recs + h * A.rec_stride + 4;
-    for (int s0 = 0; s0 < ns; s0 += 16) {
-      float4 x[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float w = u < nsp ? wt[u * ch] : 0.f;
+      v.x = fmaf(w, x[u].x, v.x);
+      v.y = fmaf(w, x[u].y, v.y);
+      v.z = fmaf(w, x[u].z, v.z);
+      v.w = fmaf(w, x[u].w, v.w);
+    }
+    for (int u0 = 16; u0 < nsp; u0 += 16) {
 #pragma unroll
       for (int u = 0; u < 16; ++u)
-        x[u] = s0 + u < ns ? __ldcg(reinterpret_cast<const float4*>(base + (s0 + u) * hs) + c4)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u] = u0 + u < nsp ? __ldcg(xb + (size_t)(k + (u0 + u) * ch) * (hs / 4))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        const float wt = s0 + u < ns ? wts[h * kMaxSplit + s0 + u] : 0.f;
-        v.x = fmaf(wt, x[u].x, v.x);
-        v.y = fmaf(wt, x[u].y, v.y);
-        v.z = fmaf(wt, x[u].z, v.z);
-        v.w = fmaf(wt, x[u].w, v.w);
+        const float w = u0 + u < nsp ? wt[(u0 + u) * ch] : 0.f;
+        v.x = fmaf(w, x[u].x, v.x);
+        v.y = fmaf(w, x[u].y, v.y);
+        v.z = fmaf(w, x[u].z, v.z);
+        v.w = fmaf(w, x[u].w, v.w);
       }
     }
-    reinterpret_cast<float4*>(acc + h * kMaxKept)[c4] = v;
+    reinterpret_cast<float4*>(part)[(size_t)k * pairs + pr] = v;
   }
   bool wv_ok = true;
   if (wv_staged && wv_bytes > 0) wv_ok = mbar_wait_bounded(&bars[kMaxStages], 0u, kWaitLimitNs);
   if (!wv_ok && tid == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
   __syncthreads();
+  // chunks added in order into chunk 0: acc[h][c] = part[h * 4 n4 + c]
+  for (int e = tid; e < pairs * 4; e += kThreads) {
+    float v = part[e];
+    for (int kk = 1; kk < ch; ++kk) v += part[(size_t)kk * pairs * 4 + e];
+    part[e] = v;
+  }
+  __syncthreads();
+  const float* acc = part;
+  const int acc_ld = 4 * n4;
   // out = (merged latent sums / L) W_up^V: thread (h, 4 consecutive dims)
   const float* wv = wv_staged ? wv_s : cd->w_up + hm[7];
   for (int e = tid; e < gq * (d_h / 4); e += kThreads) {
@@ -967,7 +1002,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (wv_ok) {
       for (int c = 0; c < nkV; ++c) {
-        const float x = acc[h * kMaxKept + c];
+        const float x = acc[h * acc_ld + c];
         const float4 w = reinterpret_cast<const float4*>(wv + (size_t)c * d_h)[d4];
         v.x = fmaf(x, w.x, v.x);
         v.y = fmaf(x, w.y, v.y);

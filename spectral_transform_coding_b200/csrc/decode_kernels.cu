@@ -13,22 +13,22 @@
 // split into fp16 hi + lo columns so scores keep ~22 bits; the z terms are two
 // more MMAs per 16-token tile.
 //
-// One kernel per decode step (attend_kernel).  Its grid is (context split,
-// KV head, sequence), in thread-block clusters of CL consecutive splits of one
-// (sequence, KV head):
+// One kernel per decode step (attend_kernel, attend_kernel.cuh); this file holds
+// its host side: the launch plan and the launch.  The grid is (context split,
+// KV head, sequence), one CTA per split:
 //   prologue (before the dependency wait; reads only the caller's q, read-only
 //     codec data, the lengths as a hint and pages that are full under the hint):
 //     bulk copies of the first pages into a CTA-wide ring of shared-memory
-//     stages; each CTA of the cluster folds its slice of the kept K coordinates
-//     (q_lat = q W_up^K^T) and the cluster exchanges the slices through
-//     distributed shared memory; the MMA B fragments of q_lat are built;
+//     stages; the fold q_lat = q W_up^K^T of all kept K coordinates; the MMA B
+//     fragments of q_lat;
 //   main loop (after the wait): 8 warps take the CTA's pages in turn and stream
 //     them through an online softmax, one page (64 tokens) per step;
-//   merges: the warps of a CTA, then the CTAs of the cluster (through
-//     distributed shared memory; each CTA lifts its slice of the value
-//     coordinates with W_up^V), then, when a sequence needs several clusters,
-//     the last cluster to finish (an arrival counter in the workspace) merges
-//     the clusters' records in a fixed order.
+//   merges: the warps of a CTA into one record per q head in the workspace;
+//     the last CTA of a (sequence, KV head) to arrive (a self-resetting counter
+//     in the workspace) merges the splits' records in split order and lifts the
+//     value latents with W_up^V.
+// The split partition (page i of a sequence goes to split i mod n_split) and the
+// merge order depend only on the final length, so results are deterministic.
 #include <cuda_runtime.h>
 
 #include <algorithm>

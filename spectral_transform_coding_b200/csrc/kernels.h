@@ -93,6 +93,11 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
                           cudaStream_t st);
 
 // gemm_sm100.cu (tcgen05)
+// Prefill encode: projection GEMM with quantise/pack/append in its epilogue;
+// positions and the plan's flag from launch_append_plan (launched before it).
+cudaError_t launch_encode_gemm(const CodecDev& h, const CodecDev* d, const uint16_t* H, int T,
+                               const int32_t* seq_ids, const int32_t* pos, const int32_t* ok_flag,
+                               const spectra_cache& cache, cudaStream_t st);
 cudaError_t launch_project_tcgen05(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
                                    float* C, int64_t ldc, cudaStream_t st);
 cudaError_t launch_gram_tcgen05(const uint16_t* H, int64_t n_tokens, int d_model, float* G,

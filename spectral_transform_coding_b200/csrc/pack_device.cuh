@@ -1,0 +1,162 @@
+// Per-token group quantiser and the packed page writer of libspectra, shared by
+// the encode kernels (quantise/pack after a separate projection, the fused
+// decode-step encode, and the projection GEMM with the quantiser in its
+// epilogue), so that every encode route writes the same bits.
+//
+// Quantiser ("SPECTRA pipeline" stage 2: groups of adjacent latent coordinates
+// share one width; stage 3: tokens are quantised per token): per token and
+// group of G fp32 latents at width b, every step one IEEE fp32 operation,
+//   s = fp16(sat((max - min) / (2^b - 1))), z = fp16(sat(min)),
+//   code = clamp(rint((x - z) / s), 0, 2^b - 1), all codes 0 when s == 0.
+// Page writer: code bits at the canonical (word, bit) addresses of the page
+// layout (fragment position of the entry, then the width rule), scale/zero
+// records per token pair.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+namespace spectra {
+namespace pack {
+
+__device__ __forceinline__ float sat16(float x) { return fminf(fmaxf(x, -65504.f), 65504.f); }
+
+// One token's group of G fp32 latents at width b (every step one IEEE fp32
+// operation): s = fp16(sat((max - min) / (2^b - 1))), z = fp16(sat(min)),
+// code = clamp(rint((x - z) / s), 0, 2^b - 1), all codes 0 when s == 0.
+template <int G>
+__device__ __forceinline__ void quantize_group(const float (&x)[G], int b, __half& s_h, __half& z_h,
+                                               uint32_t (&code)[G]) {
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int k = 1; k < G; ++k) {
+    mn = fminf(mn, x[k]);
+    mx = fmaxf(mx, x[k]);
+  }
+  const float levels = (float)((1 << b) - 1);
+  s_h = __float2half_rn(sat16(__fdiv_rn(__fsub_rn(mx, mn), levels)));
+  z_h = __float2half_rn(sat16(mn));
+  const float sf = __half2float(s_h), zf = __half2float(z_h);
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    float c = 0.f;
+    if (sf > 0.f) {
+      const float t = __fdiv_rn(__fsub_rn(x[k], zf), sf);
+      c = fminf(fmaxf(rintf(t), 0.f), levels);
+    }
+    code[k] = (uint32_t)c;
+  }
+}
+
+// Fragment position (gid, t4, slot) of entry (token tb of the block, coordinate k).
+template <int G>
+__device__ __forceinline__ void k_side_pos(int tb, int k, int* gid, int* t4, int* slot) {
+  if (G == 16) {
+    const int row = (tb & 1) ? 8 + (tb >> 1) : (tb >> 1);
+    *slot = (row >> 3) + 2 * (k >> 3) + 4 * (k & 1);
+    *gid = row & 7;
+    *t4 = (k & 7) >> 1;
+  } else {
+    const int mi = tb >> 4, tl = tb & 15;
+    const int row = (tl & 1) ? 8 + (tl >> 1) : (tl >> 1);
+    *slot = (row >> 3) + 2 * mi + 4 * (k & 1);
+    *gid = row & 7;
+    *t4 = k >> 1;
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void v_side_pos(int tb, int k, int* gid, int* t4, int* slot) {
+  if (G == 16) {
+    *slot = (k >> 3) + 2 * (tb >> 3) + 4 * (tb & 1);
+    *gid = k & 7;
+    *t4 = (tb & 7) >> 1;
+  } else {
+    const int mi = tb >> 4, tl = tb & 15;
+    *slot = mi + 2 * (tl >> 3) + 4 * (tl & 1);
+    *gid = k;
+    *t4 = (tl & 7) >> 1;
+  }
+}
+
+// Pending bits of one block word: consecutive entries that land in the same word
+// are merged.  Global words (kShared = false) are written with one atomicAnd /
+// atomicOr pair (other tokens of the block may be written concurrently or may
+// hold stale bits); a zeroed shared-memory copy of the block only needs the OR.
+struct WordBits {
+  int w;
+  uint32_t mask, val;
+};
+
+template <bool kShared>
+__device__ __forceinline__ void flush_word(uint32_t* blk, WordBits& a) {
+  if (a.w >= 0) {
+    if (!kShared) atomicAnd(blk + a.w, ~a.mask);
+    atomicOr(blk + a.w, a.val);
+  }
+  a.w = -1;
+  a.mask = a.val = 0u;
+}
+
+template <bool kShared>
+__device__ __forceinline__ void put_bits(uint32_t* blk, WordBits& a, int w, int shift, uint32_t width_mask,
+                                         uint32_t v) {
+  if (w != a.w) {
+    flush_word<kShared>(blk, a);
+    a.w = w;
+  }
+  a.mask |= width_mask << shift;
+  a.val |= (v & width_mask) << shift;
+}
+
+// Writes one code (width b) of fragment position (gid, t4, slot) into a block:
+//   b = 4: word 4 gid + t4, nibble `slot`;
+//   b = 2: word 2 gid + t4/2, bits 4 slot + 2 (t4 % 2) + {0, 1};
+//   b = 1: word gid, bit 4 slot + t4;
+//   b = 3: bits 0-1 as b = 2, bit 2 as b = 1 in words 16 + gid (second pending word);
+//   b = 8: word 2 (4 gid + t4) + (slot / 2) % 2, byte (slot % 2) + 2 (slot / 4).
+template <bool kShared>
+__device__ __forceinline__ void put_code(uint32_t* blk, WordBits& a, WordBits& a1, int b, int gid, int t4,
+                                         int slot, uint32_t code) {
+  switch (b) {
+    case 4: put_bits<kShared>(blk, a, 4 * gid + t4, 4 * slot, 0xFu, code); break;
+    case 2: put_bits<kShared>(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code); break;
+    case 1: put_bits<kShared>(blk, a, gid, 4 * slot + t4, 0x1u, code); break;
+    case 3:
+      put_bits<kShared>(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code);
+      put_bits<kShared>(blk, a1, 16 + gid, 4 * slot + t4, 0x1u, code >> 2);
+      break;
+    default:
+      put_bits<kShared>(blk, a, 2 * (4 * gid + t4) + ((slot >> 1) & 1), 8 * ((slot & 1) + 2 * (slot >> 2)), 0xFFu,
+                        code);
+      break;
+  }
+}
+
+// Scale/zero of page token tau: record of its pair u = tau/2 at index
+// (u % 8) * (P/16) + u / 8, fp16 {s[2u], s[2u+1], z[2u], z[2u+1]}.
+__device__ __forceinline__ void put_record(uint8_t* recs, int P, int tau, __half s_h, __half z_h) {
+  const int u = tau >> 1;
+  __half* rec = reinterpret_cast<__half*>(recs + 8 * ((u & 7) * (P >> 4) + (u >> 3)));
+  rec[tau & 1] = s_h;
+  rec[2 + (tau & 1)] = z_h;
+}
+
+template <int G, bool kShared>
+__device__ __forceinline__ void put_codes(uint32_t* blk, int side, int tb, int b, const uint32_t (&code)[G]) {
+  WordBits acc{-1, 0u, 0u}, acc1{-1, 0u, 0u};
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    int gid, t4, slot;
+    if (side == 0) k_side_pos<G>(tb, k, &gid, &t4, &slot);
+    else v_side_pos<G>(tb, k, &gid, &t4, &slot);
+    put_code<kShared>(blk, acc, acc1, b, gid, t4, slot, code[k]);
+  }
+  flush_word<kShared>(blk, acc);
+  flush_word<kShared>(blk, acc1);
+}
+
+
+}  // namespace pack
+}  // namespace spectra

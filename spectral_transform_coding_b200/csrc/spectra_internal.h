@@ -58,6 +58,7 @@ struct CodecDev {
   int32_t* err;                      // device error word (first error wins)
   const uint16_t* wt_down;           // bf16 bits, [n_eff_pad][d_model] (W_down transposed)
   const float* w_up;                 // kept rows of V_r^T per (head, side), see SideDev::wup_off
+  const int32_t* col_groups;         // per group of G latent columns: {b, plane_off, sz_off, side}
   HeadDev head[kMaxKV];
 };
 

@@ -5,10 +5,13 @@ shaped layers), through the C ABI.
   d_model slices runs more than once.
 - The tcgen05 projection at K = d_model = 4096 with 1024 and 2048 latent
   columns and a row count that is not a multiple of the 128-row tile.
-- The latent decode at 32,768 + 5 tokens with 8 KV heads (Llama 4x) and at
-  131,072 + 3 tokens with 7 q heads per KV head (Qwen 8x), checked on sampled
-  (sequence, q head) pairs against the oracle's decode over its own copy of
-  the pool, which must equal the library's byte for byte.
+- The latent decode at 32,768 + 5 tokens with 8 KV heads (Llama 4x), at
+  131,072 + 3 tokens with 7 q heads per KV head (Qwen 8x), and over 16
+  sequences of 32,768 + 11 tokens with 8 KV heads at 12x (the heavy-tail stress
+  layer's batch), checked on sampled (sequence, q head) pairs against the
+  oracle's decode over its own copy of the pool, which must equal the library's
+  byte for byte.  The decode's launch plan (split count, stages) depends only
+  on the head shapes, widths and batch, so these runs use the benchmark's.
 
 Bars as in the other parity tests: latents 1e-3 (per token and head-side, L2),
 packed pages bit-exact, attention 2e-3 (max over the sampled pairs of
@@ -26,6 +29,7 @@ pytestmark = pytest.mark.gpu
 LLAMA4X = [4, 2, 2, 2, 2, 2, 1, 1]          # widths of a Llama-shaped head side at 4x
 QWEN8X_K = [4, 2, 1, 1, 0, 0, 0, 0]         # Qwen-shaped head at 8x
 QWEN8X_V = [4, 3, 3, 0, 0, 0, 0, 0]
+STRESS12X = [4, 2, 0, 0, 0, 0, 0, 0]        # 170 bits per side with scale/zero
 
 
 def _codec(d_model, n_q, n_kv, wk, wv, seed, P=64):
@@ -132,4 +136,53 @@ def test_decode_llama_32k_context_8_kv_heads():
 
 def test_decode_qwen_128k_context_gqa7():
     err = _long_decode(28, 4, QWEN8X_K, QWEN8X_V, 131072 + 3, [(0, 0), (0, 20), (0, 27)], seed=31)
+    assert err <= 2e-3, err
+
+
+def test_decode_stress_12x_batch16_32k():
+    """16 sequences at 32k with 8 KV heads and 12x widths.  Sequences 0 and 11
+    (sampled) are filled with seeded latents on both sides; the other 14 with
+    device-drawn latents that only the library sees (their pages are not
+    compared, their outputs not checked)."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    seed, n_q, n_kv, B, length, P = 41, 32, 8, 16, 32768 + 11, 64
+    sampled = [0, 11]
+    codec, widths, _, W_up = _codec(512, n_q, n_kv, STRESS12X, STRESS12X, seed=seed)
+    maxp = (length + P - 1) // P + 1
+    rng = np.random.default_rng(seed + 1)
+    table = rng.permutation(B * maxp).astype(np.int32).reshape(B, maxp)
+    cache = st.LatentCache(codec, batch=B, max_pages_per_seq=maxp, device=dev(), page_table=torch.from_numpy(table))
+    lay = oracle.page_layout(oracle_widths(widths), 16, P)
+    pool = np.zeros(cache.pool.numel(), np.uint8)
+    lengths = np.zeros(B, np.int64)
+    gen = torch.Generator(device=dev())
+    gen.manual_seed(seed + 2)
+    chunk = 8192
+    for b in range(B):
+        for t0 in range(0, length, chunk):
+            n = min(chunk, length - t0)
+            seqs = np.full(n, b, np.int32)
+            if b in sampled:
+                lat = synthetic_latents(n, codec.n_eff, seed=seed + 3 + 100 * b + t0 // chunk, decay=0.5, scale=2.0)
+                lengths = oracle.append_tokens(pool, codec.page_bytes, lay, oracle_widths(widths), 16, P, table,
+                                               lengths, seqs, lat, n_kv)
+                lat_d = torch.from_numpy(lat).to(dev())
+            else:
+                lat_d = torch.randn((n, codec.n_eff), generator=gen, device=dev()) * 2.0
+            codec.quantize_append(cache, lat_d, torch.from_numpy(seqs).to(dev()))
+    codec.device_status()
+    assert cache.lengths.cpu().tolist() == [length] * B
+    got_pool = cache.pool.cpu().numpy()
+    for b in sampled:
+        for pg in table[b, :(length + P - 1) // P]:
+            sl = slice(int(pg) * codec.page_bytes, (int(pg) + 1) * codec.page_bytes)
+            assert np.array_equal(got_pool[sl], pool[sl]), f"page {pg} of sequence {b} differs from the oracle's"
+    q = (rng.standard_normal((B, n_q, 128)) * 0.6).astype(np.float32)
+    out = codec.decode_attend(cache, torch.from_numpy(q).to(dev())).cpu().numpy()
+    codec.device_status()
+    pairs = [(0, 0), (0, 17), (11, 5), (11, 31)]
+    ref = oracle.decode_reference(pool, codec.page_bytes, lay, 16, P, table, lengths, q,
+                                  kept_wup(W_up, widths, 16), n_q, n_kv, pairs=pairs)
+    err = attention_rel_err(np.stack([out[b, h] for b, h in pairs]), np.stack([ref[b, h] for b, h in pairs]))
     assert err <= 2e-3, err
