@@ -1,6 +1,7 @@
 // Internal declarations of libspectra (not part of the C ABI).
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <string>
 #include <vector>
@@ -41,7 +42,8 @@ struct DecodeOrder {
   int32_t cls[2][8];
 };
 
-struct HeadDev {
+// 16-byte aligned: kernels copy the group and class tables with 16-byte loads.
+struct alignas(16) HeadDev {
   SideDev side[2];
   int32_t sec_off;        // byte offset of the head section in a page
   int32_t sec_bytes;      // bytes of the head section (K + V)
@@ -51,7 +53,7 @@ struct HeadDev {
 };
 
 // Device-resident description of a codec; kernels read it from global memory.
-struct CodecDev {
+struct alignas(16) CodecDev {
   int32_t d_model, n_q, n_kv, gq, d_h, group, P, n_eff;
   int32_t n_eff_pad, max_kept_k, max_kept_v, max_sec_bytes;
   int64_t page_bytes;
@@ -61,6 +63,11 @@ struct CodecDev {
   const int32_t* col_groups;         // per group of G latent columns: {b, plane_off, sz_off, side}
   HeadDev head[kMaxKV];
 };
+
+static_assert(sizeof(GroupDev) == 16 && offsetof(SideDev, grp) % 16 == 0 && sizeof(SideDev) % 16 == 0,
+              "group tables are read with 16-byte loads");
+static_assert(offsetof(HeadDev, dec) % 16 == 0 && sizeof(HeadDev) % 16 == 0 && offsetof(CodecDev, head) % 16 == 0,
+              "class tables are read with 16-byte loads");
 
 // ---- host math (host_math.cpp), no CUDA needed ------------------------------
 int allocate_widths(const double* sigma2, int rank, int group, int budget, bool overhead,
