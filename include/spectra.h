@@ -268,7 +268,13 @@ SPECTRA_API spectra_status spectra_quantize_append(const spectra_codec* codec, c
  * in one kernel with one CTA per kept group (latents summed in a different
  * order than spectra_project's, so they may differ from it in the last bits;
  * the codes are those spectra_quantize_append gives for these latents); the
- * CTA that finishes last advances the lengths.  The same checks apply and a
+ * CTA that finishes last advances the lengths.  For T >= 64 with latents_out
+ * NULL (prefill) the positions are planned and checked first, then the
+ * tcgen05 projection GEMM quantises and packs each output tile in its
+ * epilogue, so no fp32 latents are written; its accumulators equal
+ * spectra_project's, so the pages equal those of spectra_project followed by
+ * spectra_quantize_append.  Otherwise (16 < T < 64, or latents_out given) the
+ * latents go through memory.  The same checks apply on every route and a
  * failure writes nothing. */
 SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, const spectra_cache* cache,
                                      const void* H, const int32_t* seq_ids, int64_t T,

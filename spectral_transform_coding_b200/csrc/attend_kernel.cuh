@@ -252,7 +252,10 @@ __device__ __forceinline__ void key_group(uint32_t blk, uint32_t rec, const Lane
 }
 
 // Values of one kept group for the CH tiles of a chunk: va += code^T (p s).
-// recA / recB: this lane's records of token pairs t4 and t4+4.
+// recA / recB: this lane's records of token pairs t4 and t4+4.  The chunk's
+// tiles are summed by the tensor cores from zero and the chunk's sum is added to
+// va in IEEE fp32: accumulating a whole context inside the MMA chain loses
+// accuracy (the positive code term and the z term nearly cancel at the end).
 template <int G, int CH, int B, bool kMask>
 __device__ __forceinline__ void value_group(uint32_t blk, uint32_t recA, uint32_t recB, const LaneAddr& L,
                                             const uint32_t (&pb)[CH][2], const uint32_t (&msk)[CH][2],
@@ -261,6 +264,7 @@ __device__ __forceinline__ void value_group(uint32_t blk, uint32_t recA, uint32_
   const uint32_t p1 = blk + 64 + L.off1;
   const uint32_t sh = lane_sh<B>(L);
   uint32_t s0[CH], s1[CH];
+  float t[4];
   static_for<CH / 2>([&](auto hi) {
     constexpr int h = decltype(hi)::value;
     const uint4 ra = ld_s128<h * 16>(recA);
@@ -279,8 +283,13 @@ __device__ __forceinline__ void value_group(uint32_t blk, uint32_t recA, uint32_
     const uint32_t a0 = kMask ? (s0[tt] & msk[tt][0]) : s0[tt];
     const uint32_t a1 = kMask ? (s1[tt] & msk[tt][1]) : s1[tt];
     const uint32_t bj[2] = {hmul2_bits(pb[tt][0], a0), hmul2_bits(pb[tt][1], a1)};
-    mma_m16n8k16(va, av, bj);
+    if constexpr (tt == 0) mma_m16n8k16_z(t, av, bj);
+    else mma_m16n8k16(t, av, bj);
   });
+  va[0] += t[0];
+  va[1] += t[1];
+  va[2] += t[2];
+  va[3] += t[3];
 }
 
 
@@ -774,12 +783,18 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
           zb[2 * h] = y.y;
           zb[2 * h + 1] = y.w;
         });
+        float tz[4];
 #pragma unroll
         for (int tt = 0; tt < CH; ++tt) {
           const uint32_t az[4] = {partial ? (za[tt] & msk[tt][0]) : za[tt], 0u,
                                   partial ? (zb[tt] & msk[tt][1]) : zb[tt], 0u};
-          mma_m16n8k16(dz, az, pb[tt]);
+          if (tt == 0) mma_m16n8k16_z(tz, az, pb[tt]);
+          else mma_m16n8k16(tz, az, pb[tt]);
         }
+        dz[0] += tz[0];
+        dz[1] += tz[1];
+        dz[2] += tz[2];
+        dz[3] += tz[3];
       }
     }
     // stage s is free: count it, and send the copy of page i + S into it
