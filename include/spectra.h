@@ -261,14 +261,16 @@ SPECTRA_API spectra_status spectra_quantize_append(const spectra_codec* codec, c
  *   H device bf16 [T][d_model]; seq_ids as above; latents_out device fp32
  *   [T][n_eff] or NULL (when given, the latents are kept there);
  *   workspace device, >= spectra_encode_workspace_bytes(T), 256-byte aligned;
- *   its first 256 bytes hold an arrival counter that must be zero when a call
+ *   its first 8448 bytes hold arrival counters that must be zero when a call
  *   starts: zero the workspace once before its first use; every call leaves
- *   the counter at zero.  Calls that share a workspace must not overlap.
+ *   the counters at zero.  Calls that share a workspace must not overlap.
  * For T <= 16 (decode steps) the projection, quantisation and packing run fused
- * in one kernel with one CTA per kept group (latents summed in a different
- * order than spectra_project's, so they may differ from it in the last bits;
- * the codes are those spectra_quantize_append gives for these latents); the
- * CTA that finishes last advances the lengths.  For T >= 64 with latents_out
+ * in one kernel: CTAs per (kept group, d_model chunk) write partial sums, the
+ * last chunk of a group adds them in chunk order and quantises the group
+ * (latents summed in a different order than spectra_project's, so they may
+ * differ from it in the last bits; the codes are those
+ * spectra_quantize_append gives for these latents); the group that finishes
+ * last advances the lengths.  For T >= 64 with latents_out
  * NULL (prefill) the positions are planned and checked first, then the
  * tcgen05 projection GEMM quantises and packs each output tile in its
  * epilogue, so no fp32 latents are written; its accumulators equal

@@ -175,13 +175,16 @@ spectra_status build_codec(const spectra_config& cfg, const int32_t* widths, con
   return SPECTRA_OK;
 }
 
-// Encode workspace: [arrival counter of the fused path, 256 B][positions][flag][latents].
-constexpr size_t kEncCounterBytes = 256;
+// Encode workspace: [counters of the fused decode-step path][positions][flag]
+// [latents, or the fused path's partial sums].
+constexpr size_t kEncCounterBytes = ((1 + kMaxFusedGroups) * 4 + 255) / 256 * 256;
 constexpr int64_t kGemmMinT = 64;  // rows from which the projection runs on the tcgen05 GEMM
 size_t encode_ws_bytes(const spectra_codec* c, int64_t T) {
   const size_t pos = ((size_t)std::max<int64_t>(T, 1) * 4 + 255) / 256 * 256;
   const size_t flag = 256;
-  const size_t lat = ((size_t)std::max<int64_t>(T, 1) * c->h.n_eff * 4 + 255) / 256 * 256;
+  size_t lat = (size_t)std::max<int64_t>(T, 1) * c->h.n_eff * 4;
+  lat = std::max(lat, encode_fused_partial_bytes(c->h, (int)std::min<int64_t>(std::max<int64_t>(T, 1), kFusedMaxT)));
+  lat = (lat + 255) / 256 * 256;
   return kEncCounterBytes + pos + flag + lat;
 }
 
@@ -657,8 +660,10 @@ spectra_status spectra_encode_append(const spectra_codec* c, const spectra_cache
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (T <= kFusedMaxT) {
     // decode steps: projection, quantisation and packing fused per kept group
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    float* part = reinterpret_cast<float*>(w + kEncCounterBytes + ((size_t)T * 4 + 255) / 256 * 256 + 256);
     CUDA_TRY(launch_encode_fused(c->h, c->d, static_cast<const uint16_t*>(H), seq_ids, (int)T, *cache,
-                                 latents_out, static_cast<int32_t*>(workspace), st));
+                                 latents_out, reinterpret_cast<int32_t*>(w), part, st));
     return SPECTRA_OK;
   }
   if (!latents_out && T >= kGemmMinT) {

@@ -256,10 +256,9 @@ __device__ __forceinline__ void key_group(uint32_t blk, uint32_t rec, const Lane
 // tiles are summed by the tensor cores from zero and the chunk's sum is added to
 // va in IEEE fp32: accumulating a whole context inside the MMA chain loses
 // accuracy (the positive code term and the z term nearly cancel at the end).
-template <int G, int CH, int B, bool kMask>
+template <int G, int CH, int B>
 __device__ __forceinline__ void value_group(uint32_t blk, uint32_t recA, uint32_t recB, const LaneAddr& L,
-                                            const uint32_t (&pb)[CH][2], const uint32_t (&msk)[CH][2],
-                                            float (&va)[4]) {
+                                            const uint32_t (&pb)[CH][2], float (&va)[4]) {
   const uint32_t p = blk + lane_off<B>(L);
   const uint32_t p1 = blk + 64 + L.off1;
   const uint32_t sh = lane_sh<B>(L);
@@ -280,9 +279,7 @@ __device__ __forceinline__ void value_group(uint32_t blk, uint32_t recA, uint32_
     constexpr int OFF = (tt / kBlockTiles) * B * 32;
     uint32_t av[4];
     frag_v<G, B, OFF, tt & 1>(p, p1, sh, L.rot1, av);
-    const uint32_t a0 = kMask ? (s0[tt] & msk[tt][0]) : s0[tt];
-    const uint32_t a1 = kMask ? (s1[tt] & msk[tt][1]) : s1[tt];
-    const uint32_t bj[2] = {hmul2_bits(pb[tt][0], a0), hmul2_bits(pb[tt][1], a1)};
+    const uint32_t bj[2] = {hmul2_bits(pb[tt][0], s0[tt]), hmul2_bits(pb[tt][1], s1[tt])};
     if constexpr (tt == 0) mma_m16n8k16_z(t, av, bj);
     else mma_m16n8k16(t, av, bj);
   });
@@ -608,6 +605,24 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     const uint32_t sec = stages_u32 + (uint32_t)(s * A.stage_bytes);
     const int pg = page_of(i);
     const int n_valid = min(P, len - pg * P);
+    if (n_valid < P) {
+      // tokens past the end (last page): their records may hold anything (NaN
+      // included); zero their scales and zeros so that they add nothing to the
+      // value sums (their scores are set to -inf below)
+      const int u0 = n_valid >> 1, nz = (P >> 1) - u0;
+      for (int e = lane; e < (nK + nV) * nz; e += 32) {
+        const int gs = e / nz, u = u0 + (e - gs * nz);
+        const int4 o = gs < nK ? ord[gs] : ord[kMaxG + gs - nK];
+        const uint32_t ra = sec + (uint32_t)o.y + 8u * (uint32_t)((u & 7) * tpp + (u >> 3));
+        if (u == u0 && (n_valid & 1)) {
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(ra + 2), "h"((unsigned short)0) : "memory");
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(ra + 6), "h"((unsigned short)0) : "memory");
+        } else {
+          asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(ra), "r"(0u) : "memory");
+        }
+      }
+      __syncwarp();
+    }
 #pragma unroll 1
     for (int c0 = 0; c0 < tpp; c0 += CH) {
       const int tok0 = c0 * 16;
@@ -708,7 +723,6 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
       // p as the B operand (tokens x heads): lane (gid, t4) needs head gid,
       // tokens (2t4, 2t4+1) and (2t4+8, 2t4+9)
       uint32_t pb[CH][2];
-      uint32_t msk[CH][2];
       float off[NT];  // p = 2^(s - m + 8)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) off[nt] = kPScaleLog2 - m_run[nt];
@@ -735,12 +749,6 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
         }
         // (columns of heads >= gq hold copies of real heads' weights; their
         // accumulator columns are never read)
-        if (partial) {
-          // tokens past the end: their records may hold anything; zero their s and z
-          const int nv = n_valid - tok0 - tt * 16;
-          msk[tt][0] = ((2 * t4 < nv) ? 0x0000ffffu : 0u) | ((2 * t4 + 1 < nv) ? 0xffff0000u : 0u);
-          msk[tt][1] = ((2 * t4 + 8 < nv) ? 0x0000ffffu : 0u) | ((2 * t4 + 9 < nv) ? 0xffff0000u : 0u);
-        }
       }
       // values: per group, sum_t (p_t s_t,j) code_t,j ...
       const uint32_t ra = sec + (uint32_t)(recVa + c0 * 8), rb = sec + (uint32_t)(recVb + c0 * 8);
@@ -751,22 +759,12 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
           constexpr int kBT = G == 16 ? 1 : 2;
           const uint32_t gb = sec + (uint32_t)g.x + (uint32_t)(c0 / kBT) * 32u * (uint32_t)g.w;
           const uint32_t ga = ra + (uint32_t)g.y, gbr = rb + (uint32_t)g.y;
-          if (!partial) {
-            switch (g.w) {
-              case 4: value_group<G, CH, 4, false>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              case 2: value_group<G, CH, 2, false>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              case 1: value_group<G, CH, 1, false>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              case 3: value_group<G, CH, 3, false>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              default: value_group<G, CH, 8, false>(gb, ga, gbr, L, pb, msk, va[c]); break;
-            }
-          } else {
-            switch (g.w) {
-              case 4: value_group<G, CH, 4, true>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              case 2: value_group<G, CH, 2, true>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              case 1: value_group<G, CH, 1, true>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              case 3: value_group<G, CH, 3, true>(gb, ga, gbr, L, pb, msk, va[c]); break;
-              default: value_group<G, CH, 8, true>(gb, ga, gbr, L, pb, msk, va[c]); break;
-            }
+          switch (g.w) {
+            case 4: value_group<G, CH, 4>(gb, ga, gbr, L, pb, va[c]); break;
+            case 2: value_group<G, CH, 2>(gb, ga, gbr, L, pb, va[c]); break;
+            case 1: value_group<G, CH, 1>(gb, ga, gbr, L, pb, va[c]); break;
+            case 3: value_group<G, CH, 3>(gb, ga, gbr, L, pb, va[c]); break;
+            default: value_group<G, CH, 8>(gb, ga, gbr, L, pb, va[c]); break;
           }
         }
       });
@@ -786,8 +784,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
         float tz[4];
 #pragma unroll
         for (int tt = 0; tt < CH; ++tt) {
-          const uint32_t az[4] = {partial ? (za[tt] & msk[tt][0]) : za[tt], 0u,
-                                  partial ? (zb[tt] & msk[tt][1]) : zb[tt], 0u};
+          const uint32_t az[4] = {za[tt], 0u, zb[tt], 0u};
           if (tt == 0) mma_m16n8k16_z(tz, az, pb[tt]);
           else mma_m16n8k16(tz, az, pb[tt]);
         }

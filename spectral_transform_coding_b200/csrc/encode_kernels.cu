@@ -3,6 +3,7 @@
 // stage 3), with groups of adjacent latent coordinates sharing one width (stage 2,
 // "grouping").
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <cuda_fp16.h>
 
 #include "device_common.cuh"
@@ -243,12 +244,17 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Fused small-batch encode (decode steps, T <= kFusedMaxT tokens): one CTA per
-// kept group projects the step's tokens onto the group's G columns (W_down rows
-// streamed once, H slices staged in shared memory), quantises and packs them,
-// all in one kernel; the positions are computed and validated by every CTA the
-// same way from the current lengths, so a failed check writes nothing anywhere.
-// A one-block commit kernel then advances the lengths.
+// Fused small-batch encode (decode steps, T <= kFusedMaxT tokens).  The
+// projection of the step's tokens is split over CTAs (kept group, d_model chunk
+// of KCH columns of H): each CTA streams its group's G rows of W_down over its
+// chunk (all of its loads in flight before the dependency wait), multiplies
+// them with the tokens' H (read after the wait), reduces across the warp and
+// writes a partial sum per (token, column) to the workspace.  The last CTA of a
+// group to arrive (a counter per group) adds the chunks' partials in chunk
+// order, quantises and packs the group for the step's tokens.  The positions
+// are computed and validated by every such CTA the same way from the current
+// lengths, so a failed check writes nothing anywhere; the last group to finish
+// (a second counter) advances the lengths.  All counters are left at zero.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -269,23 +275,62 @@ __device__ __forceinline__ int append_position(const int32_t* __restrict__ seq_i
 
 }  // namespace
 
-template <int G, int ROWS, int KC>
+namespace {
+
+// Sum of vals[v] over the 32 lanes of a warp for V values per lane (V a power
+// of two <= 32), by recursive halving: lane l ends with the total of value
+// l >> (5 - log2 V).
+template <int V>
+__device__ __forceinline__ float warp_transpose_sum(float (&vals)[V], int lane) {
+  int len = V;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (len > 1) {
+      const int half = len / 2;
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < V / 2; ++i) {
+        if (i < half) {
+          const float send = upper ? vals[i] : vals[i + half];
+          const float keep = upper ? vals[i + half] : vals[i];
+          vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      len = half;
+    } else {
+      vals[0] += __shfl_xor_sync(0xffffffffu, vals[0], o);
+    }
+  }
+  return vals[0];
+}
+
+__host__ __device__ constexpr int log2_int(int v) { return v <= 1 ? 0 : 1 + log2_int(v / 2); }
+
+constexpr int kMaxChunks = 16;  // d_model chunks per group (the plan keeps to it)
+
+}  // namespace
+
+template <int G, int TP, int BATCH>
 __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __restrict__ cd,
                                                            const uint16_t* __restrict__ H, int T,
                                                            const int32_t* __restrict__ seq_ids,
                                                            const spectra_cache cache,
                                                            float* __restrict__ latents_out,
-                                                           int32_t* __restrict__ arrivals) {
-  constexpr int CPW = G / 8;       // columns per warp (8 warps cover the group)
-  constexpr int BATCH = KC / 256;  // 16-byte chunks per column and lane per slice
-  __shared__ __align__(16) uint16_t h_s[ROWS * KC];
-  __shared__ float x_s[ROWS][G];
+                                                           int32_t* __restrict__ counters,
+                                                           float* __restrict__ part, int n_chunks, int cpc) {
+  constexpr int CPW = G / 8;        // columns per warp (8 warps cover the group)
+  constexpr int KCH = 256 * BATCH;  // d_model columns of H per chunk
+  constexpr int V = CPW * TP;       // partial sums per lane
+  __shared__ float x_s[TP][G];
   __shared__ int worst;
-  __shared__ int is_last;
+  __shared__ int flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
-  // this CTA's group: kept groups numbered head-major, K side then V side
-  int a = 0, sd_i = 0, g = blockIdx.x;
+  // this CTA's group (kept groups numbered head-major, K side then V side) and
+  // its chunks [ch0, ch1) of d_model
+  const int gi = blockIdx.x, n_part = gridDim.y;
+  const int ch0 = blockIdx.y * cpc, ch1 = min(n_chunks, ch0 + cpc);
+  int a = 0, sd_i = 0, g = gi;
   for (; a < cd->n_kv; ++a) {
     int side = 0;
     for (; side < 2; ++side) {
@@ -302,70 +347,89 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
   const GroupDev gd = sd.grp[g];
   const int d_model = cd->d_model;
   const int n0 = sd.c_col0 + gd.col + warp * CPW;  // latent columns of this warp
-  const uint16_t* wt = cd->wt_down;
-  float acc[CPW][ROWS];
-#pragma unroll
-  for (int c = 0; c < CPW; ++c)
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) acc[c][r] = 0.f;
-  const int nr = min(ROWS, T);
-  for (int kc0 = 0; kc0 < d_model; kc0 += KC) {
-    uint4 wv[CPW][BATCH];
+  // W_down rows of this warp's columns over the first chunk: read-only codec
+  // data, loaded before the wait; later chunks are loaded after it
+  uint4 wv[CPW][BATCH];
+  auto load_w = [&](int ch) {
 #pragma unroll
     for (int i = 0; i < BATCH; ++i)
 #pragma unroll
       for (int c = 0; c < CPW; ++c) {
-        const int k = kc0 + lane * 8 + 256 * i;
-        wv[c][i] = k < d_model ? __ldg(reinterpret_cast<const uint4*>(wt + (size_t)(n0 + c) * d_model + k))
-                               : make_uint4(0u, 0u, 0u, 0u);
+        const int k = ch * KCH + lane * 8 + 256 * i;
+        wv[c][i] = k < d_model
+                       ? __ldg(reinterpret_cast<const uint4*>(cd->wt_down + (size_t)(n0 + c) * d_model + k))
+                       : make_uint4(0u, 0u, 0u, 0u);
       }
-    pdl_wait();       // H, lengths and the page table may come from earlier kernels
-    __syncthreads();  // the previous slice's readers are done
-    for (int e = tid; e < ROWS * KC / 8; e += blockDim.x) {
-      const int r = e / (KC / 8), col = (e % (KC / 8)) * 8;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < nr && kc0 + col < d_model)
-        v = __ldg(reinterpret_cast<const uint4*>(H + (size_t)r * d_model + kc0 + col));
-      *reinterpret_cast<uint4*>(h_s + r * KC + col) = v;
-    }
-    __syncthreads();
+  };
+  load_w(ch0);
+  pdl_wait();  // H, lengths and the page table may come from earlier kernels
+  float acc[V];
 #pragma unroll
-    for (int i = 0; i < BATCH; ++i) {
-      const int kl = lane * 8 + 256 * i;
-      float w[CPW][8];
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  for (int ch = ch0; ch < ch1; ++ch) {
+    if (ch > ch0) load_w(ch);
 #pragma unroll
-      for (int c = 0; c < CPW; ++c) bf16x8_to_f32(wv[c][i], w[c]);
+    for (int r = 0; r < TP; ++r) {
+      if (r < T) {
 #pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        if (r < nr) {
+        for (int i = 0; i < BATCH; ++i) {
+          const int k = ch * KCH + lane * 8 + 256 * i;
           float h[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(h_s + r * KC + kl), h);
+          bf16x8_to_f32(k < d_model ? __ldg(reinterpret_cast<const uint4*>(H + (size_t)r * d_model + k))
+                                    : make_uint4(0u, 0u, 0u, 0u), h);
 #pragma unroll
-          for (int c = 0; c < CPW; ++c)
+          for (int c = 0; c < CPW; ++c) {
+            float w[8];
+            bf16x8_to_f32(wv[c][i], w);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[c][r] = fmaf(w[c][e], h[e], acc[c][r]);
+            for (int e = 0; e < 8; ++e) acc[c * TP + r] = fmaf(w[e], h[e], acc[c * TP + r]);
+          }
         }
       }
     }
   }
-  if (tid == 0) worst = 0;
-#pragma unroll
-  for (int c = 0; c < CPW; ++c)
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-      float v = acc[c][r];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && r < nr) x_s[r][warp * CPW + c] = v;
+  {
+    const float tot = warp_transpose_sum<V>(acc, lane);
+    constexpr int SH = 5 - log2_int(V);
+    const int v = lane >> SH, c = v / TP, r = v % TP;
+    if ((lane & ((1 << SH) - 1)) == 0 && r < T) {
+      if (n_part == 1) x_s[r][warp * CPW + c] = tot;
+      else part[((size_t)(gi * n_part + blockIdx.y) * TP + r) * G + warp * CPW + c] = tot;
     }
-  // positions of the step's tokens; every CTA reaches the same verdict
+  }
+  if (n_part > 1) {
+    // the last CTA of this group to arrive adds the CTAs' partial sums in order
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int t = atomicAdd(counters + 1 + gi, 1);
+      flag = t == n_part - 1;
+      if (flag) atomicExch(counters + 1 + gi, 0);
+    }
+    __syncthreads();
+    if (!flag) return;
+    __threadfence();
+    if (tid < T * G) {
+      const int r = tid / G, c = tid % G;
+      const float* pp = part + ((size_t)gi * n_part * TP + r) * G + c;
+      float v[kMaxChunks];
+#pragma unroll
+      for (int k = 0; k < kMaxChunks; ++k) v[k] = k < n_part ? __ldcg(pp + (size_t)k * TP * G) : 0.f;
+      float x = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxChunks; ++k) x += v[k];  // CTA order; absent ones add zero
+      x_s[r][c] = x;
+    }
+  }
+  if (tid == 0) worst = 0;
+  // positions of the step's tokens; every finishing CTA reaches the same verdict
   int64_t pos = 0;
   int code_err = 0;
   if (tid < T) code_err = append_position(seq_ids, tid, cache, cd->P, &pos);
   __syncthreads();
   if (code_err) atomicMax(&worst, code_err);
   __syncthreads();
-  if (worst && blockIdx.x == 0 && tid == 0) device_error(cd->err, worst);
+  if (worst && gi == 0 && tid == 0) device_error(cd->err, worst);
   if (!worst && tid < T) {
     float x[G];
 #pragma unroll
@@ -388,18 +452,18 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
     put_codes<G, false>(blkw, sd_i, tau % TB, b, code);
     put_record(page + gd.sz_off, P, tau, s_h, z_h);
   }
-  // The CTA that arrives last advances the lengths: every CTA read them (to
-  // place its tokens) before it arrived, and every page write precedes the
-  // arrival of its CTA.  The counter is left at zero for the next call.
+  // The group that finishes last advances the lengths: every finishing CTA read
+  // them (to place its tokens) before it arrived, and every page write precedes
+  // the arrival of its CTA.  The counter is left at zero for the next call.
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const int t = atomicAdd(arrivals, 1);
-    is_last = t == (int)gridDim.x - 1;
-    if (is_last) atomicExch(arrivals, 0);
+    const int t = atomicAdd(counters, 1);
+    flag = t == (int)gridDim.x - 1;
+    if (flag) atomicExch(counters, 0);
   }
   __syncthreads();
-  if (is_last && !worst && tid < T && (tid == T - 1 || seq_ids[tid + 1] != seq_ids[tid]))
+  if (flag && !worst && tid < T && (tid == T - 1 || seq_ids[tid + 1] != seq_ids[tid]))
     cache.lengths[seq_ids[tid]] = (int32_t)(pos + 1);
 }
 
@@ -467,22 +531,92 @@ cudaError_t launch_length_advance(const int32_t* seq_ids, int T, const spectra_c
   return launch_dependent(length_advance_kernel, dim3(1), dim3(32), 0, st, seq_ids, T, cache, P, err);
 }
 
+EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T) {
+  EncodeFusedPlan p{};
+  for (int a = 0; a < h.n_kv; ++a) p.n_groups += h.head[a].side[0].n_groups + h.head[a].side[1].n_groups;
+  p.tp = 1;
+  while (p.tp < T) p.tp *= 2;
+  static int sm_of_dev[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (sm_of_dev[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    sm_of_dev[dev] = n;
+  }
+  const int sms = sm_of_dev[dev];
+  // CTAs to aim for.  A step of a few sequences leaves one decode CTA per SM
+  // running beside this kernel, so one wave of CTAs that fits next to it starts
+  // early and streams W_down before its dependency wait; with more sequences the
+  // decode fills the SMs and this kernel runs after it, as wide as possible.
+  const long target = T >= 4 ? 2L * sms : (long)sms;
+  // chunks: the widest (fewest partial sums, at most 8 loads of 16 bytes per
+  // column and lane) that gives the target, at most kMaxChunks
+  p.batch = 8;
+  for (int bt = 8; bt >= 1; bt /= 2) {
+    const int nch = (h.d_model + 256 * bt - 1) / (256 * bt);
+    if (nch > kMaxChunks) break;
+    p.batch = bt;
+    if ((long)p.n_groups * nch >= target) break;
+  }
+  p.n_chunks = (h.d_model + 256 * p.batch - 1) / (256 * p.batch);
+  // consecutive chunks per CTA: one when the kernel runs after the decode (every
+  // CTA's loads then start at once), else as many as keep to the target
+  const long per_group = p.n_groups > 0 ? std::max(1L, target / p.n_groups) : 1L;
+  p.cpc = T >= 4 ? 1 : (int)((p.n_chunks + per_group - 1) / per_group);
+  p.n_part = (p.n_chunks + p.cpc - 1) / p.cpc;
+  return p;
+}
+
+size_t encode_fused_partial_bytes(const CodecDev& h, int T) {
+  const EncodeFusedPlan p = encode_fused_plan(h, T);
+  return (size_t)p.n_groups * p.n_part * p.tp * h.group * 4;
+}
+
+namespace {
+template <int G, int TP>
+cudaError_t launch_fused_tp(const EncodeFusedPlan& p, const CodecDev* d, const uint16_t* H, int T,
+                            const int32_t* seq_ids, const spectra_cache& cache, float* latents_out,
+                            int32_t* counters, float* part, cudaStream_t st) {
+  const dim3 grid(p.n_groups, p.n_part), block(256);
+  switch (p.batch) {
+    case 8:
+      return launch_dependent(encode_fused_kernel<G, TP, 8>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                              latents_out, counters, part, p.n_chunks, p.cpc);
+    case 4:
+      return launch_dependent(encode_fused_kernel<G, TP, 4>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                              latents_out, counters, part, p.n_chunks, p.cpc);
+    case 2:
+      return launch_dependent(encode_fused_kernel<G, TP, 2>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                              latents_out, counters, part, p.n_chunks, p.cpc);
+    default:
+      return launch_dependent(encode_fused_kernel<G, TP, 1>, grid, block, 0, st, d, H, T, seq_ids, cache,
+                              latents_out, counters, part, p.n_chunks, p.cpc);
+  }
+}
+
+template <int G>
+cudaError_t launch_fused_g(const EncodeFusedPlan& p, const CodecDev* d, const uint16_t* H, int T,
+                           const int32_t* seq_ids, const spectra_cache& cache, float* latents_out,
+                           int32_t* counters, float* part, cudaStream_t st) {
+  switch (p.tp) {
+    case 1: return launch_fused_tp<G, 1>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+    case 2: return launch_fused_tp<G, 2>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+    case 4: return launch_fused_tp<G, 4>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+    case 8: return launch_fused_tp<G, 8>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+    default: return launch_fused_tp<G, 16>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+  }
+}
+}  // namespace
+
 cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
-                                int T, const spectra_cache& cache, float* latents_out, int32_t* arrivals,
-                                cudaStream_t st) {
-  int n_groups = 0;
-  for (int a = 0; a < h.n_kv; ++a) n_groups += h.head[a].side[0].n_groups + h.head[a].side[1].n_groups;
-  if (n_groups == 0) return launch_length_advance(seq_ids, T, cache, h.P, st, h.err);
-  const dim3 grid(n_groups), block(256);
-  if (h.group == 16)
-    return T <= 1 ? launch_dependent(encode_fused_kernel<16, 1, 2048>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                                     latents_out, arrivals)
-                  : launch_dependent(encode_fused_kernel<16, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T, seq_ids,
-                                     cache, latents_out, arrivals);
-  return T <= 1 ? launch_dependent(encode_fused_kernel<8, 1, 4096>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                                   latents_out, arrivals)
-                : launch_dependent(encode_fused_kernel<8, kFusedMaxT, 1024>, grid, block, 0, st, d, H, T, seq_ids,
-                                   cache, latents_out, arrivals);
+                                int T, const spectra_cache& cache, float* latents_out, int32_t* counters,
+                                float* part, cudaStream_t st) {
+  const EncodeFusedPlan p = encode_fused_plan(h, T);
+  if (p.n_groups == 0) return launch_length_advance(seq_ids, T, cache, h.P, st, h.err);
+  if (T > kFusedMaxT || p.n_groups > kMaxFusedGroups || p.n_part > kMaxChunks) return cudaErrorNotSupported;
+  if (h.group == 16) return launch_fused_g<16>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+  return launch_fused_g<8>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
 }
 
 }  // namespace spectra

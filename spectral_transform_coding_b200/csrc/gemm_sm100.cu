@@ -211,9 +211,11 @@ __global__ void __launch_bounds__(128, 1) gemm_tcgen05_kernel(const __grid_const
 //     token rows) and column half (w - 4) / 4, one group of G columns at a time
 //     (tcgen05.ld 32x32b: each thread holds one token's group), quantises it in
 //     registers and writes codes and scale/zero record into the token's page.
-//     A block of 256/G tokens that the lane set covers whole is assembled in
-//     shared memory and stored with 16-byte stores; partial blocks merge their
-//     bits into the page with atomics (other tiles or calls may share them).
+//     A block of 256/G tokens that the lane set covers whole goes through a
+//     256-byte shared buffer in fragment order, from which lanes assemble the
+//     block's words and store them with 16-byte stores; partial blocks merge
+//     their bits into the page with atomics (other tiles or calls may share
+//     them).
 // Groups never straddle a column tile: every head side's columns start at a
 // multiple of G and BN is a multiple of G.  The accumulators are produced by
 // the same MMA sequence as gemm_tcgen05_kernel's (same tile shape and k order),
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tcgen05_kernel(const __grid_const
 constexpr int kEpiWarps = 8;
 constexpr int kEncThreads = 32 * (4 + kEpiWarps);
 constexpr uint32_t kEncTmemCols = 2 * BN;
-constexpr int kWbufWords = kEpiWarps * 2 * 64;  // one block (<= 64 words) per half-warp
+constexpr int kWbufWords = kEpiWarps * 2 * 64;  // one 256-byte buffer per lane set (half-warp)
 constexpr int ENC_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + kWbufWords * 4;
 
 __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
@@ -427,12 +429,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_gemm_kernel(
         pack::quantize_group<G>(x, b, s_h, z_h, code);
         uint32_t* blkw = reinterpret_cast<uint32_t*>(page + gi.y + blk * (32 * b));
         if (whole) {
-          for (int w = sub; w < 8 * b; w += TB) wb[w] = 0u;
+          uint8_t* fb = reinterpret_cast<uint8_t*>(wb);
+          pack::frag_bytes<G>(fb, gi.w, tb, code);
           __syncwarp(hm);
-          pack::put_codes<G, true>(wb, gi.w, tb, b, code);
-          __syncwarp(hm);
-          for (int w4 = sub; w4 < 2 * b; w4 += TB)
-            reinterpret_cast<uint4*>(blkw)[w4] = reinterpret_cast<const uint4*>(wb)[w4];
+          if (sub < 2 * b) reinterpret_cast<uint4*>(blkw)[sub] = pack::block_words(fb, b, sub);
           __syncwarp(hm);  // before the next group reuses the buffer
         } else if (valid) {
           pack::put_codes<G, false>(blkw, gi.w, tb, b, code);

@@ -41,13 +41,24 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
                                    const int32_t* seq_ids, const int32_t* pos, const int32_t* ok_flag,
                                    int T, const spectra_cache& cache, cudaStream_t st);
 
-// Fused encode for decode steps: projection, quantisation and packing in one
-// kernel per kept group; the CTA that arrives last (counter `arrivals`, zero
-// between calls) advances the lengths.
+// Fused encode for decode steps: projection (split over d_model chunks),
+// quantisation and packing in one kernel; the last chunk of a group to arrive
+// finishes the group and the last group advances the lengths.
 constexpr int kFusedMaxT = 16;
+// Decode-step encode plan: kept groups; d_model chunks of 256 * batch columns,
+// cpc consecutive chunks per CTA, n_part CTAs per group; token count rounded up
+// to a power of two.
+struct EncodeFusedPlan {
+  int n_groups, n_chunks, batch, cpc, n_part, tp;
+};
+constexpr int kMaxFusedGroups = kMaxKV * 2 * kMaxGroups;
+EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T);
+// Workspace bytes of the fused encode's partial sums for T tokens.
+size_t encode_fused_partial_bytes(const CodecDev& h, int T);
+// counters: int32 [1 + kMaxFusedGroups], zero between calls; part: partial sums.
 cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
-                                int T, const spectra_cache& cache, float* latents_out, int32_t* arrivals,
-                                cudaStream_t st);
+                                int T, const spectra_cache& cache, float* latents_out, int32_t* counters,
+                                float* part, cudaStream_t st);
 
 // reconstruct_kernels.cu: k^ = (code s + z) W_up^K, v^ likewise, for tokens
 // [t0, t0 + n) of sequence b; out of range or bad page ids -> device error INVALID

@@ -160,3 +160,95 @@ __device__ __forceinline__ void put_codes(uint32_t* blk, int side, int tb, int b
 
 }  // namespace pack
 }  // namespace spectra
+
+namespace spectra {
+namespace pack {
+
+// ---------------------------------------------------------------------------
+// Whole-block writer.  The TB = 256/G lanes of a lane set hold the TB tokens of
+// one code block (token tb of the block per lane).  Each lane scatters its G
+// codes into a 256-byte shared buffer in fragment order, byte 32 gid + 8 t4 +
+// slot; then the block's 8b words are assembled from consecutive bytes of
+// that buffer, four words per lane (lanes sub < 2b), and stored with one 16-byte
+// store each.  Word and bit of each entry as in the page layout's width rule.
+// ---------------------------------------------------------------------------
+template <int G>
+__device__ __forceinline__ void frag_bytes(uint8_t* fb, int side, int tb, const uint32_t (&code)[G]) {
+  if constexpr (G == 16) {
+    if (side == 0) {  // K: row = tb/2 (tb even) or 8 + tb/2, col = k
+      const int row = (tb & 1) ? 8 + (tb >> 1) : (tb >> 1);
+      uint8_t* p = fb + (row & 7) * 32 + (row >> 3);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) p[((k & 7) >> 1) * 8 + 2 * (k >> 3) + 4 * (k & 1)] = (uint8_t)code[k];
+    } else {  // V: row = k, col = tb
+      uint8_t* p = fb + ((tb & 7) >> 1) * 8 + 2 * (tb >> 3) + 4 * (tb & 1);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) p[(k & 7) * 32 + (k >> 3)] = (uint8_t)code[k];
+    }
+  } else {
+    const int mi = tb >> 4, tl = tb & 15;
+    if (side == 0) {
+      const int row = (tl & 1) ? 8 + (tl >> 1) : (tl >> 1);
+      uint8_t* p = fb + (row & 7) * 32 + (row >> 3) + 2 * mi;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) p[(k >> 1) * 8 + 4 * (k & 1)] = (uint8_t)code[k];
+    } else {
+      uint8_t* p = fb + ((tl & 7) >> 1) * 8 + mi + 2 * (tl >> 3) + 4 * (tl & 1);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) p[k * 32] = (uint8_t)code[k];
+    }
+  }
+}
+
+// four bytes (each < 16) -> their nibbles in bits 0-15
+__device__ __forceinline__ uint32_t nib4(uint32_t x) {
+  x = (x | (x >> 4)) & 0x00FF00FFu;
+  return (x | (x >> 8)) & 0x0000FFFFu;
+}
+
+// Words [4i, 4i + 4) of a block of width b from the fragment-ordered bytes
+// (f[2e], f[2e + 1]: slots 0-3 and 4-7 of entry e = 4 gid + t4).
+__device__ __forceinline__ uint4 block_words(const uint8_t* fb, int b, int i) {
+  const uint32_t* f = reinterpret_cast<const uint32_t*>(fb);
+  uint32_t w[4];
+  if (b == 4) {  // word e: nibble slot = code(e, slot)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 4 * i + j;
+      w[j] = nib4(f[2 * e]) | (nib4(f[2 * e + 1]) << 16);
+    }
+  } else if (b == 8) {  // word 2e + h: bytes of slots {0,1,4,5} (h = 0) or {2,3,6,7}
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int e = 2 * i + j;
+      w[2 * j] = __byte_perm(f[2 * e], f[2 * e + 1], 0x5410);
+      w[2 * j + 1] = __byte_perm(f[2 * e], f[2 * e + 1], 0x7632);
+    }
+  } else if (b == 2 || (b == 3 && i < 4)) {  // word d: entries 2d, 2d + 1 in bits 0-1, 2-3 of a nibble
+    const uint32_t m = b == 3 ? 0x03030303u : 0xFFFFFFFFu;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 2 * (4 * i + j);
+      w[j] = nib4((f[2 * e] & m) | ((f[2 * e + 2] & m) << 2)) |
+             (nib4((f[2 * e + 1] & m) | ((f[2 * e + 3] & m) << 2)) << 16);
+    }
+  } else {  // b = 1 (word gid), or bit 2 of b = 3 (word 16 + gid): bit 4 slot + t4
+    const int g0 = b == 3 ? 4 * (i - 4) : 4 * i;
+    const int sh = b == 3 ? 2 : 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 4 * (g0 + j);
+      uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+      for (int t4 = 0; t4 < 4; ++t4) {
+        lo |= ((f[2 * (e + t4)] >> sh) & 0x01010101u) << t4;
+        hi |= ((f[2 * (e + t4) + 1] >> sh) & 0x01010101u) << t4;
+      }
+      w[j] = nib4(lo) | (nib4(hi) << 16);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+}  // namespace pack
+}  // namespace spectra
