@@ -20,6 +20,9 @@ AttendKernel attend_kernel_ptr_g16(int NT, int CH, int MV) {
     case 242: return attend_kernel<16, 2, 4, 2>;
     case 244: return attend_kernel<16, 2, 4, 4>;
     case 248: return attend_kernel<16, 2, 4, 8>;
+    case 182: return attend_kernel<16, 1, 8, 2>;
+    case 184: return attend_kernel<16, 1, 8, 4>;
+    case 188: return attend_kernel<16, 1, 8, 8>;
     default: return nullptr;
   }
 }

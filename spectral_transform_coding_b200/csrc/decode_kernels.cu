@@ -68,7 +68,13 @@ int sm_count() {
 
 // Tiles (16 tokens) per softmax chunk: 4 when a page holds a multiple of 64
 // tokens, else 2 (pages hold a multiple of 32).
-int chunk_tiles(int P) { return (P / 16) % 4 == 0 ? 4 : 2; }
+// 16-token tiles per softmax chunk: 8 (pages of 128 tokens or more, one n-tile
+// of q heads), else 4 or 2 as the page allows.  Longer chunks amortise the
+// per-chunk work (softmax, z terms, group set-up) over more tokens.
+int chunk_tiles(int P, int NT) {
+  if (NT == 1 && (P / 16) % 8 == 0) return 8;
+  return (P / 16) % 4 == 0 ? 4 : 2;
+}
 
 
 }  // namespace
@@ -103,7 +109,8 @@ int value_group_bound(const CodecDev& h) {
 }
 
 AttendKernel attend_kernel_for(const CodecDev& h) {
-  return attend::attend_kernel_ptr(h.group, h.gq > 4 ? 2 : 1, chunk_tiles(h.P), value_group_bound(h));
+  const int NT = h.gq > 4 ? 2 : 1;
+  return attend::attend_kernel_ptr(h.group, NT, chunk_tiles(h.P, NT), value_group_bound(h));
 }
 
 // CTAs with `smem` bytes of dynamic shared memory that one SM holds.

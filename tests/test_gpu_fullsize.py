@@ -10,8 +10,9 @@ shaped layers), through the C ABI.
   sequences of 32,768 + 11 tokens with 8 KV heads at 12x (the heavy-tail stress
   layer's batch), checked on sampled (sequence, q head) pairs against the
   oracle's decode over its own copy of the pool, which must equal the library's
-  byte for byte.  The decode's launch plan (split count, stages) depends only
-  on the head shapes, widths and batch, so these runs use the benchmark's.
+  byte for byte.  The decode's launch plan (split count, stages, chunk length)
+  depends only on the head shapes, widths, page size and batch, so these runs
+  use the benchmark's.
 
 Bars as in the other parity tests: latents 1e-3 (per token and head-side, L2),
 packed pages bit-exact, attention 2e-3 (max over the sampled pairs of
@@ -140,15 +141,16 @@ def test_decode_qwen_128k_context_gqa7():
 
 
 def test_decode_stress_12x_batch16_32k():
-    """16 sequences at 32k with 8 KV heads and 12x widths.  Sequences 0 and 11
+    """16 sequences at 32k with 8 KV heads, 12x widths and the stress workload's
+    128-token pages (8-tile softmax chunks).  Sequences 0 and 11
     (sampled) are filled with seeded latents on both sides; the other 14 with
     device-drawn latents that only the library sees (their pages are not
     compared, their outputs not checked)."""
     torch = torch_mod()
     import spectral_transform_coding_b200 as st
-    seed, n_q, n_kv, B, length, P = 41, 32, 8, 16, 32768 + 11, 64
+    seed, n_q, n_kv, B, length, P = 41, 32, 8, 16, 32768 + 11, 128
     sampled = [0, 11]
-    codec, widths, _, W_up = _codec(512, n_q, n_kv, STRESS12X, STRESS12X, seed=seed)
+    codec, widths, _, W_up = _codec(512, n_q, n_kv, STRESS12X, STRESS12X, seed=seed, P=P)
     maxp = (length + P - 1) // P + 1
     rng = np.random.default_rng(seed + 1)
     table = rng.permutation(B * maxp).astype(np.int32).reshape(B, maxp)

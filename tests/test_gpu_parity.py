@@ -23,6 +23,9 @@ SHAPES = {
     "allwidths": (256, 4, 1, 128, 128, 16, [[8, 4, 3, 2, 1, 8, 1, 0], [1, 2, 3, 4, 8, 0, 3, 1]], 32),
     "zeroside": (256, 8, 1, 64, 64, 16, [[2, 1, 0, 0], [0, 0, 0, 0]], 64),
     "g8wide": (256, 16, 2, 64, 64, 8, [[8, 4, 3, 2, 1, 1, 0, 0], [3, 3, 2, 2, 1, 1, 1, 1]], 96),
+    # 128-token pages: softmax chunks of 8 tiles (one n-tile of q heads)
+    "stress12x_p128": (512, 8, 2, 128, 128, 16, [[4, 2, 0, 0, 0, 0, 0, 0], [4, 2, 0, 0, 0, 0, 0, 0]], 128),
+    "g8_p128": (256, 8, 2, 64, 64, 8, [[8, 4, 3, 2, 1, 1, 0, 0], [3, 3, 2, 2, 1, 1, 1, 1]], 128),
 }
 
 
@@ -180,8 +183,15 @@ def test_decode_peaked_queries(name):
     assert err <= 2e-3, err
 
 
-def test_decode_many_sequences_stress_shape():
-    err = _decode_case("stress12x", [257] * 16, seed=9)
+@pytest.mark.parametrize("name", ["stress12x", "stress12x_p128"])
+def test_decode_many_sequences_stress_shape(name):
+    err = _decode_case(name, [257] * 16, seed=9)
+    assert err <= 2e-3, err
+
+
+@pytest.mark.parametrize("lengths", [[1], [127], [128], [129], [1000], [0, 17]])
+def test_decode_edge_lengths_128_token_pages(lengths):
+    err = _decode_case("stress12x_p128", lengths, seed=4)
     assert err <= 2e-3, err
 
 

@@ -79,10 +79,11 @@ CONFIGS = {
         calib_tokens=8192, cache_len=131072, batch=1, spectrum_exp=2.0,
         dist="gaussian", nu=0.0, w_std=0.02, w_bf16=True, seed=2),
     # Llama shapes, multivariate Student-t (nu = 3) over the power-law
-    # covariance, 12x (floor(2048/12) = 170 bits per side), batch 16 @ 32k.
+    # covariance, 12x (floor(2048/12) = 170 bits per side), batch 16 @ 32k, in
+    # 128-token pages (the decode then takes 8-tile softmax chunks).
     "stress": WorkloadConfig(name="stress", budget_bits=170, cache_len=32768,
                              batch=16, seed=3,
-                             **dict(_LLAMA, dist="student_t", nu=3.0)),
+                             **dict(_LLAMA, dist="student_t", nu=3.0, page_tokens=128)),
     # Llama shapes, one 65,536-token prefill chunk encoded for all KV heads at 4x
     # (and 8x, see ``prefill8``), followed by one decode step.
     "prefill": WorkloadConfig(name="prefill", budget_bits=512, cache_len=65536,
