@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
 
   auto issue_copy = [&](int i, int pg_pid) {
     // copy the head section of page id pg_pid into stage i % S (one thread)
+    if (i == A.drop_page && (split | a | b) == 0) return;  // test hook: a copy that never lands
     const int s = i % S;
     const uint8_t* src = A.pool + (size_t)pg_pid * (size_t)A.page_bytes + sec_off;
     mbar_arrive_expect_tx(&bars[s], (uint32_t)sec_bytes);
@@ -587,14 +588,14 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     if (ld_volatile_s(&issued[s]) <= ph) {
       const uint64_t t0 = global_timer_ns();
       while (ld_volatile_s(&issued[s]) <= ph) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > A.wait_ns) {
           ok = false;
           break;
         }
       }
     }
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (uint32_t)(ph & 1), kWaitLimitNs));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (uint32_t)(ph & 1), A.wait_ns));
     if (!ok) {
       if (lane == 0) {
         device_error(cd->err, SPECTRA_ERR_TIMEOUT);
@@ -821,7 +822,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
   // ---- 8. drain copies that no warp consumed (errors, a hint above the length) -----
   __syncthreads();
   if (tid < S && issued[tid] > consumed[tid]) {
-    if (!mbar_wait_bounded(&bars[tid], (uint32_t)(consumed[tid] & 1), kWaitLimitNs))
+    if (!mbar_wait_bounded(&bars[tid], (uint32_t)(consumed[tid] & 1), A.wait_ns))
       device_error(cd->err, SPECTRA_ERR_TIMEOUT);
   }
   __syncthreads();
@@ -885,37 +886,32 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
       rec[tid * A.rec_stride + 1] = Ls;
     }
     __syncthreads();
-    if (tid < nkV) {
-      for (int h = 0; h < gq; ++h) {
-        const float* wt = wts + h * (kWarps + 2);
-        float v = 0.f;
+    for (int e = tid; e < gq * nkV; e += kThreads) {  // thread (head, coordinate)
+      const int h = e / nkV, c = e - h * nkV;
+      const float* wt = wts + h * (kWarps + 2);
+      float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) v = fmaf(wt[w], wsm[(w * gq + h) * kWs + 2 + tid], v);
-        rec[h * A.rec_stride + 4 + tid] = v;
-      }
+      for (int w = 0; w < kWarps; ++w) v = fmaf(wt[w], wsm[(w * gq + h) * kWs + 2 + c], v);
+      rec[h * A.rec_stride + 4 + c] = v;
     }
   }
   // ---- 10. the last CTA of this (sequence, KV head) merges the records and lifts ------
-  __threadfence();
+  // The barrier orders the CTA's record writes before thread 0's fence, which
+  // releases them (cumulatively) ahead of the arrival; the last CTA's thread 0
+  // fences again after its arrival (acquire) and the barrier passes that on.
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const int t = atomicAdd(A.cnt + unit, 1);
     const int last = t == ns - 1;
-    if (last) atomicExch(A.cnt + unit, 0);  // ready for the next call
+    if (last) __threadfence();
     flags[kFlagLast] = last;
   }
   __syncthreads();
   if (!flags[kFlagLast]) return;
-  __threadfence();
-  // W_up^V of this head into the (idle) stage ring while the records merge
   const uint32_t wv_bytes = (uint32_t)nkV * d_h * 4;
   const bool wv_staged = A.wv_staged != 0;
   float* wv_s = reinterpret_cast<float*>(stages);
-  if (tid == 0 && wv_staged && wv_bytes > 0) {
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&bars[kMaxStages], wv_bytes);
-    bulk_copy_g2s(wv_s, cd->w_up + hm[7], wv_bytes, &bars[kMaxStages]);
-  }
   float* wts = reinterpret_cast<float*>(smem + kOffQlat);   // [gq][kMaxSplit] weights (q_lat is dead)
   float* part = reinterpret_cast<float*>(smem + kOffX);     // [ch][gq][4 n4] partial merges
   float* lsum = reinterpret_cast<float*>(smem + kOffW);     // [gq] sum of weights x l
@@ -939,6 +935,12 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
 #pragma unroll
   for (int u = 0; u < 16; ++u)
     x[u] = u < nsp ? __ldcg(xb + (size_t)(k + u * ch) * (hs / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  // W_up^V of this head into the (idle) stage ring while the records merge
+  if (tid == 0 && wv_staged && wv_bytes > 0) {
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&bars[kMaxStages], wv_bytes);
+    bulk_copy_g2s(wv_s, cd->w_up + hm[7], wv_bytes, &bars[kMaxStages]);
+  }
   if (warp < gq) {  // warp h: the maximum and the weights of the splits for head h
     const int h = warp;
     float2 ml[kMaxSplit / 32];
@@ -995,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     reinterpret_cast<float4*>(part)[(size_t)k * pairs + pr] = v;
   }
   bool wv_ok = true;
-  if (wv_staged && wv_bytes > 0) wv_ok = mbar_wait_bounded(&bars[kMaxStages], 0u, kWaitLimitNs);
+  if (wv_staged && wv_bytes > 0) wv_ok = mbar_wait_bounded(&bars[kMaxStages], 0u, A.wait_ns);
   if (!wv_ok && tid == 0) device_error(cd->err, SPECTRA_ERR_TIMEOUT);
   __syncthreads();
   // chunks added in order into chunk 0: acc[h][c] = part[h * 4 n4 + c]
@@ -1027,6 +1029,9 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
     reinterpret_cast<float4*>(A.out + ((size_t)b * A.n_q + (size_t)a * gq + h) * d_h)[d4] =
         make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
   }
+  // every CTA of this unit has arrived: the counter is free for the next call
+  // (which starts only after this grid has completed)
+  if (tid == 0) A.cnt[unit] = 0;
 }
 
 

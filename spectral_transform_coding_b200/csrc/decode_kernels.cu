@@ -258,6 +258,15 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
     // then drain); the result may not change
     const char* e = std::getenv("SPECTRA_DECODE_HINT_LAG");
     args.hint_lag = e ? std::atoi(e) : 0;
+    // test hooks for the bounded waits: SPECTRA_DECODE_TEST_DROP_PAGE makes the
+    // first CTA skip the copy of that page of its list (its wait for the page
+    // then gives up and the call reports SPECTRA_ERR_TIMEOUT), and
+    // SPECTRA_DECODE_TEST_WAIT_NS shortens every wait's limit
+    const char* d = std::getenv("SPECTRA_DECODE_TEST_DROP_PAGE");
+    args.drop_page = d ? std::atoi(d) : -1;
+    const char* w = std::getenv("SPECTRA_DECODE_TEST_WAIT_NS");
+    const long long wn = w ? std::atoll(w) : 0;
+    args.wait_ns = wn > 0 ? (unsigned long long)wn : attend::kWaitLimitNs;
   }
   const auto kern = attend_kernel_for(h);
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), plan.smem_bytes);

@@ -399,16 +399,17 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
   }
   if (n_part > 1) {
     // the last CTA of this group to arrive adds the CTAs' partial sums in order
-    __threadfence();
+    // (barrier, then one thread's fence releases the partials before the
+    // arrival; the last CTA's thread fences again to acquire the others')
     __syncthreads();
     if (tid == 0) {
+      __threadfence();
       const int t = atomicAdd(counters + 1 + gi, 1);
       flag = t == n_part - 1;
-      if (flag) atomicExch(counters + 1 + gi, 0);
+      if (flag) __threadfence();
     }
     __syncthreads();
     if (!flag) return;
-    __threadfence();
     if (tid < T * G) {
       const int r = tid / G, c = tid % G;
       const float* pp = part + ((size_t)gi * n_part * TP + r) * G + c;
@@ -455,12 +456,16 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
   // The group that finishes last advances the lengths: every finishing CTA read
   // them (to place its tokens) before it arrived, and every page write precedes
   // the arrival of its CTA.  The counter is left at zero for the next call.
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const int t = atomicAdd(counters, 1);
     flag = t == (int)gridDim.x - 1;
-    if (flag) atomicExch(counters, 0);
+    if (flag) __threadfence();
+    // every CTA of this group has arrived (and, for the last group, every group):
+    // the counters are free for the next call, which starts after this grid
+    if (n_part > 1) counters[1 + gi] = 0;
+    if (flag) counters[0] = 0;
   }
   __syncthreads();
   if (flag && !worst && tid < T && (tid == T - 1 || seq_ids[tid + 1] != seq_ids[tid]))

@@ -96,3 +96,37 @@ def test_length_hint_does_not_change_the_result(lag, monkeypatch):
         got = codec.decode_attend(cache, q)
         codec.device_status()
         assert torch.equal(got, ref)
+
+
+def test_bounded_wait_gives_up_with_a_timeout_status(monkeypatch):
+    """A page copy that never lands (test hook SPECTRA_DECODE_TEST_DROP_PAGE: the
+    first CTA skips issuing it) makes that CTA's wait for the page give up after
+    the limit (shortened to 2 ms by SPECTRA_DECODE_TEST_WAIT_NS), drain its other
+    copies and finish; the call reports SPECTRA_ERR_TIMEOUT through the device
+    error word, and the next calls on the same context give the exact result."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    s = _setup("llama4x", seed=6)
+    codec = s["codec"]
+    lengths = [333, 64]
+    cache = st.LatentCache(codec, batch=len(lengths), max_pages_per_seq=8, device=dev())
+    seqs = np.concatenate([np.full(L, b, np.int32) for b, L in enumerate(lengths)])
+    lat = synthetic_latents(seqs.size, codec.n_eff, seed=12, decay=0.5, scale=2.0)
+    codec.quantize_append(cache, torch.from_numpy(lat).to(dev()), torch.from_numpy(seqs).to(dev()))
+    rng = np.random.default_rng(13)
+    q = torch.from_numpy((rng.standard_normal((len(lengths), s["n_q"], s["d_h"])) * 0.6).astype(np.float32)).to(dev())
+    ws = torch.zeros(codec.decode_workspace_bytes(len(lengths), cache.capacity), dtype=torch.uint8, device=dev())
+    ref = codec.decode_attend(cache, q, workspace=ws)
+    codec.device_status()
+    monkeypatch.setenv("SPECTRA_DECODE_TEST_DROP_PAGE", "0")
+    monkeypatch.setenv("SPECTRA_DECODE_TEST_WAIT_NS", "2000000")
+    codec.decode_attend(cache, q, workspace=ws)
+    with pytest.raises(st.SpectraError) as e:
+        codec.device_status()
+    assert e.value.status == 6  # SPECTRA_ERR_TIMEOUT
+    monkeypatch.delenv("SPECTRA_DECODE_TEST_DROP_PAGE")
+    monkeypatch.delenv("SPECTRA_DECODE_TEST_WAIT_NS")
+    for _ in range(2):  # the same workspace: its arrival counters were left at zero
+        got = codec.decode_attend(cache, q, workspace=ws)
+        codec.device_status()
+        assert torch.equal(got, ref)
