@@ -76,12 +76,12 @@ def _workload_name(cfg, layers):
 # one ncu capture of the current kernel on a 1-layer case of the workload; a
 # workload/kernel without a capture of its current code reports traffic null.
 #   attend_kernel, stress 12x (128-token pages), batch 16 x 32,771 tokens:
-#     169,248,000 B read + 3,470,336 B written for 167,787,520 packed bytes
-#   attend_kernel, Qwen 8x, 131,075 tokens: 34,034,432 B read, 0 written, for
+#     169,200,128 B read + 4,024,064 B written for 167,787,520 packed bytes
+#   attend_kernel, Qwen 8x, 131,075 tokens: 34,037,504 B read, 0 written, for
 #     33,555,200 packed bytes
 #   rt_split_kernel, Llama-shaped, 32k context: 34,214,912 B read, 0 written,
 #     for 33,560,576 packed bytes
-TRAFFIC_PER_ALGO_BYTE = {"stress": (169_248_000 + 3_470_336) / 167_787_520, "qwen": 34_034_432 / 33_555_200}
+TRAFFIC_PER_ALGO_BYTE = {"stress": (169_200_128 + 4_024_064) / 167_787_520, "qwen": 34_037_504 / 33_555_200}
 TRAFFIC_PER_PACKED_BYTE_RT = {"llama": 34_214_912 / 33_560_576}
 
 
