@@ -304,7 +304,13 @@ SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, con
  * may come straight from spectra_encode_append or spectra_quantize_append on
  * the same stream, with no synchronisation in between.  Needs d_head a
  * multiple of 16 and at most 256, at most 8 kept groups per head and side and
- * at most 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED). */
+ * at most 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED).
+ * Test hooks, read from the environment at every launch and meant for tests
+ * only: SPECTRA_DECODE_HINT_LAG (tokens taken off the early length hint; the
+ * result does not change), SPECTRA_DECODE_TEST_DROP_PAGE (the first CTA never
+ * issues the copy of that page of its list, so its bounded wait gives up and
+ * the call reports SPECTRA_ERR_TIMEOUT) and SPECTRA_DECODE_TEST_WAIT_NS (the
+ * limit of every bounded wait, default 200 ms). */
 SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, const spectra_cache* cache,
                                      const float* q, float* out, void* workspace,
                                      size_t workspace_bytes, void* stream);

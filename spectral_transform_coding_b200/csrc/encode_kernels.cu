@@ -363,6 +363,11 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
   };
   load_w(ch0);
   pdl_wait();  // H, lengths and the page table may come from earlier kernels
+  // positions of the step's tokens (their loads overlap the projection); every
+  // CTA that finishes a group reaches the same verdict from them
+  int64_t pos = 0;
+  int code_err = 0;
+  if (tid < T) code_err = append_position(seq_ids, tid, cache, cd->P, &pos);
   float acc[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
@@ -423,10 +428,6 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
     }
   }
   if (tid == 0) worst = 0;
-  // positions of the step's tokens; every finishing CTA reaches the same verdict
-  int64_t pos = 0;
-  int code_err = 0;
-  if (tid < T) code_err = append_position(seq_ids, tid, cache, cd->P, &pos);
   __syncthreads();
   if (code_err) atomicMax(&worst, code_err);
   __syncthreads();
