@@ -485,28 +485,39 @@ def run_decode(args, name, world, local):
     if check is not None:
         result["check"] = check
     if rt:
-        # algorithmic FLOPs per (token, KV head) = 2 n_kept_K d_h (lift) + 2 gq d_h
-        # (scores) + 2 gq n_kept_V (probability-weighted V latents), summed over the
-        # KV heads of a layer; reported against the fp32 CUDA-core peak (the lift runs
-        # as fp16 hi/lo MMAs, but the per-tile unpacking, rotation, scores and sums,
-        # which bound the kernel, are CUDA-core work)
+        # Two pipes.  CUDA cores: per (token, KV head) the rotation (6 FLOP per pair
+        # of dims = 3 d_h), the scores 2 gq d_h and the probability-weighted V
+        # latents 2 gq n_kept_V, against the fp32 peak.  Tensor cores: the key lift
+        # 2 n_kept_K d_h, issued as two fp16 MMAs (hi and lo parts of W_up^K), i.e.
+        # 4 n_kept_K d_h MMA FLOPs, against the bf16/fp16 dense peak.  The kernel's
+        # time bound is the larger of the two times; it is far above both (issue-
+        # and latency-bound per-tile phases).
         widths = codecs[0].state()["widths"]
         gq = cfg.n_q_heads // cfg.n_kv_heads
-        flop_tok = sum(2 * cfg.group * int((w[0] > 0).sum()) * cfg.d_head + 2 * gq * cfg.d_head
-                       + 2 * gq * cfg.group * int((w[1] > 0).sum()) for w in widths)
-        flops = B * len_after * flop_tok
+        alu_tok = sum(3 * cfg.d_head + 2 * gq * cfg.d_head + 2 * gq * cfg.group * int((w[1] > 0).sum())
+                      for w in widths)
+        mma_tok = sum(4 * cfg.group * int((w[0] > 0).sum()) * cfg.d_head for w in widths)
+        alu_flops = B * len_after * alu_tok
+        mma_flops = B * len_after * mma_tok
         alu_peak = 148 * 128 * 2 * 1965e6 / 1e12
-        tflops = flops / (dec_ms / 1e3) / 1e12
+        t_s = dec_ms / 1e3
+        alu_tflops = alu_flops / t_s / 1e12
+        mma_tflops = mma_flops / t_s / 1e12
+        bound_s = max(alu_flops / (alu_peak * 1e12), mma_flops / (peaks["bf16_tflops"] * 1e12))
         result["config"]["decode"] = f"reconstruct-then-attend, rotary base {args.rope_theta:g}"
         result["dtype"] = "u8 codes, fp16 scale/zero, fp32 lift and accumulate"
         result["roofline"] = {
             "kernel": "rt_split_kernel (keys rebuilt per 32-token tile on the tensor cores, rotated and scored "
                       "with fp32 FMAs; V summed in the latent space), timed with its combine launch",
-            "bound": "alu", "achieved": tflops, "peak": alu_peak, "unit": "TFLOP/s", "frac": tflops / alu_peak,
+            "bound": "alu", "achieved": alu_tflops, "peak": alu_peak, "unit": "TFLOP/s",
+            "frac": alu_tflops / alu_peak,
             "traffic": (TRAFFIC_PER_PACKED_BYTE_RT[name] * dec_bytes if name in TRAFFIC_PER_PACKED_BYTE_RT
                         else None),
-            "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm)",
-            "avg_launch_us": dec_ms * 1e3, "algorithmic_flops_per_launch": flops,
+            "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm); CUDA-core FLOPs only",
+            "avg_launch_us": dec_ms * 1e3, "cuda_core_flops_per_launch": alu_flops,
+            "tensor": {"mma_flops_per_launch": mma_flops, "tflops": mma_tflops, "peak": peaks["bf16_tflops"],
+                       "frac": mma_tflops / peaks["bf16_tflops"]},
+            "time_bound_us": bound_s * 1e6, "time_bound_frac": bound_s / t_s,
             "packed_bytes_per_launch": dec_bytes,
             "hbm_gbs": achieved, "hbm_frac": achieved / peaks["hbm_gbs"],
         }
