@@ -269,8 +269,11 @@ SPECTRA_API spectra_status spectra_quantize_append(const spectra_codec* codec, c
  * last chunk of a group adds them in chunk order and quantises the group
  * (latents summed in a different order than spectra_project's, so they may
  * differ from it in the last bits; the codes are those
- * spectra_quantize_append gives for these latents); the group that finishes
- * last advances the lengths.  For T >= 64 with latents_out
+ * spectra_quantize_append gives for these latents).  The lengths advance as
+ * soon as every CTA holds its positions, while the page writes may still be
+ * in flight: a kernel of this library that starts before this one completes
+ * (spectra_decode_attend) reads the lengths before its dependency wait only as
+ * a hint, 16 tokens short.  For T >= 64 with latents_out
  * NULL (prefill) the positions are planned and checked first, then the
  * tcgen05 projection GEMM quantises and packs each output tile in its
  * epilogue, so no fp32 latents are written; its accumulators equal
@@ -306,11 +309,12 @@ SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, con
  * multiple of 16 and at most 256, at most 8 kept groups per head and side and
  * at most 8 q heads per KV head (else SPECTRA_ERR_UNSUPPORTED).
  * Test hooks, read from the environment at every launch and meant for tests
- * only: SPECTRA_DECODE_HINT_LAG (tokens taken off the early length hint; the
- * result does not change), SPECTRA_DECODE_TEST_DROP_PAGE (the first CTA never
- * issues the copy of that page of its list, so its bounded wait gives up and
- * the call reports SPECTRA_ERR_TIMEOUT) and SPECTRA_DECODE_TEST_WAIT_NS (the
- * limit of every bounded wait, default 200 ms). */
+ * only: SPECTRA_DECODE_HINT_LAG (tokens taken off the early length hint beyond
+ * the built-in 16; the result does not change), SPECTRA_DECODE_TEST_DROP_PAGE
+ * (the first CTA never issues the copy of that page of its list, so its
+ * bounded wait gives up and the call reports SPECTRA_ERR_TIMEOUT) and
+ * SPECTRA_DECODE_TEST_WAIT_NS (the limit of every bounded wait, default
+ * 200 ms). */
 SPECTRA_API spectra_status spectra_decode_attend(const spectra_codec* codec, const spectra_cache* cache,
                                      const float* q, float* out, void* workspace,
                                      size_t workspace_bytes, void* stream);

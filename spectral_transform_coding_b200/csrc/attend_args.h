@@ -63,7 +63,7 @@ struct AttendArgs {
   int n_q;
   int n_kv;
   int d_h;
-  int hint_lag;     // tokens taken off the length hint (test hook, see launch_decode)
+  int hint_lag;     // tokens taken off the length hint (16, plus a test offset; see launch_decode)
   int drop_page;    // test hook: page of CTA (0, 0, 0) whose copy is never issued; -1: none
   unsigned long long wait_ns;  // limit of every bounded wait (kWaitLimitNs unless a test shortens it)
   float q_scale;

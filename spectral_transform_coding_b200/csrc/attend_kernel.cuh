@@ -350,8 +350,10 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendArgs A)
   // CTA's pages w, w + 8, ... in order, so the partition and the summation
   // order depend only on the final length.  The lengths only grow (appends)
   // while a kernel of this library may still be running before the dependency
-  // wait, so the hint read here is at most the final length, and pages that
-  // are full under it are final: their copies go out before the wait.
+  // wait, so the hint read here is at most the final length.  A running fused
+  // encode may have advanced it by up to hint_lag tokens before its page
+  // writes land, so pages full hint_lag tokens below the hint are final: their
+  // copies go out before the wait.
   int hint_raw = 0, pid = -1;
   if (warp == 0) {
     hint_raw = __ldcg(A.lengths + b);

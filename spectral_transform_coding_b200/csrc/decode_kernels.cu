@@ -17,7 +17,8 @@
 // its host side: the launch plan and the launch.  The grid is (context split,
 // KV head, sequence), one CTA per split:
 //   prologue (before the dependency wait; reads only the caller's q, read-only
-//     codec data, the lengths as a hint and pages that are full under the hint):
+//     codec data, the lengths as a hint and pages that are full 16 tokens below
+//     the hint):
 //     bulk copies of the first pages into a CTA-wide ring of shared-memory
 //     stages; the fold q_lat = q W_up^K^T of all kept K coordinates; the MMA B
 //     fragments of q_lat;
@@ -256,8 +257,12 @@ cudaError_t launch_decode(const CodecDev& h, const CodecDev* d, const spectra_ca
     // positive lag sends the copies of more pages after the dependency wait, a
     // negative one makes the kernel copy pages beyond the length, which it must
     // then drain); the result may not change
+    // The built-in lag: a fused decode-step encode that is still running may
+    // have advanced the lengths by up to kFusedMaxT tokens per sequence before
+    // its page writes land (only one such encode at a time: it writes the
+    // lengths after its own wait, when every earlier kernel has completed).
     const char* e = std::getenv("SPECTRA_DECODE_HINT_LAG");
-    args.hint_lag = e ? std::atoi(e) : 0;
+    args.hint_lag = kFusedMaxT + (e ? std::atoi(e) : 0);
     // test hooks for the bounded waits: SPECTRA_DECODE_TEST_DROP_PAGE makes the
     // first CTA skip the copy of that page of its list (its wait for the page
     // then gives up and the call reports SPECTRA_ERR_TIMEOUT), and

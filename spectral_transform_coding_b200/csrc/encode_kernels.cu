@@ -258,9 +258,10 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
 // ---------------------------------------------------------------------------
 namespace {
 
-// Cache position of token t of an append (seq_ids non-decreasing), or an error.
+// Cache position of token t of an append (seq_ids non-decreasing) and the page
+// id it lands in, or an error.
 __device__ __forceinline__ int append_position(const int32_t* __restrict__ seq_ids, int t,
-                                               const spectra_cache& c, int P, int64_t* pos) {
+                                               const spectra_cache& c, int P, int64_t* pos, int* page = nullptr) {
   const int s = seq_ids[t];
   if (s < 0 || s >= c.batch || (t > 0 && seq_ids[t - 1] > s)) return SPECTRA_ERR_ORDER;
   int first = t;
@@ -270,6 +271,7 @@ __device__ __forceinline__ int append_position(const int32_t* __restrict__ seq_i
   const int pid = c.page_table[(size_t)s * c.max_pages_per_seq + p / P];
   if (pid < 0 || (int64_t)pid >= c.n_pages) return SPECTRA_ERR_CAPACITY;
   *pos = p;
+  if (page) *page = pid;
   return 0;
 }
 
@@ -307,13 +309,14 @@ __device__ __forceinline__ float warp_transpose_sum(float (&vals)[V], int lane) 
 __host__ __device__ constexpr int log2_int(int v) { return v <= 1 ? 0 : 1 + log2_int(v / 2); }
 
 constexpr int kMaxChunks = 16;  // d_model chunks per group (the plan keeps to it)
+constexpr int kFusedMaxStageBytes = 96 * 1024;  // staged W_down per CTA
+constexpr unsigned long long kFusedWaitLimitNs = 200ull * 1000ull * 1000ull;  // bounded wait for staged copies
 
 }  // namespace
 
 template <int G, int TP, int BATCH>
-__global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __restrict__ cd,
-                                                           const uint16_t* __restrict__ H, int T,
-                                                           const int32_t* __restrict__ seq_ids,
+__global__ void __launch_bounds__(256) encode_fused_kernel(const EncodeFusedArgs A, const uint16_t* __restrict__ H,
+                                                           int T, const int32_t* __restrict__ seq_ids,
                                                            const spectra_cache cache,
                                                            float* __restrict__ latents_out,
                                                            int32_t* __restrict__ counters,
@@ -321,34 +324,40 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
   constexpr int CPW = G / 8;        // columns per warp (8 warps cover the group)
   constexpr int KCH = 256 * BATCH;  // d_model columns of H per chunk
   constexpr int V = CPW * TP;       // partial sums per lane
+  extern __shared__ __align__(128) uint8_t w_s[];  // staged chunks: [chunk - ch0 - 1][G][KCH] bf16
   __shared__ float x_s[TP][G];
+  __shared__ int64_t pos_s[TP];
+  __shared__ int pid_s[TP];
+  __shared__ __align__(8) uint64_t w_bar;
   __shared__ int worst;
   __shared__ int flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
-  // this CTA's group (kept groups numbered head-major, K side then V side) and
-  // its chunks [ch0, ch1) of d_model
+  // this CTA's kept group gi (numbered head-major, K side then V side: latent
+  // columns gi G .. gi G + G - 1) and its chunks [ch0, ch1) of d_model
   const int gi = blockIdx.x, n_part = gridDim.y;
-  const int ch0 = blockIdx.y * cpc, ch1 = min(n_chunks, ch0 + cpc);
-  int a = 0, sd_i = 0, g = gi;
-  for (; a < cd->n_kv; ++a) {
-    int side = 0;
-    for (; side < 2; ++side) {
-      const int n = cd->head[a].side[side].n_groups;
-      if (g < n) break;
-      g -= n;
-    }
-    if (side < 2) {
-      sd_i = side;
-      break;
+  const int ch0 = blockIdx.y * cpc;
+  int ch1 = min(n_chunks, ch0 + cpc);
+  const int d_model = A.d_model;
+  const int n0 = gi * G + warp * CPW;  // latent columns of this warp
+  // W_down rows of the group (read-only codec data) all go out before the
+  // wait: the first chunk into registers, this warp's columns; with `staged`
+  // the later chunks by bulk copies into shared memory, else into registers
+  // after the wait
+  const bool staged = A.staged && ch1 - ch0 > 1;
+  if (staged && tid == 0) {
+    mbar_init(&w_bar, 1);
+    fence_mbar_init();
+    uint32_t bytes = 0;
+    for (int ch = ch0 + 1; ch < ch1; ++ch) bytes += (uint32_t)(G * 2 * min(KCH, d_model - ch * KCH));
+    mbar_arrive_expect_tx(&w_bar, bytes);
+    for (int ch = ch0 + 1; ch < ch1; ++ch) {
+      const int len = min(KCH, d_model - ch * KCH);
+      for (int r = 0; r < G; ++r)
+        bulk_copy_g2s(w_s + ((size_t)(ch - ch0 - 1) * G + r) * (KCH * 2),
+                      A.wt_down + (size_t)(gi * G + r) * d_model + (size_t)ch * KCH, (uint32_t)len * 2u, &w_bar);
     }
   }
-  const SideDev& sd = cd->head[a].side[sd_i];
-  const GroupDev gd = sd.grp[g];
-  const int d_model = cd->d_model;
-  const int n0 = sd.c_col0 + gd.col + warp * CPW;  // latent columns of this warp
-  // W_down rows of this warp's columns over the first chunk: read-only codec
-  // data, loaded before the wait; later chunks are loaded after it
   uint4 wv[CPW][BATCH];
   auto load_w = [&](int ch) {
 #pragma unroll
@@ -356,23 +365,73 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
 #pragma unroll
       for (int c = 0; c < CPW; ++c) {
         const int k = ch * KCH + lane * 8 + 256 * i;
-        wv[c][i] = k < d_model
-                       ? __ldg(reinterpret_cast<const uint4*>(cd->wt_down + (size_t)(n0 + c) * d_model + k))
+        wv[c][i] = k < d_model ? __ldg(reinterpret_cast<const uint4*>(A.wt_down + (size_t)(n0 + c) * d_model + k))
+                               : make_uint4(0u, 0u, 0u, 0u);
+      }
+  };
+  auto stage_w = [&](int ch) {
+    const uint8_t* src = w_s + (size_t)(ch - ch0 - 1) * G * (KCH * 2);
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i)
+#pragma unroll
+      for (int c = 0; c < CPW; ++c) {
+        const int kl = lane * 8 + 256 * i;
+        wv[c][i] = ch * KCH + kl < d_model
+                       ? *reinterpret_cast<const uint4*>(src + ((size_t)(warp * CPW + c) * KCH + kl) * 2)
                        : make_uint4(0u, 0u, 0u, 0u);
       }
   };
   load_w(ch0);
+  const int4 cg = __ldg(reinterpret_cast<const int4*>(A.col_groups) + gi);  // {width, block off, record off, side}
   pdl_wait();  // H, lengths and the page table may come from earlier kernels
   // positions of the step's tokens (their loads overlap the projection); every
   // CTA that finishes a group reaches the same verdict from them
-  int64_t pos = 0;
-  int code_err = 0;
-  if (tid < T) code_err = append_position(seq_ids, tid, cache, cd->P, &pos);
+  if (warp == 0) {  // T <= 16
+    int e = 0;
+    int64_t pos = 0;
+    if (lane < T) {
+      int pid = 0;
+      e = append_position(seq_ids, lane, cache, A.P, &pos, &pid);
+      pos_s[lane] = pos;
+      pid_s[lane] = pid;
+    }
+    e = __reduce_max_sync(0xffffffffu, e);  // also orders the lanes' reads before the arrival
+    // Every CTA arrives once it holds its positions; the last to arrive advances
+    // the lengths at once (no CTA of this grid reads them afterwards) and leaves
+    // the counter at zero for the next call.  The lengths thus run ahead of this
+    // grid's page writes by at most T tokens per sequence until it completes; a
+    // decode that starts early copies only pages full kFusedMaxT tokens below
+    // its length hint before its own dependency wait.
+    int last = 0;
+    if (lane == 0) {
+      worst = e;
+      last = atom_add_acq_rel(counters, 1) == (int)(gridDim.x * gridDim.y) - 1;
+      if (last) counters[0] = 0;
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last && !e && lane < T && (lane == T - 1 || seq_ids[lane + 1] != seq_ids[lane]))
+      cache.lengths[seq_ids[lane]] = (int32_t)(pos + 1);
+  }
   float acc[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  if (staged) {
+    __syncthreads();  // the barrier is initialised
+    // bounded: a copy that never lands ends in a status (no writes; the
+    // arrivals below still happen), not a hang
+    if (!__syncthreads_and(mbar_wait_bounded(&w_bar, 0, A.wait_ns))) {
+      if (tid == 0) {
+        device_error(A.err, SPECTRA_ERR_TIMEOUT);
+        atomicMax(&worst, SPECTRA_ERR_TIMEOUT);
+      }
+      ch1 = ch0 + 1;
+    }
+  }
   for (int ch = ch0; ch < ch1; ++ch) {
-    if (ch > ch0) load_w(ch);
+    if (ch > ch0) {
+      if (staged) stage_w(ch);
+      else load_w(ch);
+    }
 #pragma unroll
     for (int r = 0; r < TP; ++r) {
       if (r < T) {
@@ -427,50 +486,41 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const CodecDev* __res
       x_s[r][c] = x;
     }
   }
-  if (tid == 0) worst = 0;
   __syncthreads();
-  if (code_err) atomicMax(&worst, code_err);
-  __syncthreads();
-  if (worst && gi == 0 && tid == 0) device_error(cd->err, worst);
-  if (!worst && tid < T) {
-    float x[G];
-#pragma unroll
-    for (int k = 0; k < G; ++k) x[k] = x_s[tid][k];
-    if (latents_out) {
-      float* lo = latents_out + (size_t)tid * cd->n_eff + sd.c_col0 + gd.col;
-#pragma unroll
-      for (int k = 0; k < G; ++k) lo[k] = x[k];
+  const int bad = worst;
+  if (bad && gi == 0 && tid == 0) device_error(A.err, bad);
+  // quantise and pack: half warp t takes token t, lane k of the half latent k
+  {
+    const int t = tid >> 4, k = tid & 15;
+    if (!bad && t < T) {
+      const float x = x_s[t][k < G ? k : 0];
+      if (latents_out && k < G) latents_out[(size_t)t * A.n_eff + gi * G + k] = x;
+      const int P = A.P, TB = 256 / G;
+      const int64_t pos = pos_s[t];
+      uint8_t* page = static_cast<uint8_t*>(cache.pool) + (size_t)pid_s[t] * (size_t)A.page_bytes;
+      const int tau = (int)(pos % P), b = cg.x;
+      __half s_h, z_h;
+      const uint32_t code = quantize_half_warp(x, b, s_h, z_h);
+      if (k < G) {
+        int g8, t4, slot;
+        if (cg.w == 0) k_side_pos<G>(tau % TB, k, &g8, &t4, &slot);
+        else v_side_pos<G>(tau % TB, k, &g8, &t4, &slot);
+        const CodeBits cb = code_bits(b, g8, t4, slot, code);
+        uint32_t* blkw = reinterpret_cast<uint32_t*>(page + cg.y + (tau / TB) * (32 * b));
+        // other lanes' and tokens' bits share these words: clear and set only ours
+        atomicAnd(blkw + cb.w0, ~cb.m0);
+        atomicOr(blkw + cb.w0, cb.v0);
+        if (cb.w1 >= 0) {
+          atomicAnd(blkw + cb.w1, ~cb.m1);
+          atomicOr(blkw + cb.w1, cb.v1);
+        }
+      }
+      if (k == 0) put_record(page + cg.z, P, tau, s_h, z_h);
     }
-    const int P = cd->P, TB = 256 / G;
-    const int seq = seq_ids[tid];
-    const int pid = cache.page_table[(size_t)seq * cache.max_pages_per_seq + pos / P];
-    uint8_t* page = static_cast<uint8_t*>(cache.pool) + (size_t)pid * (size_t)cd->page_bytes;
-    const int tau = (int)(pos % P);
-    const int b = gd.b;
-    __half s_h, z_h;
-    uint32_t code[G];
-    quantize_group<G>(x, b, s_h, z_h, code);
-    uint32_t* blkw = reinterpret_cast<uint32_t*>(page + gd.plane_off + (tau / TB) * (32 * b));
-    put_codes<G, false>(blkw, sd_i, tau % TB, b, code);
-    put_record(page + gd.sz_off, P, tau, s_h, z_h);
   }
-  // The group that finishes last advances the lengths: every finishing CTA read
-  // them (to place its tokens) before it arrived, and every page write precedes
-  // the arrival of its CTA.  The counter is left at zero for the next call.
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const int t = atomicAdd(counters, 1);
-    flag = t == (int)gridDim.x - 1;
-    if (flag) __threadfence();
-    // every CTA of this group has arrived (and, for the last group, every group):
-    // the counters are free for the next call, which starts after this grid
-    if (n_part > 1) counters[1 + gi] = 0;
-    if (flag) counters[0] = 0;
-  }
-  __syncthreads();
-  if (flag && !worst && tid < T && (tid == T - 1 || seq_ids[tid + 1] != seq_ids[tid]))
-    cache.lengths[seq_ids[tid]] = (int32_t)(pos + 1);
+  // every CTA of this group has arrived: its counter is free for the next call,
+  // which starts after this grid
+  if (n_part > 1 && tid == 0) counters[1 + gi] = 0;
 }
 
 // Advances the lengths of an append that writes no codes (a codec that keeps
@@ -571,6 +621,11 @@ EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T) {
   const long per_group = p.n_groups > 0 ? std::max(1L, target / p.n_groups) : 1L;
   p.cpc = T >= 4 ? 1 : (int)((p.n_chunks + per_group - 1) / per_group);
   p.n_part = (p.n_chunks + p.cpc - 1) / p.cpc;
+  // the chunks after a CTA's first go to shared memory by bulk copies before the
+  // wait when they fit beside a running decode CTA
+  const int stage = (p.cpc - 1) * h.group * 256 * p.batch * 2;
+  p.staged = p.cpc > 1 && stage <= kFusedMaxStageBytes && h.d_model % 8 == 0;
+  p.smem_bytes = p.staged ? stage : 0;
   return p;
 }
 
@@ -581,28 +636,28 @@ size_t encode_fused_partial_bytes(const CodecDev& h, int T) {
 
 namespace {
 template <int G, int TP>
-cudaError_t launch_fused_tp(const EncodeFusedPlan& p, const CodecDev* d, const uint16_t* H, int T,
+cudaError_t launch_fused_tp(const EncodeFusedPlan& p, const EncodeFusedArgs& args, const uint16_t* H, int T,
                             const int32_t* seq_ids, const spectra_cache& cache, float* latents_out,
                             int32_t* counters, float* part, cudaStream_t st) {
   const dim3 grid(p.n_groups, p.n_part), block(256);
+  auto go = [&](auto kern) -> cudaError_t {
+    if (p.smem_bytes > 0) {
+      const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), p.smem_bytes);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_dependent(kern, grid, block, p.smem_bytes, st, args, H, T, seq_ids, cache, latents_out, counters,
+                            part, p.n_chunks, p.cpc);
+  };
   switch (p.batch) {
-    case 8:
-      return launch_dependent(encode_fused_kernel<G, TP, 8>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                              latents_out, counters, part, p.n_chunks, p.cpc);
-    case 4:
-      return launch_dependent(encode_fused_kernel<G, TP, 4>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                              latents_out, counters, part, p.n_chunks, p.cpc);
-    case 2:
-      return launch_dependent(encode_fused_kernel<G, TP, 2>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                              latents_out, counters, part, p.n_chunks, p.cpc);
-    default:
-      return launch_dependent(encode_fused_kernel<G, TP, 1>, grid, block, 0, st, d, H, T, seq_ids, cache,
-                              latents_out, counters, part, p.n_chunks, p.cpc);
+    case 8: return go(encode_fused_kernel<G, TP, 8>);
+    case 4: return go(encode_fused_kernel<G, TP, 4>);
+    case 2: return go(encode_fused_kernel<G, TP, 2>);
+    default: return go(encode_fused_kernel<G, TP, 1>);
   }
 }
 
 template <int G>
-cudaError_t launch_fused_g(const EncodeFusedPlan& p, const CodecDev* d, const uint16_t* H, int T,
+cudaError_t launch_fused_g(const EncodeFusedPlan& p, const EncodeFusedArgs& d, const uint16_t* H, int T,
                            const int32_t* seq_ids, const spectra_cache& cache, float* latents_out,
                            int32_t* counters, float* part, cudaStream_t st) {
   switch (p.tp) {
@@ -621,8 +676,19 @@ cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint
   const EncodeFusedPlan p = encode_fused_plan(h, T);
   if (p.n_groups == 0) return launch_length_advance(seq_ids, T, cache, h.P, st, h.err);
   if (T > kFusedMaxT || p.n_groups > kMaxFusedGroups || p.n_part > kMaxChunks) return cudaErrorNotSupported;
-  if (h.group == 16) return launch_fused_g<16>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
-  return launch_fused_g<8>(p, d, H, T, seq_ids, cache, latents_out, counters, part, st);
+  (void)d;
+  EncodeFusedArgs args;
+  args.wt_down = h.wt_down;
+  args.col_groups = h.col_groups;
+  args.err = h.err;
+  args.page_bytes = h.page_bytes;
+  args.wait_ns = kFusedWaitLimitNs;
+  args.d_model = h.d_model;
+  args.n_eff = h.n_eff;
+  args.P = h.P;
+  args.staged = p.staged;
+  if (h.group == 16) return launch_fused_g<16>(p, args, H, T, seq_ids, cache, latents_out, counters, part, st);
+  return launch_fused_g<8>(p, args, H, T, seq_ids, cache, latents_out, counters, part, st);
 }
 
 }  // namespace spectra

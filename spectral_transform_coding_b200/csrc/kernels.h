@@ -50,8 +50,20 @@ constexpr int kFusedMaxT = 16;
 // to a power of two.
 struct EncodeFusedPlan {
   int n_groups, n_chunks, batch, cpc, n_part, tp;
+  int staged, smem_bytes;  // chunks after a CTA's first staged in shared memory (bytes per CTA)
 };
 constexpr int kMaxFusedGroups = kMaxKV * 2 * kMaxGroups;
+// What the fused encode reads of the codec, passed by value so that its first
+// W_down loads depend on no global load.
+struct EncodeFusedArgs {
+  const uint16_t* wt_down;
+  const int32_t* col_groups;  // per kept group {width, block offset, record offset, side}
+  int32_t* err;
+  int64_t page_bytes;
+  unsigned long long wait_ns;  // limit of the wait for staged W_down copies
+  int d_model, n_eff, P;
+  int staged;  // chunks after a CTA's first are bulk-copied into shared memory
+};
 EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T);
 // Workspace bytes of the fused encode's partial sums for T tokens.
 size_t encode_fused_partial_bytes(const CodecDev& h, int T);

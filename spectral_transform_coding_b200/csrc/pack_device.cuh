@@ -22,6 +22,22 @@ namespace pack {
 
 __device__ __forceinline__ float sat16(float x) { return fminf(fmaxf(x, -65504.f), 65504.f); }
 
+// Scale and zero of a group with extremes mn, mx at width b:
+// s = fp16(sat((mx - mn) / (2^b - 1))), z = fp16(sat(mn)).
+__device__ __forceinline__ void scale_zero(float mn, float mx, int b, __half& s_h, __half& z_h) {
+  const float levels = (float)((1 << b) - 1);
+  s_h = __float2half_rn(sat16(__fdiv_rn(__fsub_rn(mx, mn), levels)));
+  z_h = __float2half_rn(sat16(mn));
+}
+
+// code = clamp(rint((x - z) / s), 0, 2^b - 1), 0 when s == 0.
+__device__ __forceinline__ uint32_t code_of(float x, int b, __half s_h, __half z_h) {
+  const float sf = __half2float(s_h), zf = __half2float(z_h);
+  if (!(sf > 0.f)) return 0u;
+  const float t = __fdiv_rn(__fsub_rn(x, zf), sf);
+  return (uint32_t)fminf(fmaxf(rintf(t), 0.f), (float)((1 << b) - 1));
+}
+
 // One token's group of G fp32 latents at width b (every step one IEEE fp32
 // operation): s = fp16(sat((max - min) / (2^b - 1))), z = fp16(sat(min)),
 // code = clamp(rint((x - z) / s), 0, 2^b - 1), all codes 0 when s == 0.
@@ -34,19 +50,24 @@ __device__ __forceinline__ void quantize_group(const float (&x)[G], int b, __hal
     mn = fminf(mn, x[k]);
     mx = fmaxf(mx, x[k]);
   }
-  const float levels = (float)((1 << b) - 1);
-  s_h = __float2half_rn(sat16(__fdiv_rn(__fsub_rn(mx, mn), levels)));
-  z_h = __float2half_rn(sat16(mn));
-  const float sf = __half2float(s_h), zf = __half2float(z_h);
+  scale_zero(mn, mx, b, s_h, z_h);
 #pragma unroll
-  for (int k = 0; k < G; ++k) {
-    float c = 0.f;
-    if (sf > 0.f) {
-      const float t = __fdiv_rn(__fsub_rn(x[k], zf), sf);
-      c = fminf(fmaxf(rintf(t), 0.f), levels);
-    }
-    code[k] = (uint32_t)c;
+  for (int k = 0; k < G; ++k) code[k] = code_of(x[k], b, s_h, z_h);
+}
+
+// The same quantiser with the group spread over the 16 lanes of a half warp:
+// lane k of the half holds latent k (lanes k >= G repeat latent 0, which leaves
+// the extremes unchanged) and gets code k; s and z are the same in every lane.
+__device__ __forceinline__ uint32_t quantize_half_warp(float x, int b, __half& s_h, __half& z_h) {
+  const unsigned half = 0xFFFFu << (threadIdx.x & 16);
+  float mn = x, mx = x;
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(half, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(half, mx, o));
   }
+  scale_zero(mn, mx, b, s_h, z_h);
+  return code_of(x, b, s_h, z_h);
 }
 
 // Fragment position (gid, t4, slot) of entry (token tb of the block, coordinate k).
@@ -80,6 +101,42 @@ __device__ __forceinline__ void v_side_pos(int tb, int k, int* gid, int* t4, int
   }
 }
 
+// Block word(s) and bits of one code of width b at fragment position (gid, t4,
+// slot), the page layout's width rule:
+//   b = 4: word 4 gid + t4, nibble `slot`;
+//   b = 2: word 2 gid + t4/2, bits 4 slot + 2 (t4 % 2) + {0, 1};
+//   b = 1: word gid, bit 4 slot + t4;
+//   b = 3: bits 0-1 as b = 2, bit 2 as b = 1 in word 16 + gid (the second word);
+//   b = 8: word 2 (4 gid + t4) + (slot / 2) % 2, byte (slot % 2) + 2 (slot / 4).
+// w1 < 0 when the code has no second word.
+struct CodeBits {
+  int w0, w1;
+  uint32_t m0, v0, m1, v1;
+};
+
+__device__ __forceinline__ CodeBits code_bits(int b, int gid, int t4, int slot, uint32_t code) {
+  CodeBits r{-1, -1, 0u, 0u, 0u, 0u};
+  int sh;
+  uint32_t wm;
+  switch (b) {
+    case 4: r.w0 = 4 * gid + t4; sh = 4 * slot; wm = 0xFu; break;
+    case 2: r.w0 = 2 * gid + (t4 >> 1); sh = 4 * slot + 2 * (t4 & 1); wm = 0x3u; break;
+    case 1: r.w0 = gid; sh = 4 * slot + t4; wm = 0x1u; break;
+    case 3:
+      r.w0 = 2 * gid + (t4 >> 1);
+      sh = 4 * slot + 2 * (t4 & 1);
+      wm = 0x3u;
+      r.w1 = 16 + gid;
+      r.m1 = 1u << (4 * slot + t4);
+      r.v1 = ((code >> 2) & 1u) << (4 * slot + t4);
+      break;
+    default: r.w0 = 2 * (4 * gid + t4) + ((slot >> 1) & 1); sh = 8 * ((slot & 1) + 2 * (slot >> 2)); wm = 0xFFu; break;
+  }
+  r.m0 = wm << sh;
+  r.v0 = (code & wm) << sh;
+  return r;
+}
+
 // Pending bits of one block word: consecutive entries that land in the same word
 // are merged.  Global words (kShared = false) are written with one atomicAnd /
 // atomicOr pair (other tokens of the block may be written concurrently or may
@@ -100,38 +157,22 @@ __device__ __forceinline__ void flush_word(uint32_t* blk, WordBits& a) {
 }
 
 template <bool kShared>
-__device__ __forceinline__ void put_bits(uint32_t* blk, WordBits& a, int w, int shift, uint32_t width_mask,
-                                         uint32_t v) {
+__device__ __forceinline__ void put_bits(uint32_t* blk, WordBits& a, int w, uint32_t mask, uint32_t val) {
   if (w != a.w) {
     flush_word<kShared>(blk, a);
     a.w = w;
   }
-  a.mask |= width_mask << shift;
-  a.val |= (v & width_mask) << shift;
+  a.mask |= mask;
+  a.val |= val;
 }
 
-// Writes one code (width b) of fragment position (gid, t4, slot) into a block:
-//   b = 4: word 4 gid + t4, nibble `slot`;
-//   b = 2: word 2 gid + t4/2, bits 4 slot + 2 (t4 % 2) + {0, 1};
-//   b = 1: word gid, bit 4 slot + t4;
-//   b = 3: bits 0-1 as b = 2, bit 2 as b = 1 in words 16 + gid (second pending word);
-//   b = 8: word 2 (4 gid + t4) + (slot / 2) % 2, byte (slot % 2) + 2 (slot / 4).
+// Writes one code (width b) of fragment position (gid, t4, slot) into a block.
 template <bool kShared>
 __device__ __forceinline__ void put_code(uint32_t* blk, WordBits& a, WordBits& a1, int b, int gid, int t4,
                                          int slot, uint32_t code) {
-  switch (b) {
-    case 4: put_bits<kShared>(blk, a, 4 * gid + t4, 4 * slot, 0xFu, code); break;
-    case 2: put_bits<kShared>(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code); break;
-    case 1: put_bits<kShared>(blk, a, gid, 4 * slot + t4, 0x1u, code); break;
-    case 3:
-      put_bits<kShared>(blk, a, 2 * gid + (t4 >> 1), 4 * slot + 2 * (t4 & 1), 0x3u, code);
-      put_bits<kShared>(blk, a1, 16 + gid, 4 * slot + t4, 0x1u, code >> 2);
-      break;
-    default:
-      put_bits<kShared>(blk, a, 2 * (4 * gid + t4) + ((slot >> 1) & 1), 8 * ((slot & 1) + 2 * (slot >> 2)), 0xFFu,
-                        code);
-      break;
-  }
+  const CodeBits c = code_bits(b, gid, t4, slot, code);
+  put_bits<kShared>(blk, a, c.w0, c.m0, c.v0);
+  if (c.w1 >= 0) put_bits<kShared>(blk, a1, c.w1, c.m1, c.v1);
 }
 
 // Scale/zero of page token tau: record of its pair u = tau/2 at index
