@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const EncodeFusedArgs
   constexpr int V = CPW * TP;       // partial sums per lane
   extern __shared__ __align__(128) uint8_t w_s[];  // staged chunks: [chunk - ch0 - 1][G][KCH] bf16
   __shared__ float x_s[TP][G];
+  __shared__ float red_s[kMaxChunks * TP * G];  // cluster rank 0: the group's partial sums [rank][TP][G]
   __shared__ int64_t pos_s[TP];
   __shared__ int pid_s[TP];
   __shared__ __align__(8) uint64_t w_bar;
@@ -458,10 +459,23 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const EncodeFusedArgs
     const int v = lane >> SH, c = v / TP, r = v % TP;
     if ((lane & ((1 << SH) - 1)) == 0 && r < T) {
       if (n_part == 1) x_s[r][warp * CPW + c] = tot;
+      else if (A.cluster)
+        st_shared_cluster_f32(mapa_shared(smem_u32(&red_s[(blockIdx.y * TP + r) * G + warp * CPW + c]), 0), tot);
       else part[((size_t)(gi * n_part + blockIdx.y) * TP + r) * G + warp * CPW + c] = tot;
     }
   }
-  if (n_part > 1) {
+  if (n_part > 1 && A.cluster) {
+    // the group's CTAs are one cluster (rank = blockIdx.y): rank 0 adds the
+    // partial sums that every rank stored into its shared memory, in rank order
+    cluster_sync_all();
+    if (blockIdx.y != 0) return;
+    if (tid < T * G) {
+      const int r = tid / G, c = tid % G;
+      float x = 0.f;
+      for (int k = 0; k < n_part; ++k) x += red_s[(k * TP + r) * G + c];
+      x_s[r][c] = x;
+    }
+  } else if (n_part > 1) {
     // the last CTA of this group to arrive adds the CTAs' partial sums in order
     // (barrier, then one thread's fence releases the partials before the
     // arrival; the last CTA's thread fences again to acquire the others')
@@ -520,7 +534,7 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const EncodeFusedArgs
   }
   // every CTA of this group has arrived: its counter is free for the next call,
   // which starts after this grid
-  if (n_part > 1 && tid == 0) counters[1 + gi] = 0;
+  if (n_part > 1 && !A.cluster && tid == 0) counters[1 + gi] = 0;
 }
 
 // Advances the lengths of an append that writes no codes (a codec that keeps
@@ -626,6 +640,12 @@ EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T) {
   const int stage = (p.cpc - 1) * h.group * 256 * p.batch * 2;
   p.staged = p.cpc > 1 && stage <= kFusedMaxStageBytes && h.d_model % 8 == 0;
   p.smem_bytes = p.staged ? stage : 0;
+  // the group's CTAs add their partial sums in a cluster's shared memory when
+  // they run beside the decode (a few sequences); with more sequences the
+  // decode fills the SMs and clusters wait for whole free groups of SMs, so the
+  // partial sums go through global memory (measured: slower by 6-7 us per layer
+  // at batch 16 with clusters of 8 or 16)
+  p.cluster = T < 4 && p.n_part > 1 && p.n_part <= 8;
   return p;
 }
 
@@ -644,6 +664,15 @@ cudaError_t launch_fused_tp(const EncodeFusedPlan& p, const EncodeFusedArgs& arg
     if (p.smem_bytes > 0) {
       const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), p.smem_bytes);
       if (e != cudaSuccess) return e;
+    }
+    if (p.cluster) {
+      // the group's CTAs as one cluster (at most 8: a portable size); if the
+      // launch is refused, the partial sums go through global memory
+      EncodeFusedArgs ca = args;
+      ca.cluster = 1;
+      if (launch_dependent_cluster(kern, grid, block, p.smem_bytes, st, dim3(1, p.n_part, 1), ca, H, T, seq_ids,
+                                   cache, latents_out, counters, part, p.n_chunks, p.cpc) == cudaSuccess)
+        return cudaSuccess;
     }
     return launch_dependent(kern, grid, block, p.smem_bytes, st, args, H, T, seq_ids, cache, latents_out, counters,
                             part, p.n_chunks, p.cpc);
@@ -687,6 +716,7 @@ cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint
   args.n_eff = h.n_eff;
   args.P = h.P;
   args.staged = p.staged;
+  args.cluster = 0;
   if (h.group == 16) return launch_fused_g<16>(p, args, H, T, seq_ids, cache, latents_out, counters, part, st);
   return launch_fused_g<8>(p, args, H, T, seq_ids, cache, latents_out, counters, part, st);
 }

@@ -32,6 +32,34 @@ cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, int s
   return cudaGetLastError();
 }
 
+// As launch_dependent, in thread-block clusters of `cluster` CTAs; returns the
+// launch error (the caller falls back to a launch without clusters).
+template <typename... Args>
+cudaError_t launch_dependent_cluster(void (*kern)(Args...), dim3 grid, dim3 block, int smem, cudaStream_t st,
+                                     dim3 cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster.x;
+  attr[0].val.clusterDim.y = cluster.y;
+  attr[0].val.clusterDim.z = cluster.z;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e == cudaSuccess) return e;
+  (void)cudaGetLastError();
+  cfg.numAttrs = 1;  // without programmatic serialisation
+  e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) (void)cudaGetLastError();
+  return e;
+}
+
 // encode_kernels.cu
 cudaError_t launch_project_gemv(const CodecDev& h, const uint16_t* wt, const uint16_t* H, int T,
                                 float* C, int64_t ldc, cudaStream_t st);
@@ -51,6 +79,7 @@ constexpr int kFusedMaxT = 16;
 struct EncodeFusedPlan {
   int n_groups, n_chunks, batch, cpc, n_part, tp;
   int staged, smem_bytes;  // chunks after a CTA's first staged in shared memory (bytes per CTA)
+  int cluster;             // the n_part CTAs of a group form one thread-block cluster
 };
 constexpr int kMaxFusedGroups = kMaxKV * 2 * kMaxGroups;
 // What the fused encode reads of the codec, passed by value so that its first
@@ -62,7 +91,8 @@ struct EncodeFusedArgs {
   int64_t page_bytes;
   unsigned long long wait_ns;  // limit of the wait for staged W_down copies
   int d_model, n_eff, P;
-  int staged;  // chunks after a CTA's first are bulk-copied into shared memory
+  int staged;   // chunks after a CTA's first are bulk-copied into shared memory
+  int cluster;  // the CTAs of a group form one cluster and add their partial sums in shared memory
 };
 EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T);
 // Workspace bytes of the fused encode's partial sums for T tokens.

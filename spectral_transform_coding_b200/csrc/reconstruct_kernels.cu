@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(128) reconstruct_kernel(const CodecDev* __rest
 // A combine kernel merges the splits and applies W_up^V.
 // ---------------------------------------------------------------------------
 constexpr int kRtTokens = 32;
-constexpr int kRtPairsPerWarp = 2;  // (16-token, 8-dim pair) MMA tiles per warp and tile: d_h <= 128
+constexpr int kRtPairsPerWarp = 2;  // m-tiles (16 tokens) per warp and tile for its 8-dim pair: d_h <= 128
 constexpr int kRtThreads = 256;
 constexpr int kRtMaxSplit = 64;
 constexpr int kRtAccSlots = kMaxGQ * kRtMaxDHead / kRtThreads;  // V accumulators per thread
@@ -162,7 +162,7 @@ constexpr int kRtAccSlots = kMaxGQ * kRtMaxDHead / kRtThreads;  // V accumulator
 // Byte offsets of the split kernel's shared-memory regions (max_k, max_v:
 // largest kept coordinates per side over the heads; G: group size).
 struct RtSmem {
-  int om, bf, ws, ck, sz, cv, kh, qs, sc, ml, pg, total;
+  int om, bf, ws, ck, sz, cv, kh, qs, sc, ml, rb, pg, total;
   int ck_stride, n_grp;  // halves per K code row; groups per side (max)
   __host__ __device__ RtSmem(int d_h, int max_k, int max_v, int gq, int G) {
     ck_stride = max_k + 8;
@@ -192,6 +192,8 @@ struct RtSmem {
     ml = o;  // running max, sum and correction per q head
     o += 3 * kMaxGQ * 4;
     o = (o + 15) / 16 * 16;
+    rb = o;  // rotation of the tile's first position: {cos, sin} [d_h / 2]
+    o += kRtMaxDHead / 2 * 8;
     pg = o;  // byte offset of each tile token's page in the pool (-1: bad page id)
     o += kRtTokens * 8;
     total = o;
@@ -213,17 +215,29 @@ struct RtArgs {
   float* part;
 };
 
-// Turns (x, y) by `turns` * pi radians.  The angle, in half-turns, is reduced
-// to [-1, 1] in double (turns - 2 rint(turns / 2), exact up to the rounding of
+// cos and sin of `turns` * pi radians.  The angle, in half-turns, is reduced to
+// [-1, 1] in double (turns - 2 rint(turns / 2), exact up to the rounding of
 // `turns` itself), then sin(pi r) and cos(pi r) run in fp32.
-__device__ __forceinline__ void rope_rotate(float& x, float& y, double turns) {
+__device__ __forceinline__ float2 rope_cos_sin(double turns) {
   const double k = rint(turns * 0.5);
   const float r = (float)fma(-2.0, k, turns);
   float sn, cs;
   sincospif(r, &sn, &cs);
-  const float x2 = x * cs - y * sn, y2 = y * cs + x * sn;
+  return make_float2(cs, sn);
+}
+
+// Turns (x, y) by the angle whose {cos, sin} is cs.
+__device__ __forceinline__ void rope_apply(float& x, float& y, float2 cs) {
+  const float x2 = x * cs.x - y * cs.y, y2 = y * cs.x + x * cs.y;
   x = x2;
   y = y2;
+}
+
+__device__ __forceinline__ void rope_rotate(float& x, float& y, double turns) { rope_apply(x, y, rope_cos_sin(turns)); }
+
+// The rotation of the sum of two angles from their {cos, sin}.
+__device__ __forceinline__ float2 rope_add(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
 }
 
 // The G codes of one token in one group of width b (warp-uniform); G and the
@@ -287,6 +301,7 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   float* qs = reinterpret_cast<float*>(sm + L.qs);
   float* sc = reinterpret_cast<float*>(sm + L.sc);
   float* ml = reinterpret_cast<float*>(sm + L.ml);  // [0, 8) max, [8, 16) sum, [16, 24) correction
+  float2* rb = reinterpret_cast<float2*>(sm + L.rb);
   int64_t* pg = reinterpret_cast<int64_t*>(sm + L.pg);
   const bool rot = A.theta > 0.0;
 
@@ -339,6 +354,30 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   const int tok_end = min(min((split + 1) * per, tiles) * kRtTokens, len);
   const int n_items = kRtTokens * (ngK + sv.n_groups);
   const int n_acc = gq * nkV;
+  // The key rotation at position t0 + t is the tile's rotation at t0 (rb, per
+  // tile) followed by the rotation at offset t; this thread's (offset, dim)
+  // entries of the lift are the same in every tile, so their offset rotations
+  // are computed once, here
+  float2 roff[kRtPairsPerWarp][4];
+  // lift work of this warp: the n-tile pair np (dims 8 np.. and their rotation
+  // partners) for the m-tiles mt = q + mi * step (warps that share an np split
+  // the m-tiles), so that each B fragment is read once per tile
+  const int lift_np = warp % half_nt, lift_q = warp / half_nt, lift_step = max(1, 8 / half_nt);
+  const bool lift_on = lift_q < lift_step;
+  {
+    const int gid = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int mi = 0; mi < kRtPairsPerWarp; ++mi) {
+      const int mt = lift_q + mi * lift_step;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = mt * 16 + gid + (r < 2 ? 0 : 8), d = 8 * lift_np + 2 * t4 + (r & 1);
+        roff[mi][r] = (rot && lift_on && mt < kRtTokens / 16) ? rope_cos_sin((double)t * om[d])
+                                                               : make_float2(1.f, 0.f);
+      }
+    }
+  }
+
   float acc[kRtAccSlots];
 #pragma unroll
   for (int k = 0; k < kRtAccSlots; ++k) acc[k] = 0.f;
@@ -357,6 +396,8 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
       }
       pg[tid] = off;
     }
+    if (rot)
+      for (int i = tid; i < half; i += kRtThreads) rb[i] = rope_cos_sin((double)t0 * om[i]);
     __syncthreads();
     for (int e = tid; e < n_items; e += kRtThreads) {
       const int t = e % kRtTokens, jj = e / kRtTokens;
@@ -400,80 +441,106 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
       constexpr int kMT = kRtTokens / 16;
       float acc[kRtPairsPerWarp][2][4];
 #pragma unroll
-      for (int w = 0; w < kRtPairsPerWarp; ++w)
+      for (int mi = 0; mi < kRtPairsPerWarp; ++mi)
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-          for (int r = 0; r < 4; ++r) acc[w][h2][r] = 0.f;
+          for (int r = 0; r < 4; ++r) acc[mi][h2][r] = 0.f;
+      const int np = lift_np;
+      if (lift_on) {  // warp-uniform
+        for (int j = 0; j < ngK; ++j) {
+          // B fragments (hi, lo) and column sums of the pair's two n-tiles
+          uint32_t bh[2][2], bl[2][2];
+          float w0[2], w1[2];
 #pragma unroll
-      for (int w = 0; w < kRtPairsPerWarp; ++w) {
-        const int pp = warp + w * (kRtThreads / 32);
-        if (pp < kMT * half_nt) {  // warp-uniform
-          const int mt = pp % kMT, np = pp / kMT;
-          const int r0 = mt * 16 + gid, r1 = r0 + 8;
-          for (int j = 0; j < ngK; ++j) {
-            const __half* a0p = ck + r0 * cks + j * G + 2 * t4;
-            const __half* a1p = ck + r1 * cks + j * G + 2 * t4;
-            uint32_t af[4];
-            af[0] = *reinterpret_cast<const uint32_t*>(a0p);
-            af[1] = *reinterpret_cast<const uint32_t*>(a1p);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int ntl = np + h2 * half_nt;
+            const uint32_t* bp = bf + (j * n_nt + ntl) * 2 * KQ * 32 + lane;
             if (G == 16) {
-              af[2] = *reinterpret_cast<const uint32_t*>(a0p + 8);
-              af[3] = *reinterpret_cast<const uint32_t*>(a1p + 8);
+              bh[h2][0] = bp[0];
+              bh[h2][1] = bp[32];
+              bl[h2][0] = bp[64];
+              bl[h2][1] = bp[96];
+            } else {
+              bh[h2][0] = bp[0];
+              bl[h2][0] = bp[32];
+              bh[h2][1] = bl[h2][1] = 0u;
             }
-            const float s0 = szk[r0 * ngs + j], s1 = szk[r1 * ngs + j];
-            const float z0 = szk[(kRtTokens + r0) * ngs + j], z1 = szk[(kRtTokens + r1) * ngs + j];
+            w0[h2] = wsum[j * d_h + 8 * ntl + 2 * t4];
+            w1[h2] = wsum[j * d_h + 8 * ntl + 2 * t4 + 1];
+          }
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int ntl = np + h2 * half_nt;
-              const uint32_t* bp = bf + (j * n_nt + ntl) * 2 * KQ * 32 + lane;
-              float pr[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int mi = 0; mi < kRtPairsPerWarp; ++mi) {
+            const int mt = lift_q + mi * lift_step;
+            if (mt < kMT) {  // warp-uniform
+              const int r0 = mt * 16 + gid, r1 = r0 + 8;
+              const __half* a0p = ck + r0 * cks + j * G + 2 * t4;
+              const __half* a1p = ck + r1 * cks + j * G + 2 * t4;
+              uint32_t af[4];
+              af[0] = *reinterpret_cast<const uint32_t*>(a0p);
+              af[1] = *reinterpret_cast<const uint32_t*>(a1p);
               if (G == 16) {
-                const uint32_t bh[2] = {bp[0], bp[32]}, bl[2] = {bp[64], bp[96]};
-                mma_m16n8k16(pr, af, bh);
-                mma_m16n8k16(pr, af, bl);
-              } else {
-                mma_m16n8k8(pr, af, bp[0]);
-                mma_m16n8k8(pr, af, bp[32]);
+                af[2] = *reinterpret_cast<const uint32_t*>(a0p + 8);
+                af[3] = *reinterpret_cast<const uint32_t*>(a1p + 8);
               }
-              const float w0 = wsum[j * d_h + 8 * ntl + 2 * t4], w1 = wsum[j * d_h + 8 * ntl + 2 * t4 + 1];
-              acc[w][h2][0] = fmaf(s0, pr[0], fmaf(z0, w0, acc[w][h2][0]));
-              acc[w][h2][1] = fmaf(s0, pr[1], fmaf(z0, w1, acc[w][h2][1]));
-              acc[w][h2][2] = fmaf(s1, pr[2], fmaf(z1, w0, acc[w][h2][2]));
-              acc[w][h2][3] = fmaf(s1, pr[3], fmaf(z1, w1, acc[w][h2][3]));
+              const float s0 = szk[r0 * ngs + j], s1 = szk[r1 * ngs + j];
+              const float z0 = szk[(kRtTokens + r0) * ngs + j], z1 = szk[(kRtTokens + r1) * ngs + j];
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                float pr[4] = {0.f, 0.f, 0.f, 0.f};
+                if (G == 16) {
+                  mma_m16n8k16(pr, af, bh[h2]);
+                  mma_m16n8k16(pr, af, bl[h2]);
+                } else {
+                  mma_m16n8k8(pr, af, bh[h2][0]);
+                  mma_m16n8k8(pr, af, bl[h2][0]);
+                }
+                acc[mi][h2][0] = fmaf(s0, pr[0], fmaf(z0, w0[h2], acc[mi][h2][0]));
+                acc[mi][h2][1] = fmaf(s0, pr[1], fmaf(z0, w1[h2], acc[mi][h2][1]));
+                acc[mi][h2][2] = fmaf(s1, pr[2], fmaf(z1, w0[h2], acc[mi][h2][2]));
+                acc[mi][h2][3] = fmaf(s1, pr[3], fmaf(z1, w1[h2], acc[mi][h2][3]));
+              }
             }
           }
         }
       }
       __syncthreads();  // the codes are consumed: their bytes now take the keys
       // rows r0 / r1, dims d (n-tile np) and d + d_h/2 (n-tile np + half_nt)
+      if (lift_on) {
 #pragma unroll
-      for (int w = 0; w < kRtPairsPerWarp; ++w) {
-        const int pp = warp + w * (kRtThreads / 32);
-        if (pp < kMT * half_nt) {
-          const int mt = pp % kMT, np = pp / kMT;
-          const int r0 = mt * 16 + gid, r1 = r0 + 8;
+        for (int mi = 0; mi < kRtPairsPerWarp; ++mi) {
+          const int mt = lift_q + mi * lift_step;
+          if (mt < kMT) {
+            const int r0 = mt * 16 + gid, r1 = r0 + 8;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int t = r < 2 ? r0 : r1, d = 8 * np + 2 * t4 + (r & 1);
-            float x = acc[w][0][r], y = acc[w][1][r];
-            if (rot) rope_rotate(x, y, (double)(t0 + t) * om[d]);
-            kh[t * (d_h + 1) + d] = x;
-            kh[t * (d_h + 1) + half + d] = y;
+            for (int r = 0; r < 4; ++r) {
+              const int t = r < 2 ? r0 : r1, d = 8 * np + 2 * t4 + (r & 1);
+              float x = acc[mi][0][r], y = acc[mi][1][r];
+              if (rot) rope_apply(x, y, rope_add(rb[d], roff[mi][r]));
+              kh[t * (d_h + 1) + d] = x;
+              kh[t * (d_h + 1) + half + d] = y;
+            }
           }
         }
       }
     }
     __syncthreads();
     // ---- 3. scores (log2 units), online softmax, V latent sums --------------
-    for (int e = tid; e < gq * kRtTokens; e += kRtThreads) {
+    // two threads per (q head, token), each over half of the dims; the second
+    // half is walked from a quarter in, so that the pair's rows fall in
+    // different banks
+    for (int e2 = tid; e2 < 2 * gq * kRtTokens; e2 += kRtThreads) {  // kRtThreads even: pairs stay in a warp
+      const int e = e2 >> 1, part = e2 & 1;
       const int h = e / kRtTokens, t = e % kRtTokens;
-      float v = -INFINITY;
+      float v = 0.f;
       if (t < nt) {
-        const float* qr = qs + h * d_h;
-        const float* kr = kh + t * (d_h + 1);
+        const float* qr = qs + h * d_h + part * half;
+        const float* kr = kh + t * (d_h + 1) + part * half;
+        const int q4 = part ? (half / 4) & ~3 : 0;  // a multiple of 4, as half is
         float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
-        for (int d = 0; d < d_h; d += 4) {
+        for (int i = 0; i < half; i += 4) {
+          int d = i + q4;
+          d = d >= half ? d - half : d;  // d..d+3 stay within the half
           v0 = fmaf(qr[d], kr[d], v0);
           v1 = fmaf(qr[d + 1], kr[d + 1], v1);
           v2 = fmaf(qr[d + 2], kr[d + 2], v2);
@@ -481,7 +548,8 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
         }
         v = (v0 + v1) + (v2 + v3);
       }
-      sc[h * kRtTokens + t] = v;
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      if (part == 0) sc[h * kRtTokens + t] = t < nt ? v : -INFINITY;
     }
     __syncthreads();
     if (warp < gq) {
