@@ -162,9 +162,10 @@ constexpr int kRtAccSlots = kMaxGQ * kRtMaxDHead / kRtThreads;  // V accumulator
 // Byte offsets of the split kernel's shared-memory regions (max_k, max_v:
 // largest kept coordinates per side over the heads; G: group size).
 struct RtSmem {
-  int om, bf, ws, ck, sz, cv, kh, qs, sc, ml, rb, pg, total;
+  int om, bf, ws, ck, sz, cv, kh, qs, sc, ml, rb, pg, gt, rw, total;
   int ck_stride, n_grp;  // halves per K code row; groups per side (max)
-  __host__ __device__ RtSmem(int d_h, int max_k, int max_v, int gq, int G) {
+  // raw_bytes: bytes of one tile's slice of a page's head section
+  __host__ __device__ RtSmem(int d_h, int max_k, int max_v, int gq, int G, int raw_bytes) {
     ck_stride = max_k + 8;
     n_grp = max_k / G > 0 ? max_k / G : 1;
     int o = 0;
@@ -194,8 +195,12 @@ struct RtSmem {
     o = (o + 15) / 16 * 16;
     rb = o;  // rotation of the tile's first position: {cos, sin} [d_h / 2]
     o += kRtMaxDHead / 2 * 8;
-    pg = o;  // byte offset of each tile token's page in the pool (-1: bad page id)
-    o += kRtTokens * 8;
+    pg = o;  // byte offset of the current and the next tile's page in the pool (-1: bad page id)
+    o += 16;
+    gt = o;  // per kept group {plane_off, sz_off, width, offset in rw}: at most 32 over both sides
+    o += kMaxGroups * 16;
+    rw = o;  // the tile's codes and records, per kept group
+    o += (raw_bytes + 15) / 16 * 16;
     total = o;
   }
 };
@@ -240,39 +245,44 @@ __device__ __forceinline__ float2 rope_add(float2 a, float2 b) {
   return make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
 }
 
-// The G codes of one token in one group of width b (warp-uniform); G and the
-// side are compile-time, so the fragment positions fold to constants and the
-// word loads of all G codes issue together.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The G codes of one token in one group of width b (warp-uniform) from its
+// block staged in shared memory; G and the side are compile-time, so the
+// fragment positions fold to constants and the word loads issue together.
 template <int G, int SIDE>
-__device__ __forceinline__ void unpack_token(const uint32_t* __restrict__ blk, int b, int tb, uint32_t (&code)[G]) {
+__device__ __forceinline__ void unpack_token(const uint32_t* blk, int b, int tb, uint32_t (&code)[G]) {
   int gid[G], t4[G], slot[G];
 #pragma unroll
   for (int k = 0; k < G; ++k) frag_pos(G, SIDE, tb, k, &gid[k], &t4[k], &slot[k]);
   switch (b) {
     case 4:
 #pragma unroll
-      for (int k = 0; k < G; ++k) code[k] = (__ldg(blk + 4 * gid[k] + t4[k]) >> (4 * slot[k])) & 0xFu;
+      for (int k = 0; k < G; ++k) code[k] = (blk[4 * gid[k] + t4[k]] >> (4 * slot[k])) & 0xFu;
       break;
     case 2:
 #pragma unroll
-      for (int k = 0; k < G; ++k)
-        code[k] = (__ldg(blk + 2 * gid[k] + (t4[k] >> 1)) >> (4 * slot[k] + 2 * (t4[k] & 1))) & 0x3u;
+      for (int k = 0; k < G; ++k) code[k] = (blk[2 * gid[k] + (t4[k] >> 1)] >> (4 * slot[k] + 2 * (t4[k] & 1))) & 0x3u;
       break;
     case 1:
 #pragma unroll
-      for (int k = 0; k < G; ++k) code[k] = (__ldg(blk + gid[k]) >> (4 * slot[k] + t4[k])) & 0x1u;
+      for (int k = 0; k < G; ++k) code[k] = (blk[gid[k]] >> (4 * slot[k] + t4[k])) & 0x1u;
       break;
     case 3:
 #pragma unroll
       for (int k = 0; k < G; ++k)
-        code[k] = ((__ldg(blk + 2 * gid[k] + (t4[k] >> 1)) >> (4 * slot[k] + 2 * (t4[k] & 1))) & 0x3u) |
-                  (((__ldg(blk + 16 + gid[k]) >> (4 * slot[k] + t4[k])) & 0x1u) << 2);
+        code[k] = ((blk[2 * gid[k] + (t4[k] >> 1)] >> (4 * slot[k] + 2 * (t4[k] & 1))) & 0x3u) |
+                  (((blk[16 + gid[k]] >> (4 * slot[k] + t4[k])) & 0x1u) << 2);
       break;
     default:
 #pragma unroll
       for (int k = 0; k < G; ++k)
-        code[k] = (__ldg(blk + 2 * (4 * gid[k] + t4[k]) + ((slot[k] >> 1) & 1)) >>
-                   (8 * ((slot[k] & 1) + 2 * (slot[k] >> 2)))) & 0xFFu;
+        code[k] = (blk[2 * (4 * gid[k] + t4[k]) + ((slot[k] >> 1) & 1)] >> (8 * ((slot[k] & 1) + 2 * (slot[k] >> 2)))) &
+                  0xFFu;
       break;
   }
 }
@@ -288,7 +298,10 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   const SideDev& sk = cd->head[a].side[0];
   const SideDev& sv = cd->head[a].side[1];
   const int nkK = sk.n_kept, nkV = sv.n_kept, cvs = cd->max_kept_v + 1;
-  const RtSmem L(d_h, cd->max_kept_k, cd->max_kept_v, gq, G);
+  // P is a multiple of the tile (the codec requires a multiple of 32), so a
+  // tile never straddles a page: each tile's slice of the head section is
+  // staged in shared memory by async copies issued one tile ahead
+  const RtSmem L(d_h, cd->max_kept_k, cd->max_kept_v, gq, G, cd->max_sec_bytes / P * kRtTokens);
   const int cks = L.ck_stride, ngs = L.n_grp, n_nt = d_h / 8, half_nt = n_nt / 2;
   constexpr int KQ = G / 8;  // B fragment registers per lane (m16n8k16: 2, m16n8k8: 1)
   double* om = reinterpret_cast<double*>(sm + L.om);
@@ -303,6 +316,8 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   float* ml = reinterpret_cast<float*>(sm + L.ml);  // [0, 8) max, [8, 16) sum, [16, 24) correction
   float2* rb = reinterpret_cast<float2*>(sm + L.rb);
   int64_t* pg = reinterpret_cast<int64_t*>(sm + L.pg);
+  int4* gt = reinterpret_cast<int4*>(sm + L.gt);
+  uint8_t* rw = sm + L.rw;
   const bool rot = A.theta > 0.0;
 
   // W_up^K (stored transposed, W[c][d] = wk[d * n_kept + c]) as B fragments of
@@ -331,6 +346,21 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
   if (tid < kMaxGQ) {
     ml[tid] = -INFINITY;
     ml[kMaxGQ + tid] = 0.f;
+  }
+  const int ngAll = sk.n_groups + sv.n_groups;
+  if (warp == 1) {
+    // per kept group (K then V): page offsets, width and its slot in rw (the
+    // tile's 4 G b code bytes, then 8 record pieces of 16 bytes)
+    int acc_off = 0, mine = 0;
+    for (int jj = 0; jj < ngAll; ++jj) {
+      const int bw = (jj < sk.n_groups ? sk.grp[jj] : sv.grp[jj - sk.n_groups]).b;
+      if (jj == lane) mine = acc_off;
+      acc_off += 4 * G * bw + 128;
+    }
+    if (lane < ngAll) {
+      const GroupDev gd = lane < sk.n_groups ? sk.grp[lane] : sv.grp[lane - sk.n_groups];
+      gt[lane] = make_int4(gd.plane_off, gd.sz_off, gd.b, mine);
+    }
   }
   int len = A.lengths[b];
   if (len < 0 || (int64_t)len > (int64_t)A.max_pages * P) {
@@ -382,59 +412,86 @@ __global__ void __launch_bounds__(kRtThreads) rt_split_kernel(const RtArgs A) {
 #pragma unroll
   for (int k = 0; k < kRtAccSlots; ++k) acc[k] = 0.f;
 
+  // staged tiles: byte offset of the tile's page in the pool (-1: bad page id),
+  // read by thread 0 one tile ahead; the copies of a tile go out while the
+  // previous tile is lifted, scored and summed
+  auto tile_page = [&](int t0n) -> int64_t {
+    const int pid = A.page_table[(size_t)b * A.max_pages + t0n / P];
+    if (pid < 0 || (int64_t)pid >= A.n_pool_pages) {
+      device_error(cd->err, SPECTRA_ERR_INVALID);
+      return -1;
+    }
+    return (int64_t)pid * cd->page_bytes;
+  };
+  auto issue_tile = [&](int t0n, int64_t poff) {
+    if (poff >= 0) {
+      const int tau0 = t0n % P;
+      const uint8_t* page = A.pool + poff;
+      for (int jj = warp; jj < ngAll; jj += kRtThreads / 32) {
+        const int4 g = gt[jj];  // {plane_off, sz_off, width, slot}
+        uint8_t* dst = rw + g.w;
+        const int ncode = G * g.z / 4;  // 16-byte pieces of the tile's codes (<= 32)
+        if (lane < ncode) cp_async16(dst + 16 * lane, page + g.x + (size_t)(tau0 / TB) * 32 * g.z + 16 * lane);
+        // records of pairs tau0/2 .. tau0/2 + 15: two per row (u % 8) of the record grid
+        if (lane < 8) cp_async16(dst + 4 * G * g.z + 16 * lane, page + g.y + 8 * (lane * (P >> 4) + tau0 / 16));
+      }
+    }
+    cp_async_commit();
+  };
+  __syncthreads();  // the group table is complete
+  if (tid == 0) pg[0] = tok_begin < tok_end ? tile_page(tok_begin) : -1;
+  __syncthreads();
+  if (tok_begin < tok_end) issue_tile(tok_begin, pg[0]);
+
   for (int t0 = tok_begin; t0 < tok_end; t0 += kRtTokens) {
     const int nt = min(kRtTokens, tok_end - t0);
     // ---- 1. dequantised latents of the tile (rows past the end are zero) ----
-    if (tid < kRtTokens) {
-      int64_t off = -1;
-      if (tid < nt) {
-        const int pid = A.page_table[(size_t)b * A.max_pages + (t0 + tid) / P];
-        if (pid < 0 || (int64_t)pid >= A.n_pool_pages)
-          device_error(cd->err, SPECTRA_ERR_INVALID);
-        else
-          off = (int64_t)pid * cd->page_bytes;
+    {
+      const int64_t cur = pg[0];
+      cp_async_wait_all();
+      if (rot)
+        for (int i = tid; i < half; i += kRtThreads) rb[i] = rope_cos_sin((double)t0 * om[i]);
+      if (tid == 0 && t0 + kRtTokens < tok_end) pg[1] = tile_page(t0 + kRtTokens);
+      __syncthreads();  // the tile's bytes have landed (every thread's copies)
+      for (int e = tid; e < n_items; e += kRtThreads) {
+        const int t = e % kRtTokens, jj = e / kRtTokens;
+        const int side = jj < ngK ? 0 : 1, j = side ? jj - ngK : jj;
+        uint32_t code[G];
+        float sv_ = 0.f, zv = 0.f;
+        if (cur < 0 || t >= nt) {
+#pragma unroll
+          for (int k = 0; k < G; ++k) code[k] = 0u;
+        } else {
+          const int4 g = gt[jj];
+          const uint8_t* slot = rw + g.w;
+          const int ul = t >> 1;
+          const uint2 rec = *reinterpret_cast<const uint2*>(slot + 4 * G * g.z + 16 * (ul & 7) + 8 * (ul >> 3));
+          sv_ = (t & 1) ? half_hi(rec.x) : half_lo(rec.x);
+          zv = (t & 1) ? half_hi(rec.y) : half_lo(rec.y);
+          const uint32_t* blk = reinterpret_cast<const uint32_t*>(slot + (t / TB) * 32 * g.z);
+          if (side == 0)
+            unpack_token<G, 0>(blk, g.z, t % TB, code);
+          else
+            unpack_token<G, 1>(blk, g.z, t % TB, code);
+        }
+        if (side == 0) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(ck + t * cks + j * G);
+#pragma unroll
+          for (int k = 0; k < G; k += 2) dst[k / 2] = pack_half2((float)code[k], (float)code[k + 1]);
+          szk[t * ngs + j] = sv_;
+          szk[(kRtTokens + t) * ngs + j] = zv;
+        } else {
+          float* dst = cV + t * cvs + j * G;
+#pragma unroll
+          for (int k = 0; k < G; ++k) dst[k] = fmaf((float)code[k], sv_, zv);
+        }
       }
-      pg[tid] = off;
-    }
-    if (rot)
-      for (int i = tid; i < half; i += kRtThreads) rb[i] = rope_cos_sin((double)t0 * om[i]);
-    __syncthreads();
-    for (int e = tid; e < n_items; e += kRtThreads) {
-      const int t = e % kRtTokens, jj = e / kRtTokens;
-      const int side = jj < ngK ? 0 : 1, j = side ? jj - ngK : jj;
-      const GroupDev gd = (side ? sv : sk).grp[j];
-      const int64_t off = pg[t];
-      uint32_t code[G];
-      float sv_ = 0.f, zv = 0.f;
-      if (off < 0) {
-#pragma unroll
-        for (int k = 0; k < G; ++k) code[k] = 0u;
-      } else {
-        const uint8_t* page = A.pool + off;
-        const int tau = (t0 + t) % P, u = tau >> 1;
-        const uint32_t* blk = reinterpret_cast<const uint32_t*>(page + gd.plane_off + (tau / TB) * (32 * gd.b));
-        const uint2 rec =
-            __ldg(reinterpret_cast<const uint2*>(page + gd.sz_off + 8 * ((u & 7) * (P >> 4) + (u >> 3))));
-        sv_ = (tau & 1) ? half_hi(rec.x) : half_lo(rec.x);  // {s[2u], s[2u+1]}
-        zv = (tau & 1) ? half_hi(rec.y) : half_lo(rec.y);   // {z[2u], z[2u+1]}
-        if (side == 0)
-          unpack_token<G, 0>(blk, gd.b, tau % TB, code);
-        else
-          unpack_token<G, 1>(blk, gd.b, tau % TB, code);
-      }
-      if (side == 0) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(ck + t * cks + j * G);
-#pragma unroll
-        for (int k = 0; k < G; k += 2) dst[k / 2] = pack_half2((float)code[k], (float)code[k + 1]);
-        szk[t * ngs + j] = sv_;
-        szk[(kRtTokens + t) * ngs + j] = zv;
-      } else {
-        float* dst = cV + t * cvs + j * G;
-#pragma unroll
-        for (int k = 0; k < G; ++k) dst[k] = fmaf((float)code[k], sv_, zv);
+      __syncthreads();  // rw is consumed: the next tile's copies may land in it
+      if (t0 + kRtTokens < tok_end) {
+        if (tid == 0) pg[0] = pg[1];
+        issue_tile(t0 + kRtTokens, pg[1]);
       }
     }
-    __syncthreads();
     // ---- 2. k^ = sum_j s_j (code_j W_j) + z_j (sum of W_j) on the tensor cores ----
     {
       const int gid = lane >> 2, t4 = lane & 3;
@@ -685,7 +742,7 @@ RtPlan make_rt_plan(const CodecDev& h, int batch, int max_pages_per_seq, bool up
   // split the context so that the (KV head, sequence) pairs fill the resident
   // CTA slots once (two CTAs per SM fit at d_h = 128: about 106 KB each; more
   // are not used, so that the bound below holds for any call)
-  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq, h.group).total;
+  p.smem_bytes = RtSmem(h.d_h, h.max_kept_k, h.max_kept_v, h.gq, h.group, h.max_sec_bytes / h.P * kRtTokens).total;
   const int pairs = h.n_kv * batch;
   const int per_sm = upper_bound ? 2 : std::min(2, rt_ctas_per_sm(h.group, p.smem_bytes));
   int ns = rt_sm_count() * per_sm / pairs;
