@@ -280,7 +280,13 @@ SPECTRA_API spectra_status spectra_quantize_append(const spectra_codec* codec, c
  * spectra_project's, so the pages equal those of spectra_project followed by
  * spectra_quantize_append.  Otherwise (16 < T < 64, or latents_out given) the
  * latents go through memory.  The same checks apply on every route and a
- * failure writes nothing. */
+ * failure writes nothing.  The decode-step encode stages W_down rows in shared
+ * memory behind a bounded wait (200 ms); if it gives up, the call records
+ * SPECTRA_ERR_TIMEOUT, the lengths may already have advanced and the step's
+ * codes are undefined.  Test hooks, read from the environment at every launch
+ * and meant for tests only: SPECTRA_ENCODE_TEST_DROP_STAGE (the first CTA never
+ * issues its first staged copy, so its wait gives up) and
+ * SPECTRA_ENCODE_TEST_WAIT_NS (the wait's limit). */
 SPECTRA_API spectra_status spectra_encode_append(const spectra_codec* codec, const spectra_cache* cache,
                                      const void* H, const int32_t* seq_ids, int64_t T,
                                      float* latents_out, void* workspace, size_t workspace_bytes,

@@ -4,6 +4,7 @@
 // "grouping").
 #include <cuda_bf16.h>
 #include <algorithm>
+#include <cstdlib>
 #include <cuda_fp16.h>
 
 #include "device_common.cuh"
@@ -245,16 +246,19 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(
 
 // ---------------------------------------------------------------------------
 // Fused small-batch encode (decode steps, T <= kFusedMaxT tokens).  The
-// projection of the step's tokens is split over CTAs (kept group, d_model chunk
-// of KCH columns of H): each CTA streams its group's G rows of W_down over its
-// chunk (all of its loads in flight before the dependency wait), multiplies
-// them with the tokens' H (read after the wait), reduces across the warp and
-// writes a partial sum per (token, column) to the workspace.  The last CTA of a
-// group to arrive (a counter per group) adds the chunks' partials in chunk
-// order, quantises and packs the group for the step's tokens.  The positions
-// are computed and validated by every such CTA the same way from the current
-// lengths, so a failed check writes nothing anywhere; the last group to finish
-// (a second counter) advances the lengths.  All counters are left at zero.
+// projection of the step's tokens is split over CTAs (kept group, consecutive
+// d_model chunks of KCH columns of H): each CTA has all of its group's G rows
+// of W_down over its chunks in flight before the dependency wait (the first
+// chunk in registers, later ones staged in shared memory by bulk copies),
+// multiplies them with the tokens' H (read after the wait) and reduces across
+// the warp.  A group split over several CTAs adds their partial sums in CTA
+// order: in rank 0's shared memory when the CTAs form a cluster, else through
+// the workspace and the group's last CTA to arrive (a counter per group).
+// That CTA quantises and packs the group for the step's tokens, one half warp
+// per token.  Every CTA computes and validates the positions the same way from
+// the current lengths, so a failed check writes nothing anywhere; the last CTA
+// to hold its positions (a second counter) advances the lengths at once.  All
+// counters are left at zero.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -354,9 +358,11 @@ __global__ void __launch_bounds__(256) encode_fused_kernel(const EncodeFusedArgs
     mbar_arrive_expect_tx(&w_bar, bytes);
     for (int ch = ch0 + 1; ch < ch1; ++ch) {
       const int len = min(KCH, d_model - ch * KCH);
-      for (int r = 0; r < G; ++r)
+      for (int r = 0; r < G; ++r) {
+        if (A.drop_stage && gi == 0 && blockIdx.y == 0 && ch == ch0 + 1 && r == 0) continue;  // test hook
         bulk_copy_g2s(w_s + ((size_t)(ch - ch0 - 1) * G + r) * (KCH * 2),
                       A.wt_down + (size_t)(gi * G + r) * d_model + (size_t)ch * KCH, (uint32_t)len * 2u, &w_bar);
+      }
     }
   }
   uint4 wv[CPW][BATCH];
@@ -711,7 +717,15 @@ cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint
   args.col_groups = h.col_groups;
   args.err = h.err;
   args.page_bytes = h.page_bytes;
-  args.wait_ns = kFusedWaitLimitNs;
+  // test hooks for the bounded wait on the staged copies:
+  // SPECTRA_ENCODE_TEST_DROP_STAGE makes the first CTA skip its first staged
+  // copy (its wait then gives up and the call reports SPECTRA_ERR_TIMEOUT), and
+  // SPECTRA_ENCODE_TEST_WAIT_NS shortens the wait's limit
+  const char* ds = std::getenv("SPECTRA_ENCODE_TEST_DROP_STAGE");
+  const char* wn = std::getenv("SPECTRA_ENCODE_TEST_WAIT_NS");
+  const long long wait = wn ? std::atoll(wn) : 0;
+  args.drop_stage = ds ? 1 : 0;
+  args.wait_ns = wait > 0 ? (unsigned long long)wait : kFusedWaitLimitNs;
   args.d_model = h.d_model;
   args.n_eff = h.n_eff;
   args.P = h.P;

@@ -70,8 +70,9 @@ cudaError_t launch_quantize_append(const CodecDev& h, const CodecDev* d, const f
                                    int T, const spectra_cache& cache, cudaStream_t st);
 
 // Fused encode for decode steps: projection (split over d_model chunks),
-// quantisation and packing in one kernel; the last chunk of a group to arrive
-// finishes the group and the last group advances the lengths.
+// quantisation and packing in one kernel; a group's partial sums meet in one
+// CTA, which packs the group; the last CTA to hold its positions advances the
+// lengths.
 constexpr int kFusedMaxT = 16;
 // Decode-step encode plan: kept groups; d_model chunks of 256 * batch columns,
 // cpc consecutive chunks per CTA, n_part CTAs per group; token count rounded up
@@ -91,8 +92,9 @@ struct EncodeFusedArgs {
   int64_t page_bytes;
   unsigned long long wait_ns;  // limit of the wait for staged W_down copies
   int d_model, n_eff, P;
-  int staged;   // chunks after a CTA's first are bulk-copied into shared memory
-  int cluster;  // the CTAs of a group form one cluster and add their partial sums in shared memory
+  int staged;      // chunks after a CTA's first are bulk-copied into shared memory
+  int cluster;     // the CTAs of a group form one cluster and add their partial sums in shared memory
+  int drop_stage;  // test hook: CTA (0, 0) never issues its first staged copy (its wait then gives up)
 };
 EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T);
 // Workspace bytes of the fused encode's partial sums for T tokens.

@@ -82,6 +82,45 @@ def test_fused_encode_full_width(d_model, n_q, n_kv, wk, wv, T):
     np.testing.assert_array_equal(c1.lengths.cpu().numpy(), start + np.bincount(seqs, minlength=B))
 
 
+def test_encode_staged_wait_gives_up_with_a_timeout_status(monkeypatch):
+    """A staged W_down copy that never lands (test hook SPECTRA_ENCODE_TEST_DROP_STAGE:
+    the first CTA skips its first staged copy) makes that CTA's bounded wait give
+    up after the limit (SPECTRA_ENCODE_TEST_WAIT_NS: 2 ms).  The call reports
+    SPECTRA_ERR_TIMEOUT through the device error word, every CTA still arrives,
+    and later calls on the same workspace write exactly what a fresh workspace
+    gives.  The Llama-shaped layer at one token stages the second half of each
+    group's W_down rows."""
+    torch = torch_mod()
+    import spectral_transform_coding_b200 as st
+    codec, _, _, _ = _codec(4096, 32, 8, LLAMA4X, LLAMA4X, seed=21)
+    B = 2
+    rng = np.random.default_rng(22)
+    H = torch.from_numpy(bf16_round(rng.standard_normal((1, 4096)).astype(np.float32))).to(dev()).to(torch.bfloat16)
+    seqs = torch.ones(1, dtype=torch.int32, device=dev())
+    table = torch.from_numpy(np.arange(B * 2, dtype=np.int32).reshape(B, 2))
+
+    def cache():
+        return st.LatentCache(codec, batch=B, max_pages_per_seq=2, device=dev(), page_table=table)
+
+    ws = torch.zeros(codec.encode_workspace_bytes(1), dtype=torch.uint8, device=dev())
+    monkeypatch.setenv("SPECTRA_ENCODE_TEST_DROP_STAGE", "1")
+    monkeypatch.setenv("SPECTRA_ENCODE_TEST_WAIT_NS", "2000000")
+    codec.encode_append(cache(), H, seqs, workspace=ws)
+    with pytest.raises(st.SpectraError) as e:
+        codec.device_status()
+    assert e.value.status == 6  # SPECTRA_ERR_TIMEOUT
+    monkeypatch.delenv("SPECTRA_ENCODE_TEST_DROP_STAGE")
+    monkeypatch.delenv("SPECTRA_ENCODE_TEST_WAIT_NS")
+    for _ in range(2):
+        c1, c2 = cache(), cache()
+        codec.encode_append(c1, H, seqs, workspace=ws)
+        codec.encode_append(c2, H, seqs, workspace=torch.zeros_like(ws))
+        codec.device_status()
+        assert torch.equal(c1.pool, c2.pool)
+        np.testing.assert_array_equal(c1.lengths.cpu().numpy(), [0, 1])
+        assert torch.equal(c1.lengths, c2.lengths)
+
+
 @pytest.mark.parametrize("n_kv", [4, 8])
 def test_projection_tcgen05_full_width(n_kv):
     """H W_down on the tcgen05 GEMM at K = 4096 (64 k-blocks) with N_eff = 128 n_kv
