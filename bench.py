@@ -79,10 +79,10 @@ def _workload_name(cfg, layers):
 #     169,200,128 B read + 4,024,064 B written for 167,787,520 packed bytes
 #   attend_kernel, Qwen 8x, 131,075 tokens: 34,037,504 B read, 0 written, for
 #     33,555,200 packed bytes
-#   rt_split_kernel, Llama-shaped, 32k context: 34,214,912 B read, 0 written,
-#     for 33,560,576 packed bytes
+#   rt_split_kernel (tiles staged by cp.async), Llama-shaped, 32k context:
+#     34,244,608 B read, 0 written, for 33,560,576 packed bytes
 TRAFFIC_PER_ALGO_BYTE = {"stress": (169_200_128 + 4_024_064) / 167_787_520, "qwen": 34_037_504 / 33_555_200}
-TRAFFIC_PER_PACKED_BYTE_RT = {"llama": 34_214_912 / 33_560_576}
+TRAFFIC_PER_PACKED_BYTE_RT = {"llama": 34_244_608 / 33_560_576}
 
 
 def _oracle_decode_case(cfg, n_tok=8192, rope_theta=None):
