@@ -194,36 +194,6 @@ DecodePlan make_decode_plan(const CodecDev& h, int batch, int max_pages_per_seq)
       best_ns = ns;
     }
   }
-  // A step of a few sequences runs the next layer's fused encode (one token per
-  // sequence) beside this decode: SMs that hold one decode CTA take its CTAs
-  // while the decode runs.  With S SMs, D decode CTAs (two fit an SM), E encode
-  // CTAs and e of them beside one decode CTA, all of them find room at once when
-  // (2S - D) e >= E; more splits up to that bound shorten each CTA's page list
-  // (measured: Qwen 8x, 4 units, step 48.4 us per layer at 37 splits, 43.2 at
-  // 56; Llama 4x, 8 units, 47.2 at 18 and 56.4 at 24, past its bound of 21).
-  if (one_per_sm && ctas_per_sm(kern, p.smem_bytes) >= 2) {
-    int e_regs = 0, e_smem = 0, e_ctas = 0;
-    cudaFuncAttributes da{};
-    int dev = 0, sm_regs = 0, sm_smem = 0;
-    cudaGetDevice(&dev);
-    if (encode_fused_footprint(h, batch, &e_regs, &e_smem, &e_ctas) &&
-        cudaFuncGetAttributes(&da, reinterpret_cast<const void*>(kern)) == cudaSuccess &&
-        cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess &&
-        e_regs > 0) {
-      const int d_regs = (da.numRegs + 7) / 8 * 8 * kThreads;
-      const int d_smem = (int)da.sharedSizeBytes + p.smem_bytes + 1024;  // 1 KB reserved per CTA
-      const int by_regs = (sm_regs - d_regs) / e_regs;
-      const int by_smem = (sm_smem - d_smem) / (e_smem + 1024);
-      const int e = std::min({by_regs, by_smem, (2048 - kThreads) / 256});
-      if (e >= 1) {
-        const long d_max = 2L * sm_count() - (e_ctas + e - 1) / e;
-        const int ns_max = (int)std::min<long>(kMaxSplit, d_max / units);
-        if (ns_max > best_ns) best_ns = ns_max;
-      }
-    }
-    (void)cudaGetLastError();
-  }
   p.n_split = best_ns;
   size_t off = 0;
   auto carve = [&](size_t bytes) {

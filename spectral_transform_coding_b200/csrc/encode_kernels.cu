@@ -705,44 +705,6 @@ cudaError_t launch_fused_g(const EncodeFusedPlan& p, const EncodeFusedArgs& d, c
 }
 }  // namespace
 
-namespace {
-template <int G, int TP>
-const void* fused_ptr_tp(int batch) {
-  switch (batch) {
-    case 8: return reinterpret_cast<const void*>(encode_fused_kernel<G, TP, 8>);
-    case 4: return reinterpret_cast<const void*>(encode_fused_kernel<G, TP, 4>);
-    case 2: return reinterpret_cast<const void*>(encode_fused_kernel<G, TP, 2>);
-    default: return reinterpret_cast<const void*>(encode_fused_kernel<G, TP, 1>);
-  }
-}
-template <int G>
-const void* fused_ptr_g(int tp, int batch) {
-  switch (tp) {
-    case 1: return fused_ptr_tp<G, 1>(batch);
-    case 2: return fused_ptr_tp<G, 2>(batch);
-    case 4: return fused_ptr_tp<G, 4>(batch);
-    case 8: return fused_ptr_tp<G, 8>(batch);
-    default: return fused_ptr_tp<G, 16>(batch);
-  }
-}
-}  // namespace
-
-bool encode_fused_footprint(const CodecDev& h, int T, int* regs, int* smem, int* ctas) {
-  if (T < 1 || T > kFusedMaxT) return false;
-  const EncodeFusedPlan p = encode_fused_plan(h, T);
-  if (p.n_groups == 0) return false;
-  const void* kern = h.group == 16 ? fused_ptr_g<16>(p.tp, p.batch) : fused_ptr_g<8>(p.tp, p.batch);
-  cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return false;
-  }
-  *regs = (fa.numRegs + 7) / 8 * 8 * 256;
-  *smem = (int)fa.sharedSizeBytes + p.smem_bytes;
-  *ctas = p.n_groups * p.n_part;
-  return true;
-}
-
 cudaError_t launch_encode_fused(const CodecDev& h, const CodecDev* d, const uint16_t* H, const int32_t* seq_ids,
                                 int T, const spectra_cache& cache, float* latents_out, int32_t* counters,
                                 float* part, cudaStream_t st) {

@@ -97,9 +97,6 @@ struct EncodeFusedArgs {
   int drop_stage;  // test hook: CTA (0, 0) never issues its first staged copy (its wait then gives up)
 };
 EncodeFusedPlan encode_fused_plan(const CodecDev& h, int T);
-// Registers (all threads) and shared memory of one CTA of the fused encode
-// that T tokens launch, and its CTA count; false when it launches none.
-bool encode_fused_footprint(const CodecDev& h, int T, int* regs, int* smem, int* ctas);
 // Workspace bytes of the fused encode's partial sums for T tokens.
 size_t encode_fused_partial_bytes(const CodecDev& h, int T);
 // counters: int32 [1 + kMaxFusedGroups], zero between calls; part: partial sums.
